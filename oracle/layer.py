@@ -1,0 +1,155 @@
+"""Triple-branch W4A4G4 linear layer and its MLP pair, forward and backward.
+
+TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
+
+Follows FourTune:
+  §3.1  y = (4-bit residual branch) + (frozen low-rank stabilizer) + (LoRA):
+        y = deq(Q(X)) deq(Q(R))^T + (X S_dn) S_up + (X A) B  (+ bias)
+  §3.2  backward: the gradient flows through all three branches; only the
+        adapter (A, B) receives parameter gradients -- no gradient for R, S or
+        bias.  The 4-bit branch uses Q(G) against the same blocks of Q(R) read
+        transposed: dX = deq(Q(G)) deq(Q(R)) in this file's orientation
+        (R is stored [N, K], so the pages' Q(G) Q(R)^T is the same product).
+  §3.3  LoRA fusion: all three branches share the same input (X forward, G
+        backward); MLP fusion: FC1 -> GELU -> FC2 quantization.
+
+Readings of what the pages leave open (each is also listed in the design notes):
+  * The low-rank branches take the full-precision bf16 input (X, G), not Q(X).
+  * The down-projections L = X [S_dn | A] and P = G [S_up ; B]^T are rounded to
+    bf16 (ties-to-even) once, after exact accumulation: they feed bf16 products.
+  * dA = X^T P[:, r_s:]   and   dB = L[:, r_s:]^T G   (straight-through: Q has
+    no derivative of its own).
+  * MLP: h = bf16(FC1(X) + b1) is the saved hidden; a = GELU_tanh(h);
+    FC2's 4-bit input is Q(a) of float32 a; its low-rank input is bf16(a).
+    Backward: d_a from FC2, d_h = d_a * GELU'(h); FC1's 4-bit gradient is
+    Q(d_h) of float32 d_h and its low-rank gradient input is bf16(d_h).
+
+All GEMMs run in float64 on the exactly dequantized operands; a library matmul
+is the only primitive used.
+"""
+import numpy as np
+
+from . import block16, formats
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def _D(S_dn, A):
+    return np.concatenate([_f64(S_dn), _f64(A)], axis=1)      # [K, r_s + r]
+
+
+def _U(S_up, B):
+    return np.concatenate([_f64(S_up), _f64(B)], axis=0)      # [r_s + r, N]
+
+
+def linear_fwd(X, R_codes, R_scales, S_dn, S_up, A, B, bias=None, Qx=None):
+    """Forward.  X [M, K] (bf16 values), R codes [N, K/2] / scales [N/16, K/16].
+
+    Returns dict(y [M, N] float64, L [M, r_s+r] bf16 values, qx_codes, qx_scales).
+    `Qx` may pass precomputed (codes, scales) of the 4-bit input (used for the
+    MLP's FC2 whose 4-bit input is Q(a) of a float32 a).
+    """
+    X = _f64(X)
+    if Qx is None:
+        Qx = block16.quantize(X.astype(np.float32))
+    qx_codes, qx_scales = Qx
+    Xq = block16.dequantize(qx_codes, qx_scales)
+    Rq = block16.dequantize(R_codes, R_scales)
+    L = formats.bf16_round(X @ _D(S_dn, A))
+    y = Xq @ Rq.T + L @ _U(S_up, B)
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return dict(y=y, L=L, qx_codes=qx_codes, qx_scales=qx_scales)
+
+
+def linear_bwd(G, X, L, R_codes, R_scales, S_dn, S_up, A, B, Qg=None):
+    """Backward.  G = dL/dy [M, N] (bf16 values), X [M, K] (bf16 values),
+    L [M, r_s+r] saved by the forward.
+
+    Returns dict(dX [M, K], dA [K, r], dB [r, N], P [M, r_s+r] bf16 values,
+    qg_codes, qg_scales).  `Qg` may pass a precomputed 4-bit gradient (MLP).
+    """
+    G = _f64(G)
+    X = _f64(X)
+    L = _f64(L)
+    r_s = np.asarray(S_dn).shape[1]
+    if Qg is None:
+        Qg = block16.quantize(G.astype(np.float32))
+    qg_codes, qg_scales = Qg
+    Gq = block16.dequantize(qg_codes, qg_scales)
+    Rq = block16.dequantize(R_codes, R_scales)
+    D = _D(S_dn, A)
+    U = _U(S_up, B)
+    P = formats.bf16_round(G @ U.T)
+    dX = Gq @ Rq + P @ D.T
+    dA = X.T @ P[:, r_s:]
+    dB = L[:, r_s:].T @ G
+    return dict(dX=dX, dA=dA, dB=dB, P=P, qg_codes=qg_codes, qg_scales=qg_scales)
+
+
+# ------------------------------------------------------------------------- MLP
+_GELU_C = np.sqrt(2.0 / np.pi)
+_GELU_K = 0.044715
+
+
+def gelu_tanh(h):
+    """GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3)))."""
+    h = _f64(h)
+    return 0.5 * h * (1.0 + np.tanh(_GELU_C * (h + _GELU_K * h ** 3)))
+
+
+def gelu_tanh_grad(h):
+    """d/dh of gelu_tanh, closed form."""
+    h = _f64(h)
+    t = np.tanh(_GELU_C * (h + _GELU_K * h ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * h * (1.0 - t * t) * _GELU_C * (1.0 + 3.0 * _GELU_K * h * h)
+
+
+def mlp_fwd(X, fc1, fc2, a_f32=None):
+    """FC1 -> GELU(tanh) -> FC2, both triple-branch layers.
+
+    fc1/fc2: dict(R_codes, R_scales, S_dn, S_up, A, B, bias).
+    `a_f32` optionally overrides the float32 activation that FC2 quantizes (the
+    GPU's own a, so that downstream results compare on identical operands).
+    Returns dict(y, h, a, L1, L2, qa_codes, qa_scales, ...).
+    """
+    o1 = linear_fwd(X, fc1["R_codes"], fc1["R_scales"], fc1["S_dn"], fc1["S_up"],
+                    fc1["A"], fc1["B"], fc1.get("bias"))
+    h = formats.bf16_round(o1["y"])
+    a = gelu_tanh(h)
+    a32 = a.astype(np.float32) if a_f32 is None else np.asarray(a_f32, dtype=np.float32)
+    a_bf = formats.bf16_round(a32.astype(np.float64))
+    Qa = block16.quantize(a32)
+    o2 = linear_fwd(a_bf, fc2["R_codes"], fc2["R_scales"], fc2["S_dn"], fc2["S_up"],
+                    fc2["A"], fc2["B"], fc2.get("bias"), Qx=Qa)
+    return dict(y=o2["y"], h=h, a=a, a32=a32, a_bf=a_bf, L1=o1["L"], L2=o2["L"],
+                qx_codes=o1["qx_codes"], qx_scales=o1["qx_scales"],
+                qa_codes=Qa[0], qa_scales=Qa[1])
+
+
+def mlp_bwd(G, X, h, L1, L2, fc1, fc2, dh_f32=None, a_bf=None):
+    """Backward of mlp_fwd.  G = dL/dy [M, N2].  h, L1, L2 as saved by the forward.
+
+    `dh_f32` optionally overrides the float32 d_h that FC1's backward quantizes.
+    `a_bf` optionally overrides FC2's low-rank input bf16(a) (else recomputed
+    from h as in the forward).
+    Returns dict(dX, dA1, dB1, dA2, dB2, d_a, d_h, ...).
+    """
+    h = _f64(h)
+    if a_bf is None:
+        a_bf = formats.bf16_round(gelu_tanh(h).astype(np.float32).astype(np.float64))
+    b2 = linear_bwd(G, a_bf, L2, fc2["R_codes"], fc2["R_scales"], fc2["S_dn"], fc2["S_up"],
+                    fc2["A"], fc2["B"])
+    d_a = b2["dX"]
+    d_h = d_a * gelu_tanh_grad(h)
+    dh32 = d_h.astype(np.float32) if dh_f32 is None else np.asarray(dh_f32, dtype=np.float32)
+    dh_bf = formats.bf16_round(dh32.astype(np.float64))
+    Qdh = block16.quantize(dh32)
+    b1 = linear_bwd(dh_bf, X, L1, fc1["R_codes"], fc1["R_scales"], fc1["S_dn"], fc1["S_up"],
+                    fc1["A"], fc1["B"], Qg=Qdh)
+    return dict(dX=b1["dX"], dA1=b1["dA"], dB1=b1["dB"], dA2=b2["dA"], dB2=b2["dB"],
+                d_a=d_a, d_h=d_h, dh32=dh32, P1=b1["P"], P2=b2["P"],
+                qdh_codes=Qdh[0], qdh_scales=Qdh[1], qg_codes=b2["qg_codes"],
+                qg_scales=b2["qg_scales"])
