@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark: FourTune W4A4G4 triple-branch linear, forward + backward, on B200.
+
+One step = fourtune_linear_fwd + fourtune_linear_bwd (every kernel of the hot
+path: pack, fused X pass, FP4 GEMM + up-projection, fused G pass, FP4 dX GEMM,
+dA, dB) on the FLUX-width layer: M = 4608 tokens, K = N = 3072, stabilizer
+rank 32, LoRA rank 32, seeded synthetic bf16 data (synth.py).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is device time from CUDA events summed
+over exactly K steps (L2 flushed by a 256 MB write before each step, outside
+the events), max over ranks; `e2e` repeats the steps through the same C ABI with
+inputs in pinned host memory (H2D of X and dY, D2H of dA and dB inside the
+timed region).  `--impl reference` times the CPU oracle on a bounded sample of
+the same workload.  With N > 1 (torchrun) every rank runs an independent
+replica: the layer has no data-path exchange.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "flux-linear-3072"
+METRIC = "W4A4G4 linear fwd+bwd TFLOPS & tokens/s on 1 B200; % of dense FP4 peak"
+FALLBACK = dict(hbm_gbs=6650.0, bf16_tflops=1590.0)
+FP4_PER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
+ORACLE_ROWS = 256           # rows of the workload per CPU-oracle sample
+
+
+def layer_work(M, K, N, r_s, r):
+    """FP4 GEMM FLOPs (forward + dX; no weight gradient) and bf16 low-rank FLOPs per step."""
+    R = r_s + r
+    fp4 = 4 * M * N * K
+    lowrank = 4 * M * R * (K + N) + 2 * M * r * (K + N)
+    return fp4, lowrank
+
+
+def kernel_work(M, K, N, r_s, r):
+    """Algorithmic work per launch of each kernel: ('tensor', FLOPs) or ('hbm', bytes)."""
+    R = r_s + r
+    return {
+        "fwd.pack_lowrank": ("hbm", 2 * 2 * R * (K + N)),
+        "fwd.xpass_quant_down": ("hbm", 2 * M * K + M * K // 2 + M * K // 256 + 2 * M * R),
+        "fwd.gemm_fp4_fwd": ("tensor", 2 * M * N * K),
+        "bwd.pack_lowrank": ("hbm", 2 * 2 * R * (K + N)),
+        "bwd.gpass_quant_down": ("hbm", 2 * M * N + M * N // 2 + M * N // 256 + 2 * M * R),
+        "bwd.gemm_fp4_dx": ("tensor", 2 * M * N * K),
+        "bwd.tgrad_dA": ("hbm", 2 * M * K + 2 * M * R + 4 * K * r),
+        "bwd.tgrad_dB": ("hbm", 2 * M * N + 2 * M * R + 4 * N * r),
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=FALLBACK["hbm_gbs"], bf16_tflops=FALLBACK["bf16_tflops"],
+                    bf16_tflops_sustained=FALLBACK["bf16_tflops"], source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Reads SM clock and clock-event reasons through NVML every ~10 ms (read-only)."""
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self._nv:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for b, n in _REASONS.items() if self.reasons & b]}
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+def oracle_step(p, Rc, Rs, X, dY):
+    from oracle import layer as olayer
+    f = olayer.linear_fwd(X, Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
+    olayer.linear_bwd(dY, X, f["L"], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"])
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_inputs(rows):
+    from bit_lora_fine_b200 import synth
+    from oracle import block16
+    wl = synth.WORKLOADS[WORKLOAD]
+    spec = wl.layers[0]
+    p = synth.layer_params(spec)
+    Rc, Rs = block16.quantize(p["R"])                    # frozen weight: quantized once, outside timing
+    X = synth.layer_input(wl)[:rows]
+    dY = synth.upstream_grad(wl)[:rows]
+    return wl, spec, p, Rc, Rs, X, dY
+
+
+def time_oracle(rows, repeats=1):
+    wl, spec, p, Rc, Rs, X, dY = oracle_inputs(rows)
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle_step(p, Rc, Rs, X, dY)
+        times.append(time.perf_counter() - t0)
+    fp4, lr = layer_work(rows, spec.K, spec.N, spec.r_s, spec.r)
+    return times, (fp4 + lr)
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from bit_lora_fine_b200 import synth
+    spec = synth.WORKLOADS[WORKLOAD].layers[0]
+    wl, spec, p, Rc, Rs, X, dY = oracle_inputs(ORACLE_ROWS)
+    for _ in range(args.warmup):
+        oracle_step(p, Rc, Rs, X, dY)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(p, Rc, Rs, X, dY)
+    dt = time.perf_counter() - t0
+    fp4, lr = layer_work(ORACLE_ROWS, spec.K, spec.N, spec.r_s, spec.r)
+    value = (fp4 + lr) * args.steps / dt / 1e12
+    sample = f"{ORACLE_ROWS} of {wl.M} tokens per step, full K=N={spec.K}, ranks {spec.r_s}/{spec.r}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "tokens_per_s": ORACLE_ROWS * args.steps / dt,
+        "config": {"workload": WORKLOAD, "M": wl.M, "K": spec.K, "N": spec.N, "r_s": spec.r_s, "r": spec.r},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours (GPU)
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bit_lora_fine_b200 import fourtune as ft
+    from bit_lora_fine_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[WORKLOAD]
+    spec = wl.layers[0]
+    M, K, N, r_s, r = wl.M, spec.K, spec.N, spec.r_s, spec.r
+    p = synth.layer_params(spec)
+    X_h = synth.layer_input(wl)
+    dY_h = synth.upstream_grad(wl)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16)
+    lay = ft.Linear.from_weights(up(p["R"]), up(p["S_dn"]), up(p["S_up"]), up(p["A"]), up(p["B"]))
+    X, dY = up(X_h), up(dY_h)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    L = torch.empty((M, r_s + r), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dA = torch.zeros((K, r), dtype=torch.float32, device=dev)
+    dB = torch.zeros((r, N), dtype=torch.float32, device=dev)
+    ws_f, ws_b = lay.fwd_workspace(M), lay.bwd_workspace(M)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    nf, nb = len(ft.FWD_KERNELS), len(ft.BWD_KERNELS)
+    names = [f"fwd.{k}" for k in ft.FWD_KERNELS] + [f"bwd.{k}" for k in ft.BWD_KERNELS]
+
+    def mk_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record()                     # materialize the CUDA event
+        return evs
+
+    def step(evf=None, evb=None):
+        ft.linear_fwd(lay, X, ws=ws_f, Y=Y, L=L, events=evf)
+        ft.linear_bwd(lay, dY, X, L, ws=ws_b, dX=dX, dA=dA, dB=dB, events=evb)
+
+    for _ in range(max(args.warmup, 1)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ft.device_status(ws_f)
+    ft.device_status(ws_b)
+
+    steps = [(mk_events(2), mk_events(2 * nf), mk_events(2 * nb)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for se, evf, evb in steps:
+        flush.zero_()
+        se[0].record()
+        step(evf, evb)
+        se[1].record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ft.device_status(ws_f)
+    ft.device_status(ws_b)
+
+    total_ms = sum(se[0].elapsed_time(se[1]) for se, _, _ in steps)
+    per_kernel = {n: 0.0 for n in names}
+    for _, evf, evb in steps:
+        for i in range(nf):
+            per_kernel[names[i]] += evf[2 * i].elapsed_time(evf[2 * i + 1])
+        for i in range(nb):
+            per_kernel[names[nf + i]] += evb[2 * i].elapsed_time(evb[2 * i + 1])
+
+    # ---- end to end through the C ABI with host-resident inputs and outputs
+    X_pin = torch.from_numpy(synth.bf16_bits(X_h).view(np.int16)).pin_memory()
+    dY_pin = torch.from_numpy(synth.bf16_bits(dY_h).view(np.int16)).pin_memory()
+    dA_pin = torch.empty((K, r), dtype=torch.float32).pin_memory()
+    dB_pin = torch.empty((r, N), dtype=torch.float32).pin_memory()
+    Xv, dYv = X.view(torch.int16), dY.view(torch.int16)
+    e2e_ev = [mk_events(2) for _ in range(args.steps)]
+    for _ in range(max(args.warmup, 1)):
+        Xv.copy_(X_pin, non_blocking=True)
+        dYv.copy_(dY_pin, non_blocking=True)
+        step()
+        dA_pin.copy_(dA, non_blocking=True)
+        dB_pin.copy_(dB, non_blocking=True)
+    torch.cuda.synchronize()
+    for ev in e2e_ev:
+        flush.zero_()
+        ev[0].record()
+        Xv.copy_(X_pin, non_blocking=True)
+        dYv.copy_(dY_pin, non_blocking=True)
+        step()
+        dA_pin.copy_(dA, non_blocking=True)
+        dB_pin.copy_(dB, non_blocking=True)
+        ev[1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(ev[0].elapsed_time(ev[1]) for ev in e2e_ev)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    fp4, lr = layer_work(M, K, N, r_s, r)
+    sec = total_ms / 1e3
+    value = (fp4 + lr) * args.steps * world / sec / 1e12
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    work = kernel_work(M, K, N, r_s, r)
+    kern = {}
+    for n in names:
+        avg_ms = per_kernel[n] / args.steps
+        kind, amount = work[n]
+        if kind == "tensor":
+            ach = amount / (avg_ms / 1e3) / 1e12
+            kern[n] = {"us": avg_ms * 1e3, "achieved": ach, "unit": "TFLOP/s", "frac": ach / fp4_peak}
+        else:
+            ach = amount / (avg_ms / 1e3) / 1e9
+            kern[n] = {"us": avg_ms * 1e3, "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    dom = max(names, key=lambda n: per_kernel[n])
+    kind, amount = work[dom]
+    dk = kern[dom]
+    traffic = load_traffic(dom)
+    roofline = {"kernel": dom, "bound": kind, "achieved": dk["achieved"],
+                "peak": fp4_peak if kind == "tensor" else peaks["hbm_gbs"], "unit": dk["unit"],
+                "frac": dk["frac"], "traffic": traffic,
+                "peak_source": ("FP4 = measured bf16 burst x 4 (nominal dense ratio)" if kind == "tensor"
+                                else "measured HBM copy") + f" ({peaks['source']})",
+                "algorithmic_per_launch": amount}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4(e2m1 x e2m1, e4m3 16x16 scales)->f32; bf16 low-rank",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "r_s": r_s, "r": r, "global_batch_tokens": M * world,
+                   "l2": "flushed (256 MB write before each step, outside the timed events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single"},
+        "tokens_per_s": M * args.steps * world / sec,
+        "fp4_tflops": fp4 * args.steps * world / sec / 1e12,
+        "fp4_peak_frac": fp4 * args.steps * world / sec / 1e12 / fp4_peak,
+        "fp4_peak_tflops": fp4_peak,
+        "e2e": {"value": (fp4 + lr) * args.steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 2 * M * K + 2 * M * N, "d2h_bytes_per_step": 4 * K * r + 4 * r * N},
+        "gpu_launches": args.steps * (nf + nb),
+        "roofline": roofline,
+        "kernels": kern,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times, flop_s = time_oracle(M, repeats=1)
+        t = min(times)
+        line["cpu_baseline"] = {"value": flop_s / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+                                "kind": "oracle",
+                                "sample": f"one full fwd+bwd of the workload ({M} tokens, K=N={K}), {t:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(kernel)
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

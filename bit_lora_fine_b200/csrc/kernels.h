@@ -1,0 +1,76 @@
+// Internal host-side interface between the C-ABI layer (api.cu) and the kernel
+// files.  Not installed; the public interface is include/fourtune/fourtune.h.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ft {
+
+struct PackParams {
+  int K, N, r_s, r;
+  const void *S_dn, *A, *S_up, *B;      // bf16, row-major [K,r_s] [K,r] [r_s,N] [r,N]
+  uint16_t *Dt, *Dcat, *Ut, *Ucat;      // outputs, any may be null
+  int* zero_words;                       // status word + split counters, cleared first
+  long long n_zero_words;
+};
+
+// Quantize the rows of a bf16 input and project it onto R low-rank directions:
+// codes/scales = block16(X), L = bf16(X * W^T) with W^T given as a [R, K] map.
+struct RowpassParams {
+  int M, K, R;
+  int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
+  uint8_t* codes;                        // [M, K/2]
+  uint8_t* scales;                       // [M/16, K/16]
+  void* L;                               // bf16 [M, R]
+  float* part;                           // fp32 [nsplit, M, R] when nsplit > 1
+  int* counters;                         // [ceil(M/128)], zero on entry, left zero
+  int* status;
+};
+
+// out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1 with
+// scale(row, g) = sf[(row/16)*rs + g*gs], g the 16-wide K group; A2 [M, R2],
+// B2 [N, R2] bf16.
+struct GemmParams {
+  int M, N, K, R2;
+  const uint8_t* sfa;
+  long long sfa_rs, sfa_gs;
+  const uint8_t* sfb;
+  long long sfb_rs, sfb_gs;
+  const void* bias;                      // bf16 [N] or null
+  void* out;
+  long long ldo;
+  int out_bf16;
+  int* status;
+};
+
+// out[p, j] (+)= sum_m T[m, p] * V[m, v0 + j]   for p < P, j < r (r <= 64)
+struct TgradParams {
+  int M, P, r, v0;
+  int mt_per_split, nsplit;              // 128-row tiles per CTA along M, number of M splits
+  float* out;
+  long long out_sp, out_sj;
+  int accumulate;
+  float* part;                           // fp32 [nsplit, ceil(P/128)*128, 64] when nsplit > 1
+  int* counters;                         // [ceil(P/128)]
+  int* status;
+};
+
+cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long ld, uint8_t* codes,
+                                    uint8_t* scales, cudaStream_t stream);
+cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uint8_t* codes_t,
+                                   cudaStream_t stream);
+cudaError_t launch_pack_lowrank(const PackParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
+                           cudaStream_t stream);
+cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
+                            const CUtensorMap& tmB2, const GemmParams& p, cudaStream_t stream);
+cudaError_t launch_tgrad(const CUtensorMap& tmT, const CUtensorMap& tmV, const TgradParams& p,
+                         cudaStream_t stream);
+
+// tile sizes the host needs for tensor-map boxes and workspace sizing
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kRowTile = 128;
+
+}  // namespace ft

@@ -1,0 +1,139 @@
+// Standalone 16x16-block FP4 quantizer and the nibble transpose of its codes.
+//
+// FourTune §3.2 / §4.3: each 16x16 block carries one scale, so the transposed
+// operand of the backward GEMM is the same codes re-packed along the other
+// dimension with the same scale bytes (no requantization).
+//
+// Per block: a = max|t|; s = a / 6 (fp32 division, round to nearest);
+// sc = E4M3(s) (round to nearest even, saturate at 448); if sc decodes to 0
+// every code is +0, else code = E2M1(t / dec(sc)) (fp32 division, round to
+// nearest even, saturate at +-6, sign kept).  Codes: even column in the low
+// nibble of byte [row, col/2]; scales: one byte per block, [rows/16, cols/16].
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ft {
+
+// One warp quantizes a 16-row x 64-column strip (up to four blocks).
+// Lane l owns row (l >> 1) of the strip and the 32-column half (l & 1).
+template <typename T>
+__device__ __forceinline__ void load32(const T* src, float* v);
+
+template <>
+__device__ __forceinline__ void load32<__nv_bfloat16>(const __nv_bfloat16* src, float* v) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u = p[q];
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[q * 8 + 2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
+      v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) quantize_block16_kernel(const __nv_bfloat16* __restrict__ x, int rows,
+                                                               int cols, long long ld, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int strips_per_row = (cols + 63) / 64;
+  const long long nstrips = static_cast<long long>(rows / 16) * strips_per_row;
+  if (warp >= nstrips) return;
+  const int rb = static_cast<int>(warp / strips_per_row);
+  const int c0 = static_cast<int>(warp % strips_per_row) * 64;
+  const int r = rb * 16 + (lane >> 1);
+  const int h = lane & 1;
+  const int cstart = c0 + 32 * h;
+  const bool live = cstart < cols;           // cols % 16 == 0: a half may hold one or two blocks
+  const int nblk = live ? min(2, (cols - cstart) / 16) : 0;
+
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+  if (nblk == 2) {
+    load32(x + static_cast<long long>(r) * ld + cstart, v);
+  } else if (nblk == 1) {
+    const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<long long>(r) * ld + cstart);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint4 u = p[q];
+      uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[q * 8 + 2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
+        v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+      }
+    }
+  }
+
+  float amax[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[16 * j + i]));
+    // reduce over the 16 lanes that share this half (lane bit 0 fixed)
+#pragma unroll
+    for (int off = 2; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    amax[j] = a;
+  }
+
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    if (j >= nblk) break;
+    const float s = __fdiv_rn(amax[j], 6.0f);
+    const uint32_t sc = f32_to_e4m3(s);
+    const float d = e4m3_to_f32(sc);
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + i], d);
+    uint2 packed;
+    packed.x = f32x8_to_e2m1(q);
+    packed.y = f32x8_to_e2m1(q + 8);
+    const int cb = cstart + 16 * j;
+    *reinterpret_cast<uint2*>(codes + static_cast<long long>(r) * (cols / 2) + cb / 2) = packed;
+    if ((lane >> 1) == 0) scales[static_cast<long long>(rb) * (cols / 16) + cb / 16] = static_cast<uint8_t>(sc);
+  }
+}
+
+// codes_t[c, r/2] = nibble (r & 1) <- code of element (r, c)
+__global__ void transpose_codes_kernel(const uint8_t* __restrict__ codes, int rows, int cols,
+                                       uint8_t* __restrict__ codes_t) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long total = static_cast<long long>(cols) * (rows / 2);
+  if (i >= total) return;
+  const int c = static_cast<int>(i / (rows / 2));
+  const int rp = static_cast<int>(i % (rows / 2));
+  const uint8_t b0 = codes[static_cast<long long>(2 * rp) * (cols / 2) + c / 2];
+  const uint8_t b1 = codes[static_cast<long long>(2 * rp + 1) * (cols / 2) + c / 2];
+  const uint32_t n0 = (c & 1) ? (b0 >> 4) : (b0 & 0xF);
+  const uint32_t n1 = (c & 1) ? (b1 >> 4) : (b1 & 0xF);
+  codes_t[i] = static_cast<uint8_t>(n0 | (n1 << 4));
+}
+
+cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long ld, uint8_t* codes,
+                                    uint8_t* scales, cudaStream_t stream) {
+  const long long nstrips = static_cast<long long>(rows / 16) * ((cols + 63) / 64);
+  if (nstrips == 0) return cudaSuccess;
+  const long long threads = nstrips * 32;
+  const int block = 256;
+  const long long grid = (threads + block - 1) / block;
+  quantize_block16_kernel<<<static_cast<unsigned>(grid), block, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, cols, ld, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uint8_t* codes_t,
+                                   cudaStream_t stream) {
+  const long long total = static_cast<long long>(cols) * (rows / 2);
+  if (total == 0) return cudaSuccess;
+  const int block = 256;
+  transpose_codes_kernel<<<static_cast<unsigned>((total + block - 1) / block), block, 0, stream>>>(codes, rows,
+                                                                                                  cols, codes_t);
+  return cudaGetLastError();
+}
+
+}  // namespace ft

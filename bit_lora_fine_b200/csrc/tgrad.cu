@@ -1,0 +1,187 @@
+// Adapter gradients: out[p, j] (+)= sum_m T[m, p] V[m, v0 + j].
+//
+// FourTune §3.2: parameter gradients exist only for the LoRA adapter (no weight
+// gradient for the frozen residual or stabilizer).  With L = X [S_dn | A] and
+// P = G [S_up ; B]^T saved in bf16:
+//   dA = X^T P[:, r_s:]   (T = X,  V = P, out [K, r] row-major)
+//   dB = L[:, r_s:]^T G   (T = G,  V = L, out [r, N] row-major, written as dB^T)
+// Both are reductions over the M tokens of a tall bf16 matrix against a thin
+// one: HBM-bound (T is read once).  The tensor cores take both operands
+// MN-major straight from the TMA tiles: T tile [128 m x 128 p] (two 128-byte
+// swizzled boxes of 64 p), V tile [128 m x 64 j]; tcgen05.mma kind::f16
+// M=128 (p), N=64 (j), K=16 (m), 8 per tile.  CTAs split M; the last CTA of a
+// p-tile sums the fp32 partials in split order (deterministic).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ft {
+
+constexpr int kTgStages = 4;
+constexpr int kTgThreads = 256;
+constexpr uint32_t kTgTBox = 128 * 128;            // 128 m rows x 64 bf16
+constexpr uint32_t kTgStage = 2 * kTgTBox + kTgTBox;  // T (two boxes) + V
+constexpr uint32_t kTgSmem = 1024 + kTgStages * kTgStage + 256;
+
+__global__ void __launch_bounds__(kTgThreads, 1)
+    tgrad_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmV,
+                 const TgradParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTgStages * kTgStage);
+  uint64_t* empty = full + kTgStages;
+  uint64_t* acc_full = empty + kTgStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* s_last = abort_flag + 1;
+  volatile int* abortp = abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * 128;
+  const int split = blockIdx.y;
+  const int MT = (p.M + 127) / 128;
+  const int mt0 = split * p.mt_per_split;
+  const int mt1 = min(MT, mt0 + p.mt_per_split);
+  const int nt = max(0, mt1 - mt0);
+  const int Ppad = ((p.P + 127) / 128) * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTgStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmT);
+    tma_prefetch(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % kTgStages;
+        const uint32_t ph = (i / kTgStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
+        uint8_t* st = smem + s * kTgStage;
+        const int my = (mt0 + i) * 128;
+        mbar_arrive_expect_tx(&full[s], kTgStage);
+        tma_load_2d(st, &tmT, &full[s], p0, my);
+        tma_load_2d(st + kTgTBox, &tmT, &full[s], p0 + 64, my);
+        tma_load_2d(st + 2 * kTgTBox, &tmV, &full[s], p.v0, my);
+        issued = i + 1;
+      }
+      if (*abortp) {
+        for (int i = max(0, issued - kTgStages); i < issued; ++i)
+          mbar_wait_drain(&full[i % kTgStages], (i / kTgStages) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, 64, true, true);
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % kTgStages;
+        const uint32_t ph = (i / kTgStages) & 1;
+        if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
+        tc_fence_after();
+        const uint32_t ta = smem_u32(smem + s * kTgStage);
+        const uint32_t va = ta + 2 * kTgTBox;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          mma_bf16(tmem, desc_mnmajor_sw128(ta + 2048 * t, kTgTBox), desc_mnmajor_sw128(va + 2048 * t, kTgTBox),
+                   idesc, (i | t) != 0 ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      tc_commit(acc_full);
+      mbar_wait_drain(acc_full, 0, kWaitLimitNs);
+    }
+  } else if (warp >= 4) {
+    const bool mine = (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
+    if (lane == 0) s_last[1 + (warp - 4)] = mine ? 1 : 0;
+    named_bar_sync(1, 128);
+    const volatile int* ok4 = s_last + 1;
+    const bool go = ok4[0] && ok4[1] && ok4[2] && ok4[3];
+    if (go) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int prow = p0 + 32 * q + lane;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      uint32_t v[64];
+      {
+        uint32_t a[32], b[32];
+        tmem_ld_32x32b_x32(taddr, a);
+        tmem_ld_32x32b_x32(taddr + 32, b);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          v[e] = a[e];
+          v[32 + e] = b[e];
+        }
+      }
+      const bool prow_ok = prow < p.P;
+      if (p.nsplit == 1) {
+        if (prow_ok) {
+          for (int j = 0; j < p.r; ++j) {
+            float* o = p.out + prow * p.out_sp + j * p.out_sj;
+            const float val = __uint_as_float(v[j]);
+            *o = p.accumulate ? *o + val : val;
+          }
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(p.part + (static_cast<long long>(split) * Ppad + prow) * 64);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                               __uint_as_float(v[4 * e + 3]));
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 128) {
+          const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
+          *s_last = (prev == p.nsplit - 1);
+        }
+        named_bar_sync(1, 128);
+        if (*s_last) {
+          __threadfence();
+          if (prow_ok) {
+            for (int j = 0; j < p.r; ++j) {
+              float acc = 0.0f;
+              for (int sp = 0; sp < p.nsplit; ++sp)
+                acc += __ldcg(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64 + j);
+              float* o = p.out + prow * p.out_sp + j * p.out_sj;
+              *o = p.accumulate ? *o + acc : acc;
+            }
+          }
+          if (threadIdx.x == 128) p.counters[blockIdx.x] = 0;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+cudaError_t launch_tgrad(const CUtensorMap& tmT, const CUtensorMap& tmV, const TgradParams& p, cudaStream_t stream) {
+  cudaError_t e =
+      cudaFuncSetAttribute(tgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTgSmem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.P + 127) / 128, p.nsplit);
+  tgrad_kernel<<<grid, kTgThreads, kTgSmem, stream>>>(tmT, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace ft

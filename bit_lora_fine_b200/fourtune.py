@@ -1,0 +1,220 @@
+"""Python binding of libfourtune.so: argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; PyTorch supplies
+device memory and the current stream.  There is no fallback: if the library is
+missing or the device is not sm_100, calls raise.
+
+Names follow the C ABI in include/fourtune/fourtune.h (FourTune §3.1-§3.3):
+quantize_block16, transpose_codes, linear_fwd, linear_bwd.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfourtune.so")
+
+FT_DTYPE_F32 = 0
+FT_DTYPE_BF16 = 1
+ERRORS = {0: "FT_OK", -1: "FT_ERR_INVALID_ARG", -2: "FT_ERR_SHAPE", -3: "FT_ERR_ALIGN",
+          -4: "FT_ERR_WORKSPACE", -5: "FT_ERR_CUDA", -6: "FT_ERR_TIMEOUT", -7: "FT_ERR_UNSUPPORTED"}
+
+EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_linear_fwd_workspace_size",
+            "fourtune_linear_bwd_workspace_size", "fourtune_linear_fwd", "fourtune_linear_bwd",
+            "fourtune_linear_fwd_ws_offsets", "fourtune_linear_bwd_ws_offsets", "fourtune_device_status",
+            "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed")
+
+# kernels each call launches, in order (the *_timed entry points bracket each with events)
+FWD_KERNELS = ("pack_lowrank", "xpass_quant_down", "gemm_fp4_fwd")
+BWD_KERNELS = ("pack_lowrank", "gpass_quant_down", "gemm_fp4_dx", "tgrad_dA", "tgrad_dB")
+
+
+class FourtuneError(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {ERRORS.get(code, code)} ({code})")
+        self.code = code
+
+
+class ft_linear_t(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int64), ("N", ctypes.c_int64), ("r_s", ctypes.c_int64), ("r", ctypes.c_int64),
+                ("R_codes", ctypes.c_void_p), ("R_scales", ctypes.c_void_p), ("R_codes_t", ctypes.c_void_p),
+                ("S_dn", ctypes.c_void_p), ("S_up", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load():
+    """Load libfourtune.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_lora_fine_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.fourtune_quantize_block16.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
+    L.fourtune_transpose_codes.argtypes = [vp, i64, i64, vp, vp]
+    L.fourtune_linear_fwd_workspace_size.argtypes = [P(ft_linear_t), i64]
+    L.fourtune_linear_fwd_workspace_size.restype = sz
+    L.fourtune_linear_bwd_workspace_size.argtypes = [P(ft_linear_t), i64]
+    L.fourtune_linear_bwd_workspace_size.restype = sz
+    L.fourtune_linear_fwd.argtypes = [P(ft_linear_t), vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
+    L.fourtune_linear_bwd.argtypes = [P(ft_linear_t), vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, ctypes.c_int,
+                                      vp, sz, vp]
+    L.fourtune_linear_fwd_timed.argtypes = list(L.fourtune_linear_fwd.argtypes) + [P(vp), ctypes.c_int]
+    L.fourtune_linear_bwd_timed.argtypes = list(L.fourtune_linear_bwd.argtypes) + [P(vp), ctypes.c_int]
+    L.fourtune_linear_fwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz)]
+    L.fourtune_linear_bwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz), P(sz)]
+    L.fourtune_device_status.argtypes = [vp, vp]
+    L.fourtune_error_string.argtypes = [ctypes.c_int]
+    L.fourtune_error_string.restype = ctypes.c_char_p
+    for f in EXPORTED:
+        if f not in ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size",
+                     "fourtune_error_string"):
+            getattr(L, f).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(code, where):
+    if code != 0:
+        raise FourtuneError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, dtype, name):
+    if t is None:
+        return
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def quantize_block16(x, transposed=False):
+    """x: bf16 [rows, cols] -> (codes u8 [rows, cols/2], scales u8 [rows/16, cols/16], codes_t or None)."""
+    _need(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows // 16, cols // 16), dtype=torch.uint8, device=x.device)
+    codes_t = torch.empty((cols, rows // 2), dtype=torch.uint8, device=x.device) if transposed else None
+    _check(load().fourtune_quantize_block16(_ptr(x), rows, cols, x.stride(0), _ptr(codes), _ptr(scales),
+                                            _ptr(codes_t), _stream()), "fourtune_quantize_block16")
+    return codes, scales, codes_t
+
+
+def transpose_codes(codes, rows, cols):
+    out = torch.empty((cols, rows // 2), dtype=torch.uint8, device=codes.device)
+    _check(load().fourtune_transpose_codes(_ptr(codes), rows, cols, _ptr(out), _stream()),
+           "fourtune_transpose_codes")
+    return out
+
+
+class Linear:
+    """Device tensors of one triple-branch layer (frozen R codes/scales/codes_t, S_dn, S_up,
+    bias; trainable A, B).  Holds references so the pointers stay valid."""
+
+    def __init__(self, R_codes, R_scales, R_codes_t, S_dn, S_up, A, B, bias=None):
+        N, half_k = R_codes.shape
+        self.K, self.N = half_k * 2, N
+        self.r_s, self.r = S_dn.shape[1], A.shape[1]
+        for t, n in ((R_codes, "R_codes"), (R_scales, "R_scales"), (R_codes_t, "R_codes_t")):
+            _need(t, torch.uint8, n)
+        for t, n in ((S_dn, "S_dn"), (S_up, "S_up"), (A, "A"), (B, "B"), (bias, "bias")):
+            _need(t, torch.bfloat16, n)
+        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_codes_t=R_codes_t, S_dn=S_dn, S_up=S_up, A=A, B=B,
+                      bias=bias)
+        self.c = ft_linear_t(self.K, self.N, self.r_s, self.r, *[
+            _ptr(self.t[k]) for k in ("R_codes", "R_scales", "R_codes_t", "S_dn", "S_up", "A", "B", "bias")])
+
+    @classmethod
+    def from_weights(cls, R, S_dn, S_up, A, B, bias=None):
+        """Quantize the frozen residual weight R [N, K] (bf16) on the device."""
+        codes, scales, codes_t = quantize_block16(R, transposed=True)
+        return cls(codes, scales, codes_t, S_dn, S_up, A, B, bias)
+
+    @property
+    def R_all(self):
+        return self.r_s + self.r
+
+    def fwd_workspace(self, M):
+        n = load().fourtune_linear_fwd_workspace_size(ctypes.byref(self.c), M)
+        if n == 0:
+            raise FourtuneError(-2, "fourtune_linear_fwd_workspace_size")
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def bwd_workspace(self, M):
+        n = load().fourtune_linear_bwd_workspace_size(ctypes.byref(self.c), M)
+        if n == 0:
+            raise FourtuneError(-2, "fourtune_linear_bwd_workspace_size")
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def fwd_ws_offsets(self, M):
+        c, s = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().fourtune_linear_fwd_ws_offsets(ctypes.byref(self.c), M, ctypes.byref(c), ctypes.byref(s)),
+               "fourtune_linear_fwd_ws_offsets")
+        return c.value, s.value
+
+    def bwd_ws_offsets(self, M):
+        c, s, p = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().fourtune_linear_bwd_ws_offsets(ctypes.byref(self.c), M, ctypes.byref(c), ctypes.byref(s),
+                                                     ctypes.byref(p)), "fourtune_linear_bwd_ws_offsets")
+        return c.value, s.value, p.value
+
+
+def _events(events):
+    """List of torch.cuda.Event (already recorded once, so they exist) -> void*[]."""
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    return arr, len(events)
+
+
+def linear_fwd(layer, X, y_dtype=torch.float32, ws=None, Y=None, L=None, events=None):
+    """Y = deq(Q(X) Q(R)^T) + L [S_up ; B] + bias, L = bf16(X [S_dn | A]).  Returns (Y, L, ws).
+    `events`: optional 2*len(FWD_KERNELS) torch.cuda.Events recorded around each kernel."""
+    _need(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    Y = torch.empty((M, layer.N), dtype=y_dtype, device=X.device) if Y is None else Y
+    L = torch.empty((M, layer.R_all), dtype=torch.bfloat16, device=X.device) if L is None else L
+    ws = layer.fwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if Y.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(layer.c), _ptr(X), M, _ptr(Y), code, _ptr(L), _ptr(ws), ws.numel(), _stream())
+    if events is None:
+        _check(load().fourtune_linear_fwd(*args), "fourtune_linear_fwd")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_linear_fwd_timed(*args, arr, n), "fourtune_linear_fwd_timed")
+    return Y, L, ws
+
+
+def linear_bwd(layer, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumulate=False, ws=None, dX=None,
+               events=None):
+    """dX = deq(Q(dY)) deq(Q(R)) + P [S_dn | A]^T, dA = X^T P_B, dB = L_B^T dY.  Returns (dX, dA, dB, ws)."""
+    _need(dY, torch.bfloat16, "dY")
+    M = dY.shape[0]
+    dX = torch.empty((M, layer.K), dtype=dx_dtype, device=dY.device) if dX is None else dX
+    dA = torch.zeros((layer.K, layer.r), dtype=torch.float32, device=dY.device) if dA is None else dA
+    dB = torch.zeros((layer.r, layer.N), dtype=torch.float32, device=dY.device) if dB is None else dB
+    ws = layer.bwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if dX.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(layer.c), _ptr(dY), _ptr(X), _ptr(L), M, _ptr(dX), code, _ptr(dA), _ptr(dB),
+            int(accumulate), _ptr(ws), ws.numel(), _stream())
+    if events is None:
+        _check(load().fourtune_linear_bwd(*args), "fourtune_linear_bwd")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_linear_bwd_timed(*args, arr, n), "fourtune_linear_bwd_timed")
+    return dX, dA, dB, ws
+
+
+def device_status(ws):
+    """Synchronize and raise FourtuneError(FT_ERR_TIMEOUT) if a kernel wait expired."""
+    _check(load().fourtune_device_status(_ptr(ws), _stream()), "fourtune_device_status")

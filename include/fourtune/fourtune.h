@@ -1,0 +1,157 @@
+/*
+ * fourtune.h -- C ABI of the B200 (sm_100a) FourTune layer library.
+ *
+ * The layer is the triple-branch hybrid-precision linear of "FourTune: Towards
+ * Fully 4-Bit Efficient Post-Training for Diffusion Models" (§3.1): a frozen
+ * 4-bit residual weight R, a frozen bf16 low-rank stabilizer (S_dn, S_up) and a
+ * trainable bf16 LoRA adapter (A, B), all fed the same input:
+ *
+ *     y = deq(Q(X) Q(R)^T) + (X S_dn) S_up + (X A) B  (+ bias)
+ *
+ * with weights, activations and gradients quantized to 4 bits (W4A4G4, §3).
+ * Q is 16x16-block quantization (§3.2, §4.3 "Impact of Quantization
+ * Granularity"): FP4 E2M1 codes, one FP8 E4M3 scale per 16x16 block,
+ * round-to-nearest-even.  Because a block's scale belongs to the block, the
+ * backward product Q(G) Q(R) reads R's blocks transposed with the same codes and
+ * scales, no requantization (§3.2).
+ *
+ * Conventions (every entry point):
+ *   - Return value: FT_OK (0) or a negative FT_ERR_* code; nothing is launched
+ *     when an argument check fails.
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates device memory.  Scratch space is the caller's `ws` buffer
+ *     of at least *_workspace_size(...) bytes, 256-byte aligned; it must not be
+ *     shared by calls that may run concurrently.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  A kernel whose internal wait times out
+ *     records it in the workspace; fourtune_device_status() reports it.
+ *   - bf16 tensors are arrays of IEEE bfloat16 bit patterns (ft_bf16), row-major,
+ *     16-byte aligned.  Dimensions must be multiples of 16; K and N must also be
+ *     multiples of 32 (4-bit rows are copied in 16-byte units).
+ *   - Block16 tensor of a [rows, cols] matrix: codes uint8 [rows, cols/2]
+ *     (column 2i in the low nibble of byte i, 2i+1 in the high nibble) and
+ *     scales uint8 [rows/16, cols/16] (E4M3 bit patterns).
+ *   - Requires an sm_100 device (B200); FT_ERR_UNSUPPORTED otherwise.
+ */
+#ifndef FOURTUNE_FOURTUNE_H_
+#define FOURTUNE_FOURTUNE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FT_API __attribute__((visibility("default")))
+#else
+#define FT_API
+#endif
+
+typedef uint16_t ft_bf16;
+
+enum {
+  FT_OK = 0,
+  FT_ERR_INVALID_ARG = -1, /* null pointer, bad enum, rank out of range */
+  FT_ERR_SHAPE = -2,       /* a dimension is not a multiple of 16 (or 32 where stated) */
+  FT_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned (256 for the workspace) */
+  FT_ERR_WORKSPACE = -4,   /* ws_bytes smaller than the *_workspace_size() value */
+  FT_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed */
+  FT_ERR_TIMEOUT = -6,     /* a kernel's bounded wait expired (device status) */
+  FT_ERR_UNSUPPORTED = -7  /* not an sm_100 device, or a size this build does not handle */
+};
+
+enum { FT_DTYPE_F32 = 0, FT_DTYPE_BF16 = 1 };
+
+/* One triple-branch linear layer, y[M, N] from x[M, K]  (§3.1, §3.2).
+ *   R_codes   [N, K/2]  block16 codes of the frozen residual weight R [N, K]
+ *   R_scales  [N/16, K/16]
+ *   R_codes_t [K, N/2]  the same codes nibble-transposed (codes of R^T); the
+ *                       scales of R^T are R_scales read transposed.  Required by
+ *                       the backward (fourtune_quantize_block16 writes it).
+ *   S_dn [K, r_s], S_up [r_s, N]  frozen stabilizer (bf16)
+ *   A [K, r], B [r, N]            trainable LoRA (bf16)
+ *   bias [N] frozen bf16 or NULL
+ * Ranks: r_s >= 0, r >= 16, r_s + r <= 128, each a multiple of 16; r <= 64. */
+typedef struct {
+  int64_t K, N, r_s, r;
+  const uint8_t* R_codes;
+  const uint8_t* R_scales;
+  const uint8_t* R_codes_t;
+  const ft_bf16* S_dn;
+  const ft_bf16* S_up;
+  const ft_bf16* A;
+  const ft_bf16* B;
+  const ft_bf16* bias;
+} ft_linear_t;
+
+/* Block16 quantization of a bf16 matrix x [rows, cols] with row stride `ld`
+ * elements (§2.3 Round(W/s), §3.2, §4.3): per 16x16 block, s = amax/6 in fp32,
+ * scale = E4M3(s) (nearest-even, saturating at 448, subnormals kept), codes =
+ * E2M1(x / scale) (nearest-even, saturating at +-6, sign kept; all +0 when the
+ * scale is 0).  Writes codes [rows, cols/2], scales [rows/16, cols/16] and, if
+ * codes_t is not NULL, the transposed codes [cols, rows/2].  Used offline for
+ * the frozen residual weight.  rows, cols multiples of 16; ld multiple of 8. */
+FT_API int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                              uint8_t* scales, uint8_t* codes_t, void* stream);
+
+/* Nibble transpose of block16 codes: codes [rows, cols/2] -> codes_t [cols, rows/2]
+ * (§3.2: the transposed operand keeps its codes and scales). */
+FT_API int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, uint8_t* codes_t, void* stream);
+
+/* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
+FT_API size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M);
+FT_API size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M);
+
+/* Forward (§3.1, §3.3 LoRA fusion).  X [M, K] bf16.  Writes
+ *   Y [M, N] (y_dtype FT_DTYPE_F32 or FT_DTYPE_BF16, row stride N)
+ *   L_saved [M, r_s + r] bf16 = bf16(X [S_dn | A]), kept for the backward.
+ * One pass reads X once, quantizes it and computes L; the 4-bit GEMM then adds
+ * L [S_up ; B] and the bias in its accumulator. */
+FT_API int fourtune_linear_fwd(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
+                        ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward (§3.2).  dY [M, N] bf16 (the incoming gradient G), X and L_saved from
+ * the forward.  Writes
+ *   dX [M, K] = deq(Q(G)) deq(Q(R)) + P [S_dn | A]^T   (dx_dtype F32 or BF16)
+ *   dA [K, r] fp32 = X^T P[:, r_s:]     dB [r, N] fp32 = L[:, r_s:]^T G
+ * with P = bf16(G [S_up ; B]^T).  accumulate = 1 adds into dA and dB, 0
+ * overwrites.  R, S and bias receive no gradient. */
+FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, const ft_bf16* X, const ft_bf16* L_saved,
+                        int64_t M, void* dX, int dx_dtype, float* dA, float* dB, int accumulate, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* The same calls, recording caller-created CUDA events (cudaEvent_t as void*) on
+ * `stream` around each kernel they launch: events[2k] before and events[2k+1]
+ * after kernel k (NULL entries and k >= n_events/2 are skipped).  Kernels, in
+ * order -- forward: 0 pack low-rank factors, 1 fused X pass (quantize + X D),
+ * 2 FP4 GEMM with up-projection; backward: 0 pack, 1 fused G pass (quantize +
+ * G U^T), 2 FP4 dX GEMM, 3 dA, 4 dB.  Used for live per-kernel timing. */
+FT_API int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
+                                     ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream,
+                                     void* const* events, int n_events);
+FT_API int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const ft_bf16* X,
+                                     const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA,
+                                     float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream,
+                                     void* const* events, int n_events);
+
+/* Byte offsets, inside the workspace of the last fwd / bwd call with these sizes,
+ * of the block16 activation (fwd: Q(X)) or gradient (bwd: Q(G)) codes and scales,
+ * and (bwd) of P [M, r_s + r] bf16.  For inspection and tests; unused -> NULL. */
+FT_API int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off);
+FT_API int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off,
+                                   size_t* P_off);
+
+/* Synchronizes `stream` and returns FT_ERR_TIMEOUT if a kernel of the last call
+ * that used `ws` recorded an expired wait, FT_ERR_CUDA on a CUDA error, else FT_OK. */
+FT_API int fourtune_device_status(const void* ws, void* stream);
+
+/* Static description of an FT_* code. */
+FT_API const char* fourtune_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOURTUNE_FOURTUNE_H_ */

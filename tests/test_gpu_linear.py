@@ -1,0 +1,118 @@
+"""GPU triple-branch linear (fwd + bwd) vs the oracle.
+
+FourTune §3.1 (three branches), §3.2 (4-bit backward on transposed blocks, no
+gradient for frozen parts), §3.3 (LoRA fusion).  Bar: Q(X) and Q(G) codes and
+scales bit-identical; y, dX, dA, dB, L, P within the normwise 2e-3 tolerance of
+tests/helpers.py; the bf16 intermediates L and P within one bf16 ulp of the
+oracle's (both round once after accumulating); bf16 outputs equal to the
+rounding of the fp32 outputs.
+"""
+import numpy as np
+import pytest
+
+from bit_lora_fine_b200 import synth
+from oracle import block16, formats, layer as olayer
+from tests.helpers import TOL, bf16_ulps, normwise, random_layer, to_dev_bf16, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _device_layer(ft, p):
+    import torch
+    dev = {k: (to_dev_bf16(v) if v is not None else None) for k, v in p.items() if k in
+           ("R", "S_dn", "S_up", "A", "B", "bias")}
+    lay = ft.Linear.from_weights(dev["R"], dev["S_dn"], dev["S_up"], dev["A"], dev["B"], dev["bias"])
+    torch.cuda.synchronize()
+    return lay
+
+
+def run_and_check(ft, p, M, check_bf16=True):
+    import torch
+    X, dY = p["X"], p["dY"]
+    lay = _device_layer(ft, p)
+    R_codes, R_scales = block16.quantize(p["R"])
+    np.testing.assert_array_equal(lay.t["R_codes"].cpu().numpy(), R_codes)
+    np.testing.assert_array_equal(lay.t["R_scales"].cpu().numpy(), R_scales)
+    np.testing.assert_array_equal(lay.t["R_codes_t"].cpu().numpy(), block16.transpose_pack(R_codes))
+
+    Xd, dYd = to_dev_bf16(X), to_dev_bf16(dY)
+    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32)
+    ft.device_status(ws)
+    co, so = lay.fwd_ws_offsets(M)
+    K, N = lay.K, lay.N
+    qx_codes = ws[co:co + M * K // 2].view(M, K // 2).cpu().numpy()
+    qx_scales = ws[so:so + (M // 16) * (K // 16)].view(M // 16, K // 16).cpu().numpy()
+
+    ref = olayer.linear_fwd(X, R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
+    np.testing.assert_array_equal(qx_scales, ref["qx_scales"])
+    np.testing.assert_array_equal(qx_codes, ref["qx_codes"])
+    assert bf16_ulps(to_host(L), ref["L"]) <= 1.0          # bf16 output: at most one rounding flip
+    assert normwise(to_host(Y), ref["y"]) <= TOL, normwise(to_host(Y), ref["y"])
+
+    if check_bf16:
+        Yb, _, _ = ft.linear_fwd(lay, Xd, torch.bfloat16, ws=ws)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(to_host(Yb), to_host(Y.to(torch.bfloat16)))
+
+    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32)
+    ft.device_status(wsb)
+    gc, gs, po = lay.bwd_ws_offsets(M)
+    qg_codes = wsb[gc:gc + M * N // 2].view(M, N // 2).cpu().numpy()
+    qg_scales = wsb[gs:gs + (M // 16) * (N // 16)].view(M // 16, N // 16).cpu().numpy()
+    R_all = lay.R_all
+    P = wsb[po:po + M * R_all * 2].view(torch.bfloat16).view(M, R_all)
+
+    # backward reference on the GPU's own saved L (the saved tensor is the interface)
+    b = olayer.linear_bwd(dY, X, to_host(L), R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"])
+    np.testing.assert_array_equal(qg_scales, b["qg_scales"])
+    np.testing.assert_array_equal(qg_codes, b["qg_codes"])
+    assert bf16_ulps(to_host(P), b["P"]) <= 1.0
+    assert normwise(to_host(dX), b["dX"]) <= TOL, normwise(to_host(dX), b["dX"])
+    assert normwise(to_host(dA), b["dA"]) <= TOL, normwise(to_host(dA), b["dA"])
+    assert normwise(to_host(dB), b["dB"]) <= TOL, normwise(to_host(dB), b["dB"])
+
+    # accumulate = 1 adds into dA, dB
+    dX2, dA2, dB2, _ = ft.linear_bwd(lay, dYd, Xd, L, torch.float32, dA=dA.clone(), dB=dB.clone(),
+                                     accumulate=True, ws=wsb)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_host(dA2), 2 * to_host(dA))
+    np.testing.assert_array_equal(to_host(dB2), 2 * to_host(dB))
+    np.testing.assert_array_equal(to_host(dX2), to_host(dX))       # deterministic
+    return dict(Y=Y, dX=dX, dA=dA, dB=dB, lay=lay)
+
+
+@pytest.mark.parametrize("M,K,N,r_s,r,bias", [
+    (16, 32, 32, 0, 16, False),        # smallest: one 16-row block, one K group pair
+    (144, 96, 288, 16, 32, False),     # ragged M tile (128+16), K block (96 of 256), N tile (256+32)
+    (400, 320, 544, 32, 64, True),     # ragged everything, rank 96, bias
+    (128, 256, 256, 16, 16, False),    # exactly one tile
+])
+def test_edge_shapes(cuda_lib, M, K, N, r_s, r, bias):
+    p = random_layer(K, N, r_s, r, seed=M + K + N, bias=bias, M=M)
+    run_and_check(cuda_lib, p, M)
+
+
+def test_config_linear_256x512x512(cuda_lib):
+    wl = synth.WORKLOADS["linear-256x512x512"]
+    spec = wl.layers[0]
+    p = synth.layer_params(spec)
+    p["X"] = synth.layer_input(wl)
+    p["dY"] = synth.upstream_grad(wl)
+    run_and_check(cuda_lib, p, wl.M)
+
+
+def test_special_case_zero_adapter(cuda_lib):
+    """B = 0: the LoRA branch adds nothing and dA is exactly 0 (§3.2)."""
+    p = random_layer(256, 256, 16, 16, seed=3, M=128)
+    p["B"] = np.zeros_like(p["B"])
+    out = run_and_check(cuda_lib, p, 128, check_bf16=False)
+    assert np.all(to_host(out["dA"]) == 0)
+
+
+def test_config_flux_linear_3072(cuda_lib):
+    """FLUX-width linear at its full size (M=4608, K=N=3072, ranks 32/32)."""
+    wl = synth.WORKLOADS["flux-linear-3072"]
+    p = synth.layer_params(wl.layers[0])
+    p["X"] = synth.layer_input(wl)
+    p["dY"] = synth.upstream_grad(wl)
+    run_and_check(cuda_lib, p, wl.M, check_bf16=True)

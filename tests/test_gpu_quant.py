@@ -1,0 +1,78 @@
+"""GPU block16 quantizer vs the oracle: codes and scales must be bit-identical
+(FourTune §3.2, §4.3 16x16 blocks; E2M1 codes, E4M3 scales, nearest-even)."""
+import numpy as np
+import pytest
+
+from bit_lora_fine_b200 import synth
+from oracle import block16
+from tests.helpers import to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quant(cuda_lib, x, transposed=True):
+    codes, scales, codes_t = cuda_lib.quantize_block16(to_dev_bf16(x), transposed=transposed)
+    return codes.cpu().numpy(), scales.cpu().numpy(), None if codes_t is None else codes_t.cpu().numpy()
+
+
+def _check(cuda_lib, x):
+    c, s, ct = _gpu_quant(cuda_lib, x)
+    rc, rs = block16.quantize(x)
+    np.testing.assert_array_equal(s, rs)
+    np.testing.assert_array_equal(c, rc)
+    np.testing.assert_array_equal(ct, block16.transpose_pack(rc))
+
+
+def test_worked_ties_probe(cuda_lib):
+    # block amax 6 -> scale 1.0: the element codes are the E2M1 rounding ties,
+    # including the sign of small negatives and saturation; second block row: scale midpoints
+    b = np.zeros((32, 32), np.float32)
+    b[0, 0] = 6.0
+    b[1, :16] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.1, -0.0, 0.2500001, 2.9, -5.5, 4.5, 1.0, -6.0]
+    b[16, 0] = 6.375                        # s = 1.0625 -> scale 1.0, element saturates
+    b[16, 16] = 6 * 3 * 2.0 ** -9           # subnormal scale 0x03
+    b[0, 16] = 6 * 1000.0                   # scale saturates at 448
+    b[16:32, 16] = np.float32(1e-3)         # tiny block: after rounding to bf16 still small
+    b = synth.to_bf16(b)
+    _check(cuda_lib, b)
+
+
+@pytest.mark.parametrize("shape,std,seed", [((16, 16), 1.0, 0), ((32, 48), 0.02, 1), ((48, 80), 5.0, 2),
+                                            ((64, 96), 1e-4, 3), ((256, 512), 1.0, 4), ((144, 208), 0.3, 5)])
+def test_random_shapes(cuda_lib, shape, std, seed):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal(shape) * std).astype(np.float32)
+    x[:, rng.integers(shape[1])] *= 40
+    _check(cuda_lib, synth.to_bf16(x))            # both sides see the same bf16 values
+
+
+def test_zero_and_negative_zero_blocks(cuda_lib):
+    x = np.zeros((32, 32), np.float32)
+    x[0:16, 16:32] = -0.0
+    x[16, 16] = 3.0
+    _check(cuda_lib, synth.to_bf16(x))
+
+
+def test_flux_weight_full(cuda_lib):
+    """The FLUX-width residual weight R [3072, 3072] ~ N(0, 0.02), bit-exact in full."""
+    spec = synth.WORKLOADS["flux-linear-3072"].layers[0]
+    R = synth.layer_params(spec)["R"]
+    _check(cuda_lib, R)
+
+
+def test_row_stride(cuda_lib):
+    """A strided view (row stride 96 elements, 64 columns) through the C ABI."""
+    import ctypes
+    import torch
+    rng = np.random.default_rng(7)
+    big = synth.to_bf16(rng.standard_normal((48, 96)).astype(np.float32))
+    xd = to_dev_bf16(big)[:, 16:80]
+    c = torch.empty((48, 32), dtype=torch.uint8, device="cuda")
+    s = torch.empty((3, 4), dtype=torch.uint8, device="cuda")
+    rc = cuda_lib.load().fourtune_quantize_block16(
+        ctypes.c_void_p(xd.data_ptr()), 48, 64, 96, ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(s.data_ptr()),
+        None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    rc_, rs_ = block16.quantize(np.ascontiguousarray(big[:, 16:80]))
+    np.testing.assert_array_equal(s.cpu().numpy(), rs_)
+    np.testing.assert_array_equal(c.cpu().numpy(), rc_)
