@@ -486,6 +486,43 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   return FT_OK;
 }
 
+int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
+                               uint8_t* codes, uint8_t* scales, ft_bf16* L, void* stream) {
+  if (!X || !W || !codes || !scales || !L) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || M % 16 || K % 32) return FT_ERR_SHAPE;
+  if (R < 16 || R % 16 || R > 128 || M > (1 << 30) || K > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(X) || !al16(W) || !al16(codes) || !al16(L)) return FT_ERR_ALIGN;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  // the same K split as the workspace path, so both compute identical results
+  const RowSplit rs = row_split(M, K, di.num_sms);
+  const size_t header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
+  const size_t need = header + (rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * M * R * 4 : 0);
+  if (need > ft::kRowpassStaticScratchBytes) return FT_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (ft::rowpass_static_scratch(&scratch) != cudaSuccess) return FT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  // status word and split counters must start at zero; the array keeps what the last call left
+  if (cudaMemsetAsync(base, 0, header, s) != cudaSuccess) return FT_ERR_CUDA;
+  CUtensorMap tmX, tmW;
+  if (!map_bf16(&tmX, X, K, M, 128) || !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
+  RowpassParams rp{};
+  rp.M = static_cast<int>(M);
+  rp.K = static_cast<int>(K);
+  rp.R = static_cast<int>(R);
+  rp.kt_per_split = rs.kt_per_split;
+  rp.nsplit = rs.nsplit;
+  rp.codes = codes;
+  rp.scales = scales;
+  rp.L = L;
+  rp.part = reinterpret_cast<float*>(base + header);
+  rp.counters = reinterpret_cast<int*>(base + 16);
+  rp.status = reinterpret_cast<int*>(base);
+  return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
+}
+
 int fourtune_device_status(const void* ws, void* stream) {
   if (!ws) return FT_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

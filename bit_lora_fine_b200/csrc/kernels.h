@@ -68,6 +68,11 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
 cudaError_t launch_tgrad(const CUtensorMap& tmT, const CUtensorMap& tmV, const TgradParams& p,
                          cudaStream_t stream);
 
+// Size of the row pass's file-scope scratch array (allocation-free entry point)
+// and the lookup of its device address on the current device.
+constexpr size_t kRowpassStaticScratchBytes = size_t(16) << 20;
+cudaError_t rowpass_static_scratch(void** out);
+
 // tile sizes the host needs for tensor-map boxes and workspace sizing
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;

@@ -16,6 +16,8 @@
 //   warps 4..7     quantize the same smem tile (one warp per two 16-row blocks),
 //                  then drain the accumulator: L in bf16, or fp32 partials that
 //                  the last CTA of the row tile sums in split order.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -283,6 +285,35 @@ cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const
   if (p.R <= 64) return launch_rowpass_t<64>(tmX, tmW, p, stream);
   if (p.R <= 128) return launch_rowpass_t<128>(tmX, tmW, p, stream);
   return launch_rowpass_t<256>(tmX, tmW, p, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the row pass.  Its split-K partial sums, split
+// counters and status word live in this file-scope device array instead of a
+// caller-provided workspace, for callers that cannot allocate device memory.
+// Every GPU that loads the library holds the array until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_rowpass_static_scratch[kRowpassStaticScratchBytes];
+
+// Device address of the array for the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+cudaError_t rowpass_static_scratch(void** out) {
+  static void* addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_rowpass_static_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace ft

@@ -23,7 +23,8 @@ ERRORS = {0: "FT_OK", -1: "FT_ERR_INVALID_ARG", -2: "FT_ERR_SHAPE", -3: "FT_ERR_
 EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_linear_fwd_workspace_size",
             "fourtune_linear_bwd_workspace_size", "fourtune_linear_fwd", "fourtune_linear_bwd",
             "fourtune_linear_fwd_ws_offsets", "fourtune_linear_bwd_ws_offsets", "fourtune_device_status",
-            "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed")
+            "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed",
+            "fourtune_quant_down_static")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("pack_lowrank", "xpass_quant_down", "gemm_fp4_fwd")
@@ -69,6 +70,7 @@ def load():
     L.fourtune_linear_bwd_timed.argtypes = list(L.fourtune_linear_bwd.argtypes) + [P(vp), ctypes.c_int]
     L.fourtune_linear_fwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz)]
     L.fourtune_linear_bwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz), P(sz)]
+    L.fourtune_quant_down_static.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp, vp]
     L.fourtune_device_status.argtypes = [vp, vp]
     L.fourtune_error_string.argtypes = [ctypes.c_int]
     L.fourtune_error_string.restype = ctypes.c_char_p
@@ -213,6 +215,22 @@ def linear_bwd(layer, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumu
         arr, n = _events(events)
         _check(load().fourtune_linear_bwd_timed(*args, arr, n), "fourtune_linear_bwd_timed")
     return dX, dA, dB, ws
+
+
+def quant_down_static(X, W, codes=None, scales=None, L=None):
+    """Allocation-free fused row pass: block16(X) and L = bf16(X W^T), X [M, K], W [R, K] bf16.
+    The library keeps this call's scratch in a fixed device array (no workspace);
+    overlapping calls race.  Returns (codes, scales, L)."""
+    _need(X, torch.bfloat16, "X")
+    _need(W, torch.bfloat16, "W")
+    M, K = X.shape
+    R = W.shape[0]
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device) if codes is None else codes
+    scales = torch.empty((M // 16, K // 16), dtype=torch.uint8, device=X.device) if scales is None else scales
+    L = torch.empty((M, R), dtype=torch.bfloat16, device=X.device) if L is None else L
+    _check(load().fourtune_quant_down_static(_ptr(X), M, K, _ptr(W), R, _ptr(codes), _ptr(scales), _ptr(L),
+                                             _stream()), "fourtune_quant_down_static")
+    return codes, scales, L
 
 
 def device_status(ws):

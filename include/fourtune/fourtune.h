@@ -143,6 +143,29 @@ FT_API int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, s
 FT_API int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off,
                                    size_t* P_off);
 
+/* Fused row pass without a workspace.  The FourTune paper has no counterpart to
+ * this entry point; it exists for callers that cannot allocate device memory
+ * to hand the library a workspace -- plugin or embedding hosts that own all
+ * device memory and offer no scratch allocator, and runtimes that forbid any
+ * allocation once they have started.  It computes what the forward's first
+ * kernel computes, for any bf16 input X [M, K] and down-projection rows
+ * W [R, K] (bf16, K contiguous; for the layer, W = [S_dn | A]^T):
+ *   codes [M, K/2], scales [M/16, K/16] = block16(X)   and   L [M, R] = bf16(X W^T).
+ * The caller still owns X, W and the outputs.  Scratch (split-K partial sums,
+ * split counters, status word) lives in one device array inside the library,
+ * FT_STATIC_SCRATCH_BYTES (16 MiB) on every GPU that loads the library, kept
+ * until the process exits; no cudaMalloc, cudaFree or other allocation is made.
+ * The first call on a device looks up the array's device address on that
+ * device, so make that first call before any stream capture begins.  Every
+ * call shares the array: calls that overlap on the GPU (other streams, other
+ * host threads) race and corrupt each other's results; serialize them.
+ * Returns FT_ERR_WORKSPACE when the problem needs more scratch than the array
+ * holds (only for M in the millions of tokens), FT_ERR_UNSUPPORTED for R
+ * outside 16..128 (multiples of 16), else as the other calls. */
+#define FT_STATIC_SCRATCH_BYTES (16u << 20)
+FT_API int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
+                                      uint8_t* codes, uint8_t* scales, ft_bf16* L, void* stream);
+
 /* Synchronizes `stream` and returns FT_ERR_TIMEOUT if a kernel of the last call
  * that used `ws` recorded an expired wait, FT_ERR_CUDA on a CUDA error, else FT_OK. */
 FT_API int fourtune_device_status(const void* ws, void* stream);
