@@ -2,8 +2,8 @@
 """Benchmark: FourTune W4A4G4 triple-branch linear, forward + backward, on B200.
 
 One step = fourtune_linear_fwd + fourtune_linear_bwd (every kernel of the hot
-path: pack, fused X pass, FP4 GEMM + up-projection, fused G pass, FP4 dX GEMM,
-dA, dB) on the FLUX-width layer: M = 4608 tokens, K = N = 3072, stabilizer
+path: fused X pass, FP4 GEMM + up-projection, fused G pass, FP4 dX GEMM, dA and
+dB) on the FLUX-width layer: M = 4608 tokens, K = N = 3072, stabilizer
 rank 32, LoRA rank 32, seeded synthetic bf16 data (synth.py).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -49,14 +49,11 @@ def kernel_work(M, K, N, r_s, r):
     """Algorithmic work per launch of each kernel: ('tensor', FLOPs) or ('hbm', bytes)."""
     R = r_s + r
     return {
-        "fwd.pack_lowrank": ("hbm", 2 * 2 * R * (K + N)),
         "fwd.xpass_quant_down": ("hbm", 2 * M * K + M * K // 2 + M * K // 256 + 2 * M * R),
         "fwd.gemm_fp4_fwd": ("tensor", 2 * M * N * K),
-        "bwd.pack_lowrank": ("hbm", 2 * 2 * R * (K + N)),
         "bwd.gpass_quant_down": ("hbm", 2 * M * N + M * N // 2 + M * N // 256 + 2 * M * R),
         "bwd.gemm_fp4_dx": ("tensor", 2 * M * N * K),
-        "bwd.tgrad_dA": ("hbm", 2 * M * K + 2 * M * R + 4 * K * r),
-        "bwd.tgrad_dB": ("hbm", 2 * M * N + 2 * M * R + 4 * N * r),
+        "bwd.tgrad_dA_dB": ("hbm", 2 * M * K + 2 * M * N + 4 * M * R + 4 * (K + N) * r),
     }
 
 

@@ -249,26 +249,40 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
-// E2M1 code of a float, written out from the format's definition: magnitudes
-// 0, .5, 1, 1.5, 2, 3, 4, 6 (codes 0..7), round to nearest with ties to the
-// even code, saturate at 6, sign bit copied from the input (so -0.1 -> 0x8).
-// The tie points are 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5: at a tie the even
-// code wins, hence ">" at ties whose lower neighbour is even and ">=" where
-// the upper one is.
-__device__ __forceinline__ uint32_t f32_to_e2m1(float q) {
-  const float a = fabsf(q);
-  const uint32_t mag = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
-                       static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
-                       static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
-                       static_cast<uint32_t>(a > 5.0f);
-  return mag | ((__float_as_uint(q) >> 28) & 0x8u);
-}
-// eight floats -> 32 bits of E2M1 codes, element i in bits 4i..4i+3
+// eight floats -> 32 bits of E2M1 codes, element i in bits 4i..4i+3: the
+// hardware conversion rounds to nearest even, saturates at +-6 and keeps the
+// sign of zero (the parity tests check every E2M1 tie, both signs, against the
+// oracle's table search)
 __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
-  uint32_t r = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) r |= f32_to_e2m1(v[i]) << (4 * i);
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return r;
+}
+
+// Block16 quantization of 32 consecutive values of one row (two 16-column
+// blocks) given the two block maxima: scale = E4M3(amax / 6), code =
+// E2M1(v / dec(scale)), all +0 when the scale decodes to 0.  Writes four
+// 32-bit words of codes (element i of block j in word 2j + i/8) and the two
+// scale bytes.
+__device__ __forceinline__ void quantize_2blocks(const float* v, const float* amax, uint32_t* packed,
+                                                 uint32_t* sc) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
+    const float d = e4m3_to_f32(sc[j]);
+    float q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + e], d);
+    packed[2 * j] = f32x8_to_e2m1(q);
+    packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
+  }
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }

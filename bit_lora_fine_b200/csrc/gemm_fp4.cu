@@ -5,21 +5,23 @@
 // is fused with the stabilizer/LoRA up-projection, since the branch outputs are
 // summed anyway.  §3.2: the backward dX product reads the weight blocks
 // transposed with the same codes and scales -- here the B operand is the
-// nibble-transposed copy of R's codes and the scale of (row, k-group) is looked
-// up with swapped strides in R's own [N/16, K/16] scale array.
+// nibble-transposed copy of R's codes and the scale of (row, k-group) is read
+// transposed from R's own [N/16, K/16] scale array.
 //
 //   out[m, n] = sum_k deq(A)[m, k] deq(B)[n, k]  (+ sum_j A2[m, j] B2[n, j])  (+ bias[n])
 //
 // CTA tile 128 x BN (BN = 256), K-block = 256 FP4 elements (one 128-byte
 // swizzle row per operand row).  Warp roles:
-//   warp 0 lane 0  TMA: A codes [128 x 128 B], B codes [BN x 128 B]; for the bf16
-//                  extra blocks A2 [128 x 64] and B2 [BN x 64] into the same slots
+//   warp 0 lane 0  TMA: A codes [128 x 128 B], B codes [BN x 128 B] and the
+//                  K-block's compact 16x16 scale tiles; for the bf16 extra
+//                  blocks A2 [128 x 64] and B2 (K-major [BN x 64] or MN-major
+//                  [64 x BN] in four boxes) into the same slots
 //   warp 1         TMEM owner; lane 0 copies the stage's scale vectors smem->TMEM
 //                  (tcgen05.cp 32x128b.warpx4) and issues
 //                  tcgen05.mma kind::mxf4nvf4.block_scale.block16 (M=128, N=BN,
 //                  K=64) x 4 per K-block, then kind::f16 for the extra blocks
-//   warp 2         expands the compact 16x16 scales of the K-block into the
-//                  per-row layout the MMA reads (one 16-byte pattern per 16 rows)
+//   warp 2         expands the compact scales into the per-row layout the MMA
+//                  reads (one 16-byte pattern per 16 rows)
 //   warps 4..7     epilogue: TMEM -> registers -> + bias -> fp32/bf16 stores
 #include "common.cuh"
 #include "kernels.h"
@@ -37,7 +39,10 @@ struct GemmLayout {
   static constexpr uint32_t kSFA = 4 * 512;                  // 4 MMA K-steps x 512 B
   static constexpr uint32_t kSFB = 4 * kNC * 512;
   static constexpr uint32_t kStage = kA + kB + kSFA + kSFB;  // multiple of 1024
-  static constexpr uint32_t kSmem = 1024 + kGmStages * kStage + 256;
+  static constexpr uint32_t kCA = 8 * 16;                    // compact A scales: 8 row-blocks x 16 groups
+  static constexpr uint32_t kCB = (BN / 16) * 16;            // compact B scales: BN/16 row-blocks x 16 groups
+  static constexpr uint32_t kCStage = kCA + kCB;
+  static constexpr uint32_t kSmem = 1024 + kGmStages * (kStage + kCStage) + 256;
   // TMEM columns: accumulator, then per stage 16 (SFA) + 16*kNC (SFB)
   static constexpr uint32_t kSfColsPerStage = 16 + 16 * kNC;
   static constexpr uint32_t kTmemUsed = BN + kGmStages * kSfColsPerStage;
@@ -48,14 +53,17 @@ template <int BN>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const GemmParams p) {
   using Lay = GemmLayout<BN>;
   static_assert(Lay::kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(Lay::kTmemUsed <= 512, "TMEM budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGmStages * Lay::kStage);
-  uint64_t* empty = full + kGmStages;
+  uint8_t* compact = smem + kGmStages * Lay::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(compact + kGmStages * Lay::kCStage);
+  uint64_t* sf_ready = full + kGmStages;
+  uint64_t* empty = sf_ready + kGmStages;
   uint64_t* acc_full = empty + kGmStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -72,8 +80,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGmStages; ++s) {
-      mbar_init(&full[s], 2);   // producer (expect_tx) + scale stager
-      mbar_init(&empty[s], 1);  // MMA commit
+      mbar_init(&full[s], 1);      // producer (expect_tx)
+      mbar_init(&sf_ready[s], 1);  // scale stager
+      mbar_init(&empty[s], 1);     // MMA commit
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -90,6 +99,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       tma_prefetch(&tmA2);
       tma_prefetch(&tmB2);
     }
+    if (p.sf_tma) {
+      tma_prefetch(&tmSFA);
+      tma_prefetch(&tmSFB);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -104,13 +117,28 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         const uint32_t ph = (i / kGmStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
         uint8_t* st = smem + s * Lay::kStage;
-        mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
         if (i < KB) {
+          mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + (p.sf_tma ? Lay::kCStage : 0u));
           tma_load_2d(st, &tmA, &full[s], i * 128, m0);
           tma_load_2d(st + Lay::kA, &tmB, &full[s], i * 128, n0);
+          if (p.sf_tma) {
+            uint8_t* cs = compact + s * Lay::kCStage;
+            tma_load_2d(cs, &tmSFA, &full[s], i * 16, m0 / 16);
+            if (p.sfb_transposed)
+              tma_load_2d(cs + Lay::kCA, &tmSFB, &full[s], n0 / 16, i * 16);
+            else
+              tma_load_2d(cs + Lay::kCA, &tmSFB, &full[s], i * 16, n0 / 16);
+          }
         } else {
-          tma_load_2d(st, &tmA2, &full[s], (i - KB) * 64, m0);
-          tma_load_2d(st + Lay::kA, &tmB2, &full[s], (i - KB) * 64, n0);
+          const int e = i - KB;
+          mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
+          tma_load_2d(st, &tmA2, &full[s], e * 64, m0);
+          if (p.b2_mn_major) {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) tma_load_2d(st + Lay::kA + 8192 * c, &tmB2, &full[s], n0 + 64 * c, e * 64);
+          } else {
+            tma_load_2d(st + Lay::kA, &tmB2, &full[s], e * 64, n0);
+          }
         }
         issued = i + 1;
       }
@@ -122,11 +150,12 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc4 = idesc_fp4_block16(128, BN);
-      const uint32_t idesc16 = idesc_bf16(128, BN, false, false);
+      const uint32_t idesc16 = idesc_bf16(128, BN, false, p.b2_mn_major != 0);
       for (int i = 0; i < T; ++i) {
         const int s = i % kGmStages;
         const uint32_t ph = (i / kGmStages) & 1;
         if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
+        if (!mbar_wait(&sf_ready[s], ph, p.status, abortp)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + s * Lay::kStage);
         const uint32_t b_addr = a_addr + Lay::kA;
@@ -149,8 +178,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                             (i | t) != 0 ? 1u : 0u);
         } else {
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-            mma_bf16(tmem, desc_kmajor_sw128(a_addr + 32 * t), desc_kmajor_sw128(b_addr + 32 * t), idesc16, 1u);
+          for (int t = 0; t < 4; ++t) {
+            const uint64_t bdesc =
+                p.b2_mn_major ? desc_mnmajor_sw128(b_addr + 2048 * t, 8192) : desc_kmajor_sw128(b_addr + 32 * t);
+            mma_bf16(tmem, desc_kmajor_sw128(a_addr + 32 * t), bdesc, idesc16, 1u);
+          }
         }
         tc_commit(&empty[s]);
       }
@@ -171,38 +203,52 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const uint32_t ph = (i / kGmStages) & 1;
       if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
       if (i < KB) {
+        if (p.sf_tma && !mbar_wait(&full[s], ph, p.status, abortp)) break;
         uint8_t* sfa = smem + s * Lay::kStage + Lay::kA + Lay::kB;
         uint8_t* sfb = sfa + Lay::kSFA;
+        const uint8_t* cA = compact + s * Lay::kCStage;
+        const uint8_t* cB = cA + Lay::kCA;
         if (lane < nA + nB) {
           const bool isA = lane < nA;
           const int idx = isA ? lane : lane - nA;
           const int hh = idx & 1;
-          int t, c;
-          if (isA) {
-            t = idx >> 1;
-            c = 0;
-          } else {
-            t = idx / (2 * Lay::kNC);
-            c = (idx >> 1) % Lay::kNC;
-          }
-          const uint8_t* src = isA ? p.sfa : p.sfb;
-          const long long rs = isA ? p.sfa_rs : p.sfb_rs;
-          const long long gs = isA ? p.sfa_gs : p.sfb_gs;
-          const int rb0 = (isA ? m0 : n0 + 128 * c) / 16 + hh;
-          const int nrb = isA ? Mb : Nb;
-          const int g0 = i * 16 + t * 4;
+          const int t = isA ? idx >> 1 : idx / (2 * Lay::kNC);
+          const int c = isA ? 0 : (idx >> 1) % Lay::kNC;
           uint32_t word[4];
+          if (p.sf_tma) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int rb = rb0 + 2 * w;
-            uint32_t wv = 0;
+            for (int w = 0; w < 4; ++w) {
+              const int rb = c * 8 + hh + 2 * w;   // row-block within the tile
+              if (isA) {
+                word[w] = *reinterpret_cast<const uint32_t*>(cA + rb * 16 + 4 * t);
+              } else if (!p.sfb_transposed) {
+                word[w] = *reinterpret_cast<const uint32_t*>(cB + rb * 16 + 4 * t);
+              } else {
+                uint32_t wv = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int g = g0 + j;
-              const uint32_t b = (rb < nrb && g < KG) ? src[rb * rs + g * gs] : 0u;
-              wv |= b << (8 * j);
+                for (int j = 0; j < 4; ++j) wv |= static_cast<uint32_t>(cB[(4 * t + j) * 16 + rb]) << (8 * j);
+                word[w] = wv;
+              }
             }
-            word[w] = wv;
+          } else {
+            const uint8_t* src = isA ? p.sfa : p.sfb;
+            const long long rs = isA ? p.sfa_rs : p.sfb_rs;
+            const long long gs = isA ? p.sfa_gs : p.sfb_gs;
+            const int rb0 = (isA ? m0 : n0 + 128 * c) / 16 + hh;
+            const int nrb = isA ? Mb : Nb;
+            const int g0 = i * 16 + t * 4;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int rb = rb0 + 2 * w;
+              uint32_t wv = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int g = g0 + j;
+                const uint32_t b = (rb < nrb && g < KG) ? src[rb * rs + g * gs] : 0u;
+                wv |= b << (8 * j);
+              }
+              word[w] = wv;
+            }
           }
           const uint4 pat = make_uint4(word[0], word[1], word[2], word[3]);
           uint8_t* chunk = isA ? sfa + t * 512 : sfb + (t * Lay::kNC + c) * 512;
@@ -213,7 +259,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full[s]);
+      if (lane == 0) mbar_arrive(&sf_ready[s]);
     }
   } else if (warp >= 4) {
     if (mbar_wait(acc_full, 0, p.status, abortp)) {
@@ -276,14 +322,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 }
 
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
-                            const CUtensorMap& tmB2, const GemmParams& p, cudaStream_t stream) {
+                            const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
+                            const GemmParams& p, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
   using Lay = GemmLayout<BN>;
   cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Lay::kSmem));
   if (e != cudaSuccess) return e;
   dim3 grid((p.N + BN - 1) / BN, (p.M + 127) / 128);
-  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, p);
+  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, tmSFA, tmSFB, p);
   return cudaGetLastError();
 }
 

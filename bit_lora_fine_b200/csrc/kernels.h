@@ -7,18 +7,12 @@
 
 namespace ft {
 
-struct PackParams {
-  int K, N, r_s, r;
-  const void *S_dn, *A, *S_up, *B;      // bf16, row-major [K,r_s] [K,r] [r_s,N] [r,N]
-  uint16_t *Dt, *Dcat, *Ut, *Ucat;      // outputs, any may be null
-  int* zero_words;                       // status word + split counters, cleared first
-  long long n_zero_words;
-};
-
 // Quantize the rows of a bf16 input and project it onto R low-rank directions:
-// codes/scales = block16(X), L = bf16(X * W^T) with W^T given as a [R, K] map.
+// codes/scales = block16(X), L = bf16(X W) where W is either D [K, R] (R
+// contiguous, read MN-major) or W^T [R, K] (K contiguous, read K-major).
 struct RowpassParams {
   int M, K, R;
+  int w_mn_major;                        // 1: D [K, R]; 0: W^T [R, K]
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
@@ -28,11 +22,16 @@ struct RowpassParams {
   int* status;
 };
 
-// out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1 with
-// scale(row, g) = sf[(row/16)*rs + g*gs], g the 16-wide K group; A2 [M, R2],
-// B2 [N, R2] bf16.
+// out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1.
+// Scales: with sf_tma the compact [rows/16, K/16] tiles come by TMA (B's read
+// transposed when sfb_transposed: B's scale(row, g) = array[g, row/16]);
+// otherwise scale(row, g) = sf[(row/16)*rs + g*gs] by plain loads.
+// A2 [M, R2] bf16; B2 is [N, R2] (K-major) or U [R2, N] (b2_mn_major).
 struct GemmParams {
   int M, N, K, R2;
+  int b2_mn_major;
+  int sf_tma;
+  int sfb_transposed;
   const uint8_t* sfa;
   long long sfa_rs, sfa_gs;
   const uint8_t* sfb;
@@ -52,7 +51,7 @@ struct TgradParams {
   long long out_sp, out_sj;
   int accumulate;
   float* part;                           // fp32 [nsplit, ceil(P/128)*128, 64] when nsplit > 1
-  int* counters;                         // [ceil(P/128)]
+  int* counters;                         // [ceil(P/128)], zero on entry, left zero
   int* status;
 };
 
@@ -60,13 +59,15 @@ cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long
                                     uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uint8_t* codes_t,
                                    cudaStream_t stream);
-cudaError_t launch_pack_lowrank(const PackParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream);
+int rowpass_ctas_per_sm(int R, int w_mn_major);
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
-                            const CUtensorMap& tmB2, const GemmParams& p, cudaStream_t stream);
-cudaError_t launch_tgrad(const CUtensorMap& tmT, const CUtensorMap& tmV, const TgradParams& p,
-                         cudaStream_t stream);
+                            const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
+                            const GemmParams& p, cudaStream_t stream);
+cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
+                          const CUtensorMap& tmT1, const CUtensorMap& tmV1, const TgradParams& p1,
+                          cudaStream_t stream);
 
 // Size of the row pass's file-scope scratch array (allocation-free entry point)
 // and the lookup of its device address on the current device.
@@ -76,6 +77,5 @@ cudaError_t rowpass_static_scratch(void** out);
 // tile sizes the host needs for tensor-map boxes and workspace sizing
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
-constexpr int kRowTile = 128;
 
 }  // namespace ft

@@ -81,21 +81,16 @@ __global__ void __launch_bounds__(256) quantize_block16_kernel(const __nv_bfloat
     amax[j] = a;
   }
 
+  if (nblk == 0) return;
+  uint32_t packed[4], sc[2];
+  quantize_2blocks(v, amax, packed, sc);
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     if (j >= nblk) break;
-    const float s = __fdiv_rn(amax[j], 6.0f);
-    const uint32_t sc = f32_to_e4m3(s);
-    const float d = e4m3_to_f32(sc);
-    float q[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + i], d);
-    uint2 packed;
-    packed.x = f32x8_to_e2m1(q);
-    packed.y = f32x8_to_e2m1(q + 8);
     const int cb = cstart + 16 * j;
-    *reinterpret_cast<uint2*>(codes + static_cast<long long>(r) * (cols / 2) + cb / 2) = packed;
-    if ((lane >> 1) == 0) scales[static_cast<long long>(rb) * (cols / 16) + cb / 16] = static_cast<uint8_t>(sc);
+    *reinterpret_cast<uint2*>(codes + static_cast<long long>(r) * (cols / 2) + cb / 2) =
+        make_uint2(packed[2 * j], packed[2 * j + 1]);
+    if ((lane >> 1) == 0) scales[static_cast<long long>(rb) * (cols / 16) + cb / 16] = static_cast<uint8_t>(sc[j]);
   }
 }
 

@@ -8,14 +8,18 @@
 // (P = G [S_up; B]^T).
 //
 // CTA = 128 rows x a contiguous range of 64-column tiles (split-K when M alone
-// gives too few CTAs).  Warp roles:
-//   warp 0 lane 0  TMA producer: X tile [128 x 64] bf16 and W tile [R x 64] bf16
-//                  (both 128-byte rows, 128-byte swizzle) into a 4-stage ring
-//   warp 1         TMEM owner; lane 0 issues tcgen05.mma kind::f16
-//                  (M=128, N=R, K=16) x 4 per tile, fp32 accumulator in TMEM
-//   warps 4..7     quantize the same smem tile (one warp per two 16-row blocks),
-//                  then drain the accumulator: L in bf16, or fp32 partials that
-//                  the last CTA of the row tile sums in split order.
+// gives too few CTAs; two CTAs fit on an SM for R <= 64).  Warp roles:
+//   warp 0 lane 0  TMA producer: input tile [128 x 64] bf16 (128-byte rows,
+//                  128-byte swizzle) and the projection tile, into a 4-stage ring
+//   warp 1         TMEM owner; lane 0 issues tcgen05.mma kind::f16 (M=128,
+//                  N=R rounded as below, K=16) x 4 per tile into TMEM
+//   warps 4..11    each quantizes one 16-row block of the same smem tile, then
+//                  the eight drain the accumulator (two warps per TMEM lane
+//                  quadrant): L in bf16, or fp32 partials that the last CTA of
+//                  the row tile sums in split order (deterministic).
+// The projection matrix is read either K-major (W^T [R, K], rows of 128 bytes,
+// N = R) or MN-major (D [K, R] with R contiguous: TMA boxes of 64 k-rows x 64
+// r, N = R rounded up to 64, the extra columns zero-filled by the TMA).
 #include <mutex>
 
 #include "common.cuh"
@@ -24,12 +28,21 @@
 namespace ft {
 
 constexpr int kRpStages = 4;
-constexpr int kRpThreads = 256;
+constexpr int kRpThreads = 384;
+constexpr int kRpQuantWarps = 8;
 constexpr uint32_t kRpXBytes = 128 * 128;  // 128 rows x 64 bf16
 
-__host__ __device__ constexpr uint32_t rp_w_bytes_padded(int R) { return ((R * 128) + 1023u) & ~1023u; }
-__host__ __device__ constexpr uint32_t rp_stage_bytes(int R) { return kRpXBytes + rp_w_bytes_padded(R); }
-__host__ __device__ constexpr uint32_t rp_smem_bytes(int R) { return 1024 + kRpStages * rp_stage_bytes(R) + 256; }
+__host__ __device__ constexpr int rp_mn_chunks(int R) { return (R + 63) / 64; }
+__host__ __device__ constexpr int rp_n_mma(int R, int mn) { return mn ? 64 * rp_mn_chunks(R) : R; }
+__host__ __device__ constexpr uint32_t rp_w_bytes(int R, int mn) {
+  return mn ? 8192u * rp_mn_chunks(R) : static_cast<uint32_t>(R) * 128u;
+}
+__host__ __device__ constexpr uint32_t rp_stage_bytes(int R, int mn) {
+  return kRpXBytes + ((rp_w_bytes(R, mn) + 1023u) & ~1023u);
+}
+__host__ __device__ constexpr uint32_t rp_smem_bytes(int R, int mn) {
+  return 1024 + kRpStages * rp_stage_bytes(R, mn) + 256;
+}
 
 template <int RCOLS>
 __global__ void __launch_bounds__(kRpThreads, 1)
@@ -38,15 +51,17 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int R = p.R;
-  const uint32_t w_bytes = static_cast<uint32_t>(R) * 128;
-  const uint32_t stage_bytes = rp_stage_bytes(R);
+  const int mn = p.w_mn_major;
+  const int nmma = rp_n_mma(R, mn);
+  const uint32_t w_bytes = rp_w_bytes(R, mn);
+  const uint32_t stage_bytes = rp_stage_bytes(R, mn);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRpStages * stage_bytes);
   uint64_t* empty = full + kRpStages;
   uint64_t* acc_full = empty + kRpStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
-  volatile int* s_ok = s_last + 1;  // [4]
+  volatile int* s_ok = s_last + 1;  // [kRpQuantWarps]
   volatile int* abortp = abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -60,7 +75,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRpStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrive per quantizer warp
+      mbar_init(&empty[s], 1 + kRpQuantWarps);  // MMA commit + one arrive per quantizer warp
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -87,9 +102,15 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         const uint32_t ph = (i / kRpStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
         uint8_t* st = smem + s * stage_bytes;
+        const int kc = (kt0 + i) * 64;
         mbar_arrive_expect_tx(&full[s], kRpXBytes + w_bytes);
-        tma_load_2d(st, &tmX, &full[s], (kt0 + i) * 64, m0);
-        tma_load_2d(st + kRpXBytes, &tmW, &full[s], (kt0 + i) * 64, 0);
+        tma_load_2d(st, &tmX, &full[s], kc, m0);
+        if (mn) {
+          for (int c = 0; c < rp_mn_chunks(R); ++c)
+            tma_load_2d(st + kRpXBytes + 8192 * c, &tmW, &full[s], 64 * c, kc);
+        } else {
+          tma_load_2d(st + kRpXBytes, &tmW, &full[s], kc, 0);
+        }
         issued = i + 1;
       }
       if (*abortp) {  // let copies already in flight land before the CTA exits
@@ -99,7 +120,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, R, false, false);
+      const uint32_t idesc = idesc_bf16(128, nmma, false, mn != 0);
       for (int i = 0; i < nt; ++i) {
         const int s = i % kRpStages;
         const uint32_t ph = (i / kRpStages) & 1;
@@ -108,21 +129,24 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         const uint32_t xa = smem_u32(smem + s * stage_bytes);
         const uint32_t wa = xa + kRpXBytes;
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          mma_bf16(tmem, desc_kmajor_sw128(xa + 32 * t), desc_kmajor_sw128(wa + 32 * t), idesc,
-                   (i | t) != 0 ? 1u : 0u);
+        for (int t = 0; t < 4; ++t) {
+          const uint64_t bdesc = mn ? desc_mnmajor_sw128(wa + 2048 * t, 8192) : desc_kmajor_sw128(wa + 32 * t);
+          mma_bf16(tmem, desc_kmajor_sw128(xa + 32 * t), bdesc, idesc, (i | t) != 0 ? 1u : 0u);
+        }
         tc_commit(&empty[s]);
       }
       tc_commit(acc_full);
       mbar_wait_drain(acc_full, 0, kWaitLimitNs);  // every MMA done before TMEM can be freed
     }
   } else if (warp >= 4) {
-    const int w4 = warp - 4;
-    const int h = lane & 1;
+    const int w8 = warp - 4;        // 16-row block of the tile this warp quantizes
+    const int h = lane & 1;         // 32-column half of the 64-column tile
+    const int r = w8 * 16 + (lane >> 1);
     const long long half_k = p.K / 2;
     const int kblocks = p.K / 16;
+    const bool block_row_ok = m0 + w8 * 16 < p.M;
     bool ok = true;
-    for (int i = 0; i < nt && ok; ++i) {
+    for (int i = 0; i < nt; ++i) {
       const int s = i % kRpStages;
       const uint32_t ph = (i / kRpStages) & 1;
       if (!mbar_wait(&full[s], ph, p.status, abortp)) {
@@ -130,75 +154,61 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         break;
       }
       const uint8_t* tile = smem + s * stage_bytes;
-      const int kcol0 = (kt0 + i) * 64;
+      float v[32];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int rbl = 2 * w4 + rr;
-        const int r = rbl * 16 + (lane >> 1);
-        float v[32];
+      for (int q = 0; q < 4; ++q) {
+        const int phys = (4 * h + q) ^ (r & 7);
+        const uint4 u = *reinterpret_cast<const uint4*>(tile + r * 128 + phys * 16);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int phys = (4 * h + q) ^ (r & 7);
-          const uint4 u = *reinterpret_cast<const uint4*>(tile + r * 128 + phys * 16);
-          const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[q * 8 + 2 * e] = bf16_bits_to_f32(wd[e] & 0xFFFFu);
-            v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
-          }
-        }
-        float amax[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          float a = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(v[16 * j + e]));
-#pragma unroll
-          for (int off = 2; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-          amax[j] = a;
-        }
-        const int cstart = kcol0 + 32 * h;
-        if (m0 + rbl * 16 < p.M && cstart < p.K) {
-          uint32_t packed[4];
-          uint32_t sc[2];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
-            const float d = e4m3_to_f32(sc[j]);
-            float q[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + e], d);
-            packed[2 * j] = f32x8_to_e2m1(q);
-            packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
-          }
-          const long long grow = m0 + r;
-          *reinterpret_cast<uint4*>(p.codes + grow * half_k + cstart / 2) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          if ((lane >> 1) == 0) {
-            const long long srow = (m0 / 16 + rbl) * static_cast<long long>(kblocks);
-            p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
-            p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          v[q * 8 + 2 * e] = bf16_bits_to_f32(wd[e] & 0xFFFFu);
+          v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
+      float amax[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(v[16 * j + e]));
+#pragma unroll
+        for (int off = 2; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        amax[j] = a;
+      }
+      const int cstart = (kt0 + i) * 64 + 32 * h;
+      if (block_row_ok && cstart < p.K) {
+        uint32_t packed[4], sc[2];
+        quantize_2blocks(v, amax, packed, sc);
+        *reinterpret_cast<uint4*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        if ((lane >> 1) == 0) {
+          const long long srow = (m0 / 16 + w8) * static_cast<long long>(kblocks);
+          p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
+          p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
+        }
+      }
     }
 
-    // ---- epilogue: accumulator -> L (bf16) or fp32 partials.  The four warps
+    // ---- epilogue: accumulator -> L (bf16) or fp32 partials.  All eight warps
     // agree on whether to run it, so the named barriers below are always
     // reached by all of them.
-    bool mine = ok && mbar_wait(acc_full, 0, p.status, abortp);
-    if (lane == 0) s_ok[w4] = mine ? 1 : 0;
-    named_bar_sync(1, 128);
-    const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
+    const bool mine = ok && mbar_wait(acc_full, 0, p.status, abortp);
+    if (lane == 0) s_ok[w8] = mine ? 1 : 0;
+    named_bar_sync(1, 32 * kRpQuantWarps);
+    bool go = true;
+#pragma unroll
+    for (int w = 0; w < kRpQuantWarps; ++w) go = go && s_ok[w];
     if (go) {
       tc_fence_after();
-      const int q = warp & 3;
+      const int q = warp & 3;                       // TMEM lane quadrant of this warp
       const int row = m0 + 32 * q + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
       const bool row_ok = row < p.M;
-      for (int c0 = 0; c0 < R; c0 += 16) {
+      const int half = (warp - 4) >> 2;             // which 16-column chunks this warp drains
+      for (int c0 = 16 * half; c0 < R; c0 += 32) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(taddr + c0, v);
         tmem_ld_wait();
@@ -224,21 +234,22 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       if (p.nsplit > 1) {
         // the last CTA of this row tile to finish sums every split's partial, in split order
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kRpQuantWarps);
         if (threadIdx.x == 128) {
           const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
           *s_last = (prev == p.nsplit - 1);
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kRpQuantWarps);
         if (*s_last) {
           __threadfence();
           if (row_ok) {
-            for (int c0 = 0; c0 < R; c0 += 8) {
+            for (int c0 = 8 * half; c0 < R; c0 += 16) {
               float acc[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
               for (int sp = 0; sp < p.nsplit; ++sp) {
-                const float4* src = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * p.M + row) * R + c0);
+                const float4* src =
+                    reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * p.M + row) * R + c0);
                 const float4 a = __ldcg(src), b = __ldcg(src + 1);
                 acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
                 acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
 template <int RCOLS>
 static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                                     cudaStream_t stream) {
-  const uint32_t smem = rp_smem_bytes(p.R);
+  const uint32_t smem = rp_smem_bytes(p.R, p.w_mn_major);
   cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -281,10 +292,14 @@ static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& t
 
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream) {
-  if (p.R <= 32) return launch_rowpass_t<32>(tmX, tmW, p, stream);
-  if (p.R <= 64) return launch_rowpass_t<64>(tmX, tmW, p, stream);
-  if (p.R <= 128) return launch_rowpass_t<128>(tmX, tmW, p, stream);
-  return launch_rowpass_t<256>(tmX, tmW, p, stream);
+  const int n = rp_n_mma(p.R, p.w_mn_major);
+  if (n <= 32) return launch_rowpass_t<32>(tmX, tmW, p, stream);
+  if (n <= 64) return launch_rowpass_t<64>(tmX, tmW, p, stream);
+  return launch_rowpass_t<128>(tmX, tmW, p, stream);
+}
+
+int rowpass_ctas_per_sm(int R, int w_mn_major) {
+  return rp_smem_bytes(R, w_mn_major) * 2 <= 227u * 1024u ? 2 : 1;
 }
 
 // ---------------------------------------------------------------------------

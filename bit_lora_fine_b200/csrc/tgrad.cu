@@ -5,12 +5,13 @@
 // P = G [S_up ; B]^T saved in bf16:
 //   dA = X^T P[:, r_s:]   (T = X,  V = P, out [K, r] row-major)
 //   dB = L[:, r_s:]^T G   (T = G,  V = L, out [r, N] row-major, written as dB^T)
-// Both are reductions over the M tokens of a tall bf16 matrix against a thin
-// one: HBM-bound (T is read once).  The tensor cores take both operands
-// MN-major straight from the TMA tiles: T tile [128 m x 128 p] (two 128-byte
-// swizzled boxes of 64 p), V tile [128 m x 64 j]; tcgen05.mma kind::f16
-// M=128 (p), N=64 (j), K=16 (m), 8 per tile.  CTAs split M; the last CTA of a
-// p-tile sums the fp32 partials in split order (deterministic).
+// Both problems run in one launch (the CTA index selects the problem).  Each is
+// a reduction over the M tokens of a tall bf16 matrix against a thin one:
+// HBM-bound (T is read once).  The tensor cores take both operands MN-major
+// straight from the TMA tiles: T tile [128 m x 128 p] (two 128-byte swizzled
+// boxes of 64 p), V tile [128 m x 64 j]; tcgen05.mma kind::f16 M=128 (p),
+// N=64 (j), K=16 (m), 8 per tile.  CTAs split M; the last CTA of a p-tile sums
+// the fp32 partials in split order (deterministic).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,8 +24,9 @@ constexpr uint32_t kTgStage = 2 * kTgTBox + kTgTBox;  // T (two boxes) + V
 constexpr uint32_t kTgSmem = 1024 + kTgStages * kTgStage + 256;
 
 __global__ void __launch_bounds__(kTgThreads, 1)
-    tgrad_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmV,
-                 const TgradParams p) {
+    tgrad_kernel(const __grid_constant__ CUtensorMap tmT0, const __grid_constant__ CUtensorMap tmV0,
+                 const __grid_constant__ CUtensorMap tmT1, const __grid_constant__ CUtensorMap tmV1,
+                 const TgradParams p0, const TgradParams p1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTgStages * kTgStage);
@@ -33,11 +35,21 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
+  volatile int* s_ok = s_last + 1;  // [4]
   volatile int* abortp = abort_flag;
 
+  // which problem and tile this CTA owns
+  const int tiles0 = ((p0.P + 127) / 128) * p0.nsplit;
+  const bool second = static_cast<int>(blockIdx.x) >= tiles0;
+  const TgradParams& p = second ? p1 : p0;
+  const CUtensorMap* tmT = second ? &tmT1 : &tmT0;
+  const CUtensorMap* tmV = second ? &tmV1 : &tmV0;
+  const int local = second ? static_cast<int>(blockIdx.x) - tiles0 : static_cast<int>(blockIdx.x);
+  const int ptile = local / p.nsplit;
+  const int split = local % p.nsplit;
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p0 = blockIdx.x * 128;
-  const int split = blockIdx.y;
+  const int pbase = ptile * 128;
   const int MT = (p.M + 127) / 128;
   const int mt0 = split * p.mt_per_split;
   const int mt1 = min(MT, mt0 + p.mt_per_split);
@@ -58,8 +70,8 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch(&tmT);
-    tma_prefetch(&tmV);
+    tma_prefetch(tmT);
+    tma_prefetch(tmV);
   }
   tc_fence_before();
   __syncthreads();
@@ -76,9 +88,9 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         uint8_t* st = smem + s * kTgStage;
         const int my = (mt0 + i) * 128;
         mbar_arrive_expect_tx(&full[s], kTgStage);
-        tma_load_2d(st, &tmT, &full[s], p0, my);
-        tma_load_2d(st + kTgTBox, &tmT, &full[s], p0 + 64, my);
-        tma_load_2d(st + 2 * kTgTBox, &tmV, &full[s], p.v0, my);
+        tma_load_2d(st, tmT, &full[s], pbase, my);
+        tma_load_2d(st + kTgTBox, tmT, &full[s], pbase + 64, my);
+        tma_load_2d(st + 2 * kTgTBox, tmV, &full[s], p.v0, my);
         issued = i + 1;
       }
       if (*abortp) {
@@ -107,16 +119,15 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     }
   } else if (warp >= 4) {
     const bool mine = (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
-    if (lane == 0) s_last[1 + (warp - 4)] = mine ? 1 : 0;
+    if (lane == 0) s_ok[warp - 4] = mine ? 1 : 0;
     named_bar_sync(1, 128);
-    const volatile int* ok4 = s_last + 1;
-    const bool go = ok4[0] && ok4[1] && ok4[2] && ok4[3];
+    const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
     if (go) {
       tc_fence_after();
       const int q = warp & 3;
-      const int prow = p0 + 32 * q + lane;
+      const int prow = pbase + 32 * q + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      uint32_t v[64];
+      float acc[64];
       {
         uint32_t a[32], b[32];
         tmem_ld_32x32b_x32(taddr, a);
@@ -124,44 +135,49 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          v[e] = a[e];
-          v[32 + e] = b[e];
+          acc[e] = __uint_as_float(a[e]);
+          acc[32 + e] = __uint_as_float(b[e]);
         }
       }
-      const bool prow_ok = prow < p.P;
-      if (p.nsplit == 1) {
-        if (prow_ok) {
-          for (int j = 0; j < p.r; ++j) {
-            float* o = p.out + prow * p.out_sp + j * p.out_sj;
-            const float val = __uint_as_float(v[j]);
-            *o = p.accumulate ? *o + val : val;
-          }
-        }
-      } else {
+      bool write = true;
+      if (p.nsplit > 1) {
         float4* dst = reinterpret_cast<float4*>(p.part + (static_cast<long long>(split) * Ppad + prow) * 64);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
-                               __uint_as_float(v[4 * e + 3]));
+        for (int e = 0; e < 16; ++e) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
         __threadfence();
         named_bar_sync(1, 128);
         if (threadIdx.x == 128) {
-          const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
+          const int prev = atomicAdd(&p.counters[ptile], 1);
           *s_last = (prev == p.nsplit - 1);
         }
         named_bar_sync(1, 128);
-        if (*s_last) {
+        write = *s_last != 0;
+        if (write) {
+          // sum every split's partial row in split order (vector loads, registers only)
           __threadfence();
-          if (prow_ok) {
-            for (int j = 0; j < p.r; ++j) {
-              float acc = 0.0f;
-              for (int sp = 0; sp < p.nsplit; ++sp)
-                acc += __ldcg(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64 + j);
-              float* o = p.out + prow * p.out_sp + j * p.out_sj;
-              *o = p.accumulate ? *o + acc : acc;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+          for (int sp = 0; sp < p.nsplit; ++sp) {
+            const float4* src = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float4 x = __ldcg(src + e);
+              acc[4 * e] += x.x;
+              acc[4 * e + 1] += x.y;
+              acc[4 * e + 2] += x.z;
+              acc[4 * e + 3] += x.w;
             }
           }
-          if (threadIdx.x == 128) p.counters[blockIdx.x] = 0;
+          if (threadIdx.x == 128) p.counters[ptile] = 0;
+        }
+      }
+      if (write && prow < p.P) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          if (j < p.r) {
+            float* o = p.out + prow * p.out_sp + j * p.out_sj;
+            *o = p.accumulate ? *o + acc[j] : acc[j];
+          }
         }
       }
     }
@@ -175,12 +191,15 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   }
 }
 
-cudaError_t launch_tgrad(const CUtensorMap& tmT, const CUtensorMap& tmV, const TgradParams& p, cudaStream_t stream) {
+cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
+                          const CUtensorMap& tmT1, const CUtensorMap& tmV1, const TgradParams& p1,
+                          cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(tgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTgSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid((p.P + 127) / 128, p.nsplit);
-  tgrad_kernel<<<grid, kTgThreads, kTgSmem, stream>>>(tmT, tmV, p);
+  const int tiles0 = ((p0.P + 127) / 128) * p0.nsplit;
+  const int tiles1 = ((p1.P + 127) / 128) * p1.nsplit;
+  tgrad_kernel<<<tiles0 + tiles1, kTgThreads, kTgSmem, stream>>>(tmT0, tmV0, tmT1, tmV1, p0, p1);
   return cudaGetLastError();
 }
 

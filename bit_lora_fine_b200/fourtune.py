@@ -27,8 +27,8 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_quant_down_static")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
-FWD_KERNELS = ("pack_lowrank", "xpass_quant_down", "gemm_fp4_fwd")
-BWD_KERNELS = ("pack_lowrank", "gpass_quant_down", "gemm_fp4_dx", "tgrad_dA", "tgrad_dB")
+FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
+BWD_KERNELS = ("gpass_quant_down", "gemm_fp4_dx", "tgrad_dA_dB")
 
 
 class FourtuneError(RuntimeError):
@@ -40,8 +40,7 @@ class FourtuneError(RuntimeError):
 class ft_linear_t(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int64), ("N", ctypes.c_int64), ("r_s", ctypes.c_int64), ("r", ctypes.c_int64),
                 ("R_codes", ctypes.c_void_p), ("R_scales", ctypes.c_void_p), ("R_codes_t", ctypes.c_void_p),
-                ("S_dn", ctypes.c_void_p), ("S_up", ctypes.c_void_p), ("A", ctypes.c_void_p),
-                ("B", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+                ("D", ctypes.c_void_p), ("U", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
 
 
 _lib = None
@@ -122,27 +121,39 @@ def transpose_codes(codes, rows, cols):
 
 
 class Linear:
-    """Device tensors of one triple-branch layer (frozen R codes/scales/codes_t, S_dn, S_up,
-    bias; trainable A, B).  Holds references so the pointers stay valid."""
+    """Device tensors of one triple-branch layer: frozen R codes/scales/codes_t and bias,
+    D = [S_dn | A] [K, r_s + r] and U = [S_up ; B] [r_s + r, N] (bf16).  The LoRA factors
+    are views: A = D[:, r_s:], B = U[r_s:, :].  Holds references so pointers stay valid."""
 
-    def __init__(self, R_codes, R_scales, R_codes_t, S_dn, S_up, A, B, bias=None):
+    def __init__(self, R_codes, R_scales, R_codes_t, D, U, r_s, bias=None):
         N, half_k = R_codes.shape
         self.K, self.N = half_k * 2, N
-        self.r_s, self.r = S_dn.shape[1], A.shape[1]
+        self.r_s = r_s
+        self.r = D.shape[1] - r_s
         for t, n in ((R_codes, "R_codes"), (R_scales, "R_scales"), (R_codes_t, "R_codes_t")):
             _need(t, torch.uint8, n)
-        for t, n in ((S_dn, "S_dn"), (S_up, "S_up"), (A, "A"), (B, "B"), (bias, "bias")):
+        for t, n in ((D, "D"), (U, "U"), (bias, "bias")):
             _need(t, torch.bfloat16, n)
-        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_codes_t=R_codes_t, S_dn=S_dn, S_up=S_up, A=A, B=B,
-                      bias=bias)
+        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_codes_t=R_codes_t, D=D, U=U, bias=bias)
         self.c = ft_linear_t(self.K, self.N, self.r_s, self.r, *[
-            _ptr(self.t[k]) for k in ("R_codes", "R_scales", "R_codes_t", "S_dn", "S_up", "A", "B", "bias")])
+            _ptr(self.t[k]) for k in ("R_codes", "R_scales", "R_codes_t", "D", "U", "bias")])
 
     @classmethod
     def from_weights(cls, R, S_dn, S_up, A, B, bias=None):
-        """Quantize the frozen residual weight R [N, K] (bf16) on the device."""
+        """Quantize the frozen residual weight R [N, K] (bf16) on the device and
+        concatenate the stabilizer and LoRA factors along the rank."""
         codes, scales, codes_t = quantize_block16(R, transposed=True)
-        return cls(codes, scales, codes_t, S_dn, S_up, A, B, bias)
+        D = torch.cat([S_dn, A], dim=1).contiguous()
+        U = torch.cat([S_up, B], dim=0).contiguous()
+        return cls(codes, scales, codes_t, D, U, S_dn.shape[1], bias)
+
+    @property
+    def A(self):
+        return self.t["D"][:, self.r_s:]
+
+    @property
+    def B(self):
+        return self.t["U"][self.r_s:, :]
 
     @property
     def R_all(self):

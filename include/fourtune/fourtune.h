@@ -70,19 +70,22 @@ enum { FT_DTYPE_F32 = 0, FT_DTYPE_BF16 = 1 };
  *   R_codes_t [K, N/2]  the same codes nibble-transposed (codes of R^T); the
  *                       scales of R^T are R_scales read transposed.  Required by
  *                       the backward (fourtune_quantize_block16 writes it).
- *   S_dn [K, r_s], S_up [r_s, N]  frozen stabilizer (bf16)
- *   A [K, r], B [r, N]            trainable LoRA (bf16)
+ *   D [K, r_s + r] = [S_dn | A]   down-projections, bf16 row-major: the frozen
+ *                       stabilizer's S_dn in columns 0..r_s-1, the LoRA A after it
+ *   U [r_s + r, N] = [S_up ; B]   up-projections, bf16 row-major: S_up rows first,
+ *                       then the LoRA B
  *   bias [N] frozen bf16 or NULL
- * Ranks: r_s >= 0, r >= 16, r_s + r <= 128, each a multiple of 16; r <= 64. */
+ * The stabilizer and the adapter share the input (§3.3), so their factors are
+ * stored concatenated along the rank and applied as one product each way; A
+ * and B are views into D and U (A has row stride r_s + r).
+ * Ranks: r_s >= 0, 16 <= r <= 64, r_s + r <= 128, each a multiple of 16. */
 typedef struct {
   int64_t K, N, r_s, r;
   const uint8_t* R_codes;
   const uint8_t* R_scales;
   const uint8_t* R_codes_t;
-  const ft_bf16* S_dn;
-  const ft_bf16* S_up;
-  const ft_bf16* A;
-  const ft_bf16* B;
+  const ft_bf16* D;
+  const ft_bf16* U;
   const ft_bf16* bias;
 } ft_linear_t;
 
@@ -106,7 +109,7 @@ FT_API size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64
 
 /* Forward (§3.1, §3.3 LoRA fusion).  X [M, K] bf16.  Writes
  *   Y [M, N] (y_dtype FT_DTYPE_F32 or FT_DTYPE_BF16, row stride N)
- *   L_saved [M, r_s + r] bf16 = bf16(X [S_dn | A]), kept for the backward.
+ *   L_saved [M, r_s + r] bf16 = bf16(X D), kept for the backward.
  * One pass reads X once, quantizes it and computes L; the 4-bit GEMM then adds
  * L [S_up ; B] and the bias in its accumulator. */
 FT_API int fourtune_linear_fwd(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
@@ -114,9 +117,9 @@ FT_API int fourtune_linear_fwd(const ft_linear_t* layer, const ft_bf16* X, int64
 
 /* Backward (§3.2).  dY [M, N] bf16 (the incoming gradient G), X and L_saved from
  * the forward.  Writes
- *   dX [M, K] = deq(Q(G)) deq(Q(R)) + P [S_dn | A]^T   (dx_dtype F32 or BF16)
+ *   dX [M, K] = deq(Q(G)) deq(Q(R)) + P D^T   (dx_dtype F32 or BF16)
  *   dA [K, r] fp32 = X^T P[:, r_s:]     dB [r, N] fp32 = L[:, r_s:]^T G
- * with P = bf16(G [S_up ; B]^T).  accumulate = 1 adds into dA and dB, 0
+ * with P = bf16(G U^T).  accumulate = 1 adds into dA and dB, 0
  * overwrites.  R, S and bias receive no gradient. */
 FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, const ft_bf16* X, const ft_bf16* L_saved,
                         int64_t M, void* dX, int dx_dtype, float* dA, float* dB, int accumulate, void* ws,
@@ -125,9 +128,9 @@ FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, cons
 /* The same calls, recording caller-created CUDA events (cudaEvent_t as void*) on
  * `stream` around each kernel they launch: events[2k] before and events[2k+1]
  * after kernel k (NULL entries and k >= n_events/2 are skipped).  Kernels, in
- * order -- forward: 0 pack low-rank factors, 1 fused X pass (quantize + X D),
- * 2 FP4 GEMM with up-projection; backward: 0 pack, 1 fused G pass (quantize +
- * G U^T), 2 FP4 dX GEMM, 3 dA, 4 dB.  Used for live per-kernel timing. */
+ * order -- forward: 0 fused X pass (quantize + X D), 1 FP4 GEMM with
+ * up-projection; backward: 0 fused G pass (quantize + G U^T), 1 FP4 dX GEMM,
+ * 2 dA and dB.  Used for live per-kernel timing. */
 FT_API int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
                                      ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
@@ -149,7 +152,7 @@ FT_API int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, s
  * device memory and offer no scratch allocator, and runtimes that forbid any
  * allocation once they have started.  It computes what the forward's first
  * kernel computes, for any bf16 input X [M, K] and down-projection rows
- * W [R, K] (bf16, K contiguous; for the layer, W = [S_dn | A]^T):
+ * W [R, K] (bf16, K contiguous; for the layer, W = D^T = [S_dn | A]^T):
  *   codes [M, K/2], scales [M/16, K/16] = block16(X)   and   L [M, R] = bf16(X W^T).
  * The caller still owns X, W and the outputs.  Scratch (split-K partial sums,
  * split counters, status word) lives in one device array inside the library,

@@ -28,6 +28,20 @@ def bf16_ulps(got, ref):
     return float((np.abs(got - ref) / ulp).max())
 
 
+def check_bf16_dot(got, ref, absdot, n):
+    """A bf16-rounded dot product of length n: the GPU accumulates in fp32, the oracle
+    exactly, then both round once.  Elementwise bound: one bf16 ulp of the result plus
+    the fp32 accumulation bound n * 2^-24 * sum|a_k b_k| (absdot); and normwise within
+    one bf16 ulp of the largest element."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    mag = np.maximum(np.abs(ref), 2.0 ** -126)
+    bound = 2.0 ** (np.floor(np.log2(mag)) - 7) + n * 2.0 ** -24 * np.asarray(absdot)
+    bad = np.abs(got - ref) > bound
+    assert not bad.any(), f"{int(bad.sum())} elements beyond the bf16-dot bound"
+    assert normwise(got, ref) <= 2.0 ** -8
+
+
 def to_dev_bf16(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda").to(torch.bfloat16)
@@ -38,6 +52,31 @@ def to_host(t):
     if t.dtype == torch.bfloat16:
         return t.float().cpu().numpy().astype(np.float64)
     return t.cpu().numpy()
+
+
+def tie_tensor(rows, cols, seed=0):
+    """bf16 values that hit every E2M1 rounding tie exactly: in each 16x16 block
+    the largest magnitude is 6 d for an E4M3 value d (so the block scale is d and
+    element / scale is exact), the other entries are +-t d for the ties t in
+    {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5} and their bf16 neighbours one ulp
+    either side, plus +-0.  d runs over normal and subnormal E4M3 scales."""
+    from oracle import formats  # test-side construction only
+    rng = np.random.default_rng(seed)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    scodes = [0x01, 0x03, 0x07, 0x08, 0x1B, 0x30, 0x38, 0x3D, 0x4F, 0x66, 0x70]
+    t = np.zeros((rows, cols), np.float32)
+    for bi in range(rows // 16):
+        for bj in range(cols // 16):
+            d = formats.E4M3_TABLE[scodes[(bi * 7 + bj) % len(scodes)]]
+            vals = np.concatenate([ties * d, -ties * d]).astype(np.float32)
+            up = synth.bf16_from_bits(synth.bf16_bits(vals) + np.uint16(1))
+            dn = synth.bf16_from_bits(synth.bf16_bits(vals) - np.uint16(1))
+            pool = np.concatenate([vals, up, dn, np.float32([0.0, -0.0])])
+            blk = rng.choice(pool, size=(16, 16))
+            blk[0, 0] = np.float32(6 * d) * rng.choice([-1, 1])
+            t[bi * 16:(bi + 1) * 16, bj * 16:(bj + 1) * 16] = blk
+    assert np.array_equal(synth.to_bf16(t), t), "tie tensor must be bf16-exact"
+    return t
 
 
 def random_layer(K, N, r_s, r, seed=0, w_std=0.02, b_std=1e-3, bias=False, M=None, x_outliers=4):

@@ -43,7 +43,7 @@ def test_error_strings(lib):
 
 def _layer(K=64, N=64, r_s=16, r=16, ptr=256):
     p = ctypes.c_void_p(ptr)
-    return fourtune.ft_linear_t(K, N, r_s, r, p, p, p, p, p, p, p, None)
+    return fourtune.ft_linear_t(K, N, r_s, r, p, p, p, p, p, None)
 
 
 def test_argument_checks_without_device(lib):
@@ -63,7 +63,7 @@ def test_argument_checks_without_device(lib):
     L = _layer(r=80)
     assert lib.fourtune_linear_fwd(ctypes.byref(L), p, 16, p, 0, p, p, 1 << 20, s) == -7
     L = _layer()
-    L.A = ctypes.c_void_p(264)
+    L.D = ctypes.c_void_p(264)
     assert lib.fourtune_linear_fwd(ctypes.byref(L), p, 16, p, 0, p, p, 1 << 20, s) == -3
     # bad dtype code, bad M
     L = _layer()

@@ -5,7 +5,7 @@ import pytest
 
 from bit_lora_fine_b200 import synth
 from oracle import block16
-from tests.helpers import to_dev_bf16
+from tests.helpers import tie_tensor, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -35,6 +35,13 @@ def test_worked_ties_probe(cuda_lib):
     b[16:32, 16] = np.float32(1e-3)         # tiny block: after rounding to bf16 still small
     b = synth.to_bf16(b)
     _check(cuda_lib, b)
+
+
+def test_every_e2m1_tie(cuda_lib):
+    """All seven E2M1 ties, both signs, one bf16 ulp either side, under normal and
+    subnormal scales: the codes must be the oracle's nearest-even table search."""
+    x = tie_tensor(176, 224, seed=1)
+    _check(cuda_lib, x)
 
 
 @pytest.mark.parametrize("shape,std,seed", [((16, 16), 1.0, 0), ((32, 48), 0.02, 1), ((48, 80), 5.0, 2),
