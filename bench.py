@@ -9,8 +9,8 @@ rank 32, LoRA rank 32, seeded synthetic bf16 data (synth.py).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints one JSON line (rank 0).  `value` is device time from CUDA events summed
-over exactly K steps (L2 flushed by a 256 MB write before each step, outside
-the events), max over ranks; `e2e` repeats the steps through the same C ABI with
+over exactly K steps (L2 flushed before each step, outside the events, by a
+256 MB write followed by a 256 MB read of another buffer), max over ranks; `e2e` repeats the steps through the same C ABI with
 inputs in pinned host memory (H2D of X and dY, D2H of dA and dB inside the
 timed region).  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload.  With N > 1 (torchrun) every rank runs an independent
@@ -207,7 +207,17 @@ def run_ours(args, rank, world, local_rank):
     dA = torch.zeros((K, r), dtype=torch.float32, device=dev)
     dB = torch.zeros((r, N), dtype=torch.float32, device=dev)
     ws_f, ws_b = lay.fwd_workspace(M), lay.bwd_workspace(M)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    # L2 flush before every step: write 256 MB (> 126 MB L2), then read another
+    # 256 MB so that no input of the step is cached and no dirty line is left
+    # for the step's reads to write back
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    class _Flush:
+        def zero_(self):
+            flush_w.zero_()
+            flush_r.sum()
+    flush = _Flush()
 
     nf, nb = len(ft.FWD_KERNELS), len(ft.BWD_KERNELS)
     names = [f"fwd.{k}" for k in ft.FWD_KERNELS] + [f"bwd.{k}" for k in ft.BWD_KERNELS]
@@ -321,7 +331,8 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4(e2m1 x e2m1, e4m3 16x16 scales)->f32; bf16 low-rank",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "r_s": r_s, "r": r, "global_batch_tokens": M * world,
-                   "l2": "flushed (256 MB write before each step, outside the timed events)",
+                   "l2": "flushed before each step outside the timed events: 256 MB write, then 256 MB read of "
+                         "another buffer (no input cached, no dirty lines)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single"},
         "tokens_per_s": M * args.steps * world / sec,
         "fp4_tflops": fp4 * args.steps * world / sec / 1e12,

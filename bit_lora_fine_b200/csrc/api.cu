@@ -54,6 +54,13 @@ bool map_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols / 2, rows, cols / 2, 128, box_rows,
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// GEMM output [rows, cols] fp32 or bf16: boxes of 128 bytes x 32 rows, 128-byte swizzle
+bool map_out(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, bool bf16) {
+  return bf16 ? make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, cols * 2, 64, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B)
+              : make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, cols, rows, cols * 4, 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+}
 // compact scales [rows, cols] bytes, unswizzled boxes of 16 bytes x box_rows
 bool map_scales(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, cols, 16, box_rows,
@@ -111,10 +118,10 @@ struct RowSplit {
   int nsplit, kt_per_split;
 };
 // enough CTAs for every SM (two per SM when they fit), never more splits than tiles
-RowSplit row_split(int64_t M, int64_t K, int64_t R, int mn, int num_sms) {
+RowSplit row_split(int64_t M, int64_t K, int64_t R, int mn, int num_sms, int max_split) {
   const int MT = cdiv(M, 128), KT = cdiv(K, 64);
   const int target = num_sms * ft::rowpass_ctas_per_sm(static_cast<int>(R), mn);
-  const int ns = MT >= target ? 1 : std::max(1, std::min(KT, target / MT));
+  const int ns = MT >= target ? 1 : std::max(1, std::min({KT, target / MT, max_split}));
   const int per = cdiv(KT, ns);
   return {cdiv(KT, per), per};
 }
@@ -138,7 +145,7 @@ struct FwdWs {
 FwdWs fwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   FwdWs w{};
   const int64_t R = L->r_s + L->r;
-  w.rs = row_split(M, L->K, R, 1, num_sms);
+  w.rs = row_split(M, L->K, R, 1, num_sms, ft::kRowpassMaxClusterSplit);
   w.counters = 16;
   w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
   size_t o = w.header;
@@ -146,8 +153,7 @@ FwdWs fwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   o = up256(o + static_cast<size_t>(M * L->K / 2));
   w.scales = o;
   o = up256(o + static_cast<size_t>((M / 16) * (L->K / 16)));
-  w.part = o;
-  if (w.rs.nsplit > 1) o = up256(o + static_cast<size_t>(w.rs.nsplit) * M * R * 4);
+  w.part = o;  // unused: split partials are reduced inside the cluster
   w.total = o;
   return w;
 }
@@ -160,7 +166,7 @@ struct BwdWs {
 BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   BwdWs w{};
   const int64_t R = L->r_s + L->r;
-  w.rs = row_split(M, L->N, R, 0, num_sms);
+  w.rs = row_split(M, L->N, R, 0, num_sms, ft::kRowpassMaxClusterSplit);
   w.sA = m_split(M, L->K, std::max(1, num_sms / 2));
   w.sB = m_split(M, L->N, std::max(1, num_sms / 2));
   const int MT = cdiv(M, 128), KTl = cdiv(L->K, 128), NTl = cdiv(L->N, 128);
@@ -175,8 +181,7 @@ BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   o = up256(o + static_cast<size_t>((M / 16) * (L->N / 16)));
   w.P = o;
   o = up256(o + static_cast<size_t>(M * R * 2));
-  w.part_rp = o;
-  if (w.rs.nsplit > 1) o = up256(o + static_cast<size_t>(w.rs.nsplit) * M * R * 4);
+  w.part_rp = o;  // unused: split partials are reduced inside the cluster
   w.part_dA = o;
   if (w.sA.nsplit > 1) o = up256(o + static_cast<size_t>(w.sA.nsplit) * KTl * 128 * 64 * 4);
   w.part_dB = o;
@@ -322,6 +327,7 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   rp.w_mn_major = 1;
   rp.kt_per_split = w.rs.kt_per_split;
   rp.nsplit = w.rs.nsplit;
+  rp.cluster_reduce = w.rs.nsplit > 1;
   rp.codes = base + w.codes;
   rp.scales = base + w.scales;
   rp.L = L_saved;
@@ -363,7 +369,9 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   gp.ldo = N;
   gp.out_bf16 = y_dtype == FT_DTYPE_BF16;
   gp.status = status;
-  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, gp, s));
+  CUtensorMap tmO;
+  if (!map_out(&tmO, Y, N, M, gp.out_bf16 != 0)) return FT_ERR_CUDA;
+  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, gp, s));
   return FT_OK;
 }
 
@@ -409,6 +417,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   rp.w_mn_major = 0;
   rp.kt_per_split = w.rs.kt_per_split;
   rp.nsplit = w.rs.nsplit;
+  rp.cluster_reduce = w.rs.nsplit > 1;
   rp.codes = base + w.codes;
   rp.scales = base + w.scales;
   rp.L = base + w.P;
@@ -451,7 +460,9 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   gp.ldo = K;
   gp.out_bf16 = dx_dtype == FT_DTYPE_BF16;
   gp.status = status;
-  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, gp, s));
+  CUtensorMap tmO;
+  if (!map_out(&tmO, dX, K, M, gp.out_bf16 != 0)) return FT_ERR_CUDA;
+  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, gp, s));
 
   // dA = X^T P[:, r_s:] and dB = L[:, r_s:]^T G (computed as dB^T, stored transposed), one launch
   CUtensorMap tmTa, tmVa, tmTb, tmVb;
@@ -494,7 +505,7 @@ int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_
   int st = device_info(&di);
   if (st) return st;
   // W^T [R, K] read K-major (the backward pass's layout) with its own split choice
-  const RowSplit rs = row_split(M, K, R, 0, di.num_sms);
+  const RowSplit rs = row_split(M, K, R, 0, di.num_sms, 1 << 20);
   const size_t header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
   const size_t need = header + (rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * M * R * 4 : 0);
   if (need > ft::kRowpassStaticScratchBytes) return FT_ERR_WORKSPACE;
@@ -513,6 +524,7 @@ int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_
   rp.w_mn_major = 0;
   rp.kt_per_split = rs.kt_per_split;
   rp.nsplit = rs.nsplit;
+  rp.cluster_reduce = 0;  // partials in the static scratch, summed by the last CTA
   rp.codes = codes;
   rp.scales = scales;
   rp.L = L;

@@ -88,8 +88,36 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// bar.sync is the aligned barrier: reconverge the warp first
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA in the cluster arrives and waits (release/acquire).
+// The non-aligned forms: a warp may reach this with its lanes diverged.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// address of the same shared-memory location in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t map_cluster(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(caddr)
+               : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -105,6 +133,20 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// 2-D tiled store of one box from shared memory (bulk-group completion).
+// Elements of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -266,20 +308,39 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
   return r;
 }
 
-// Block16 quantization of 32 consecutive values of one row (two 16-column
-// blocks) given the two block maxima: scale = E4M3(amax / 6), code =
-// E2M1(v / dec(scale)), all +0 when the scale decodes to 0.  Writes four
-// 32-bit words of codes (element i of block j in word 2j + i/8) and the two
-// scale bytes.
+// Block16 quantization of 32 consecutive bf16 values of one row (two 16-column
+// blocks) given the two block maxima: scale = E4M3(amax / 6) (IEEE division),
+// code = E2M1(v / dec(scale)) rounded to nearest even, all +0 when the scale
+// decodes to 0.  Writes four 32-bit words of codes (element i of block j in word
+// 2j + i/8) and the two scale bytes.
+//
+// The per-element division is replaced by an exact equivalent.  v is bf16 (at
+// most 8 significant bits) and d = dec(scale) an E4M3 value (at most 4), so v/d
+// is either exactly one of the E2M1 rounding ties (0.25, 0.75, 1.25, 1.75, 2.5,
+// 3.5, 5, either sign) or at least 1/255 (relative) away from every one of them
+// (the difference of two such products is a multiple of the smaller power of
+// two).  q = v * (1/d), with the reciprocal correctly rounded, is within 2^-22
+// (relative) of v/d; rounding q to 19 mantissa bits therefore lands exactly on
+// the tie when v/d is one and otherwise moves q by less than 2^-19, never across
+// a tie.  The nearest-even conversion of that q is the code of v/d, i.e. of the
+// IEEE quotient fp32(v / d) (which can only equal a tie when v/d does).
+__device__ __forceinline__ float snap19(float q) {
+  return __uint_as_float((__float_as_uint(q) + 0x8u) & ~0xFu);
+}
 __device__ __forceinline__ void quantize_2blocks(const float* v, const float* amax, uint32_t* packed,
                                                  uint32_t* sc) {
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
     const float d = e4m3_to_f32(sc[j]);
+    if (d == 0.0f) {
+      packed[2 * j] = packed[2 * j + 1] = 0u;
+      continue;
+    }
+    const float rd = __frcp_rn(d);
     float q[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + e], d);
+    for (int e = 0; e < 16; ++e) q[e] = snap19(v[16 * j + e] * rd);
     packed[2 * j] = f32x8_to_e2m1(q);
     packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
   }

@@ -22,7 +22,9 @@
 //                  K=64) x 4 per K-block, then kind::f16 for the extra blocks
 //   warp 2         expands the compact scales into the per-row layout the MMA
 //                  reads (one 16-byte pattern per 16 rows)
-//   warps 4..7     epilogue: TMEM -> registers -> + bias -> fp32/bf16 stores
+//   warps 4..7     epilogue: TMEM -> registers (+ bias) -> fp32/bf16 rows staged
+//                  in the now idle pipeline smem (128-byte swizzled boxes of 32
+//                  rows) -> TMA tensor stores, which clip rows/columns past M, N
 #include "common.cuh"
 #include "kernels.h"
 
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using Lay = GemmLayout<BN>;
   static_assert(Lay::kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(Lay::kTmemUsed <= 512, "TMEM budget");
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
+    tma_prefetch(&tmOut);
     if (EB) {
       tma_prefetch(&tmA2);
       tma_prefetch(&tmB2);
@@ -263,56 +266,65 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     }
   } else if (warp >= 4) {
     if (mbar_wait(acc_full, 0, p.status, abortp)) {
+      __syncwarp();
+      // Every MMA has completed, so every TMA load has landed and been consumed:
+      // the pipeline smem is free.  Warp q stages its 32 rows x BN columns as
+      // boxes of 32 rows x 128 bytes (128-byte swizzle, 4 KB each) at q * (BN/ebox) * 4 KB.
       tc_fence_after();
       const int q = warp & 3;
-      const int row = m0 + 32 * q + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      const bool row_ok = row < p.M;
       const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
+      const int ebox = p.out_bf16 ? 64 : 32;               // elements per 128-byte box row
+      uint8_t* region = smem + q * (BN / ebox) * 4096;
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c0, v);
         tmem_ld_wait();
-        const int nb = n0 + c0;
-        if (!row_ok || nb >= p.N) continue;
         float f[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        const int nb = n0 + c0;
         if (bias) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (nb + e < p.N) f[e] += __bfloat162float(bias[nb + e]);
         }
-        const bool full_chunk = nb + 32 <= p.N;
+        uint8_t* row = region + (c0 / ebox) * 4096 + lane * 128;
         if (p.out_bf16) {
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(row) * p.ldo + nb;
-          if (full_chunk) {
-            uint32_t w[16];
+          const int j0 = (c0 % 64) / 8;                    // first 16-byte chunk of this 32-column slice
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+          for (int k = 0; k < 4; ++k) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b = __floats2bfloat162_rn(f[8 * k + 2 * e], f[8 * k + 2 * e + 1]);
               w[e] = *reinterpret_cast<const uint32_t*>(&b);
             }
-            uint4* d = reinterpret_cast<uint4*>(o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-          } else {
-            for (int e = 0; e < 32 && nb + e < p.N; ++e) o[e] = __float2bfloat16_rn(f[e]);
+            *reinterpret_cast<uint4*>(row + (((j0 + k) ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          float* o = static_cast<float*>(p.out) + static_cast<long long>(row) * p.ldo + nb;
-          if (full_chunk) {
-            float4* d = reinterpret_cast<float4*>(o);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
-          } else {
-            for (int e = 0; e < 32 && nb + e < p.N; ++e) o[e] = f[e];
-          }
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(row + ((k ^ (lane & 7)) * 16)) =
+                make_uint4(__float_as_uint(f[4 * k]), __float_as_uint(f[4 * k + 1]), __float_as_uint(f[4 * k + 2]),
+                           __float_as_uint(f[4 * k + 3]));
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && m0 + 32 * q < p.M) {
+        for (int b = 0; b < BN / ebox; ++b) {
+          const int x = n0 + b * ebox;
+          if (x < p.N) tma_store_2d(&tmOut, region + b * 4096, x, m0 + 32 * q);
+        }
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      __syncwarp();
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -323,14 +335,14 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
-                            const GemmParams& p, cudaStream_t stream) {
+                            const CUtensorMap& tmOut, const GemmParams& p, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
   using Lay = GemmLayout<BN>;
   cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Lay::kSmem));
   if (e != cudaSuccess) return e;
   dim3 grid((p.N + BN - 1) / BN, (p.M + 127) / 128);
-  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, tmSFA, tmSFB, p);
+  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, tmSFA, tmSFB, tmOut, p);
   return cudaGetLastError();
 }
 

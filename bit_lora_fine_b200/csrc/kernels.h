@@ -14,13 +14,16 @@ struct RowpassParams {
   int M, K, R;
   int w_mn_major;                        // 1: D [K, R]; 0: W^T [R, K]
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
+  int cluster_reduce;                    // splits of a row tile form a cluster and reduce through DSMEM
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
   void* L;                               // bf16 [M, R]
-  float* part;                           // fp32 [nsplit, M, R] when nsplit > 1
-  int* counters;                         // [ceil(M/128)], zero on entry, left zero
+  float* part;                           // fp32 [nsplit, M, R] when nsplit > 1 and no cluster
+  int* counters;                         // [ceil(M/128)], zero on entry, left zero (no cluster)
   int* status;
 };
+// largest split count the cluster reduction handles (portable cluster size)
+constexpr int kRowpassMaxClusterSplit = 8;
 
 // out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1.
 // Scales: with sf_tma the compact [rows/16, K/16] tiles come by TMA (B's read
@@ -62,9 +65,10 @@ cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uin
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream);
 int rowpass_ctas_per_sm(int R, int w_mn_major);
+// tmOut: the output [M, N] (fp32 or bf16) with 128-byte x 32-row boxes, 128-byte swizzle
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
-                            const GemmParams& p, cudaStream_t stream);
+                            const CUtensorMap& tmOut, const GemmParams& p, cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
                           const CUtensorMap& tmT1, const CUtensorMap& tmV1, const TgradParams& p1,
                           cudaStream_t stream);

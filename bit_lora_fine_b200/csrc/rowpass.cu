@@ -15,8 +15,14 @@
 //                  N=R rounded as below, K=16) x 4 per tile into TMEM
 //   warps 4..11    each quantizes one 16-row block of the same smem tile, then
 //                  the eight drain the accumulator (two warps per TMEM lane
-//                  quadrant): L in bf16, or fp32 partials that the last CTA of
-//                  the row tile sums in split order (deterministic).
+//                  quadrant).  One split: L in bf16 straight from TMEM.  Several
+//                  splits: the splits of a row tile form a thread-block cluster;
+//                  each CTA parks its fp32 partial in its own (now idle) smem and
+//                  every CTA sums one slice of rows over all ranks in rank order
+//                  through distributed shared memory (deterministic, no global
+//                  partials).  A global-memory variant (partials in scratch, the
+//                  last CTA of the row tile sums them) serves the static-scratch
+//                  entry point.
 // The projection matrix is read either K-major (W^T [R, K], rows of 128 bytes,
 // N = R) or MN-major (D [K, R] with R contiguous: TMA boxes of 64 k-rows x 64
 // r, N = R rounded up to 64, the extra columns zero-filled by the TMA).
@@ -202,16 +208,26 @@ __global__ void __launch_bounds__(kRpThreads, 1)
 #pragma unroll
     for (int w = 0; w < kRpQuantWarps; ++w) go = go && s_ok[w];
     if (go) {
+      __syncwarp();
       tc_fence_after();
       const int q = warp & 3;                       // TMEM lane quadrant of this warp
       const int row = m0 + 32 * q + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
       const bool row_ok = row < p.M;
       const int half = (warp - 4) >> 2;             // which 16-column chunks this warp drains
+      float* parked = reinterpret_cast<float*>(smem) + (32 * q + lane) * (R + 4);
       for (int c0 = 16 * half; c0 < R; c0 += 32) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(taddr + c0, v);
         tmem_ld_wait();
+        if (p.cluster_reduce) {                     // park the partial in this CTA's smem
+          float4* dst = reinterpret_cast<float4*>(parked + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          continue;
+        }
         if (!row_ok) continue;
         if (p.nsplit == 1) {
           uint32_t w[8];
@@ -231,7 +247,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
       }
-      if (p.nsplit > 1) {
+      if (p.nsplit > 1 && !p.cluster_reduce) {
         // the last CTA of this row tile to finish sums every split's partial, in split order
         __threadfence();
         named_bar_sync(1, 32 * kRpQuantWarps);
@@ -270,6 +286,44 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     }
   }
 
+  if (p.cluster_reduce) {
+    // every split of this row tile has parked its partial: rank c sums rows
+    // [c * rows_per, (c + 1) * rows_per) over ranks 0..nsplit-1 in order
+    __syncwarp();
+    cluster_sync_all();
+    if (warp >= 4) {
+      const int ns = p.nsplit;
+      const int rows_per = (128 + ns - 1) / ns;
+      const int r_lo = static_cast<int>(cluster_ctarank()) * rows_per;
+      const int r_hi = min(128, r_lo + rows_per);
+      const int c4n = R / 4;
+      const uint32_t base = smem_u32(smem);
+      for (int idx = threadIdx.x - 128; idx < (r_hi - r_lo) * c4n; idx += 32 * kRpQuantWarps) {
+        const int rl = r_lo + idx / c4n;
+        const int c = 4 * (idx % c4n);
+        const uint32_t off = base + static_cast<uint32_t>((rl * (R + 4) + c) * 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < ns; ++j) {
+          const float4 v = ld_cluster_f4(map_cluster(off, static_cast<uint32_t>(j)));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int grow = m0 + rl;
+        if (grow < p.M) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x, acc.y);
+          const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z, acc.w);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.L) + static_cast<long long>(grow) * R + c) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while another may still read its smem
+  }
+
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -285,9 +339,19 @@ static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& t
   cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((p.M + 127) / 128, p.nsplit);
-  rowpass_kernel<RCOLS><<<grid, kRpThreads, smem, stream>>>(tmX, tmW, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.M + 127) / 128, p.nsplit);
+  cfg.blockDim = dim3(kRpThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = p.cluster_reduce ? p.nsplit : 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, rowpass_kernel<RCOLS>, tmX, tmW, p);
 }
 
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,

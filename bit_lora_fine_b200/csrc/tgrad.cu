@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     named_bar_sync(1, 128);
     const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
     if (go) {
+      __syncwarp();
       tc_fence_after();
       const int q = warp & 3;
       const int prow = pbase + 32 * q + lane;
@@ -183,6 +184,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

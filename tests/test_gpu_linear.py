@@ -128,3 +128,22 @@ def test_config_flux_linear_3072(cuda_lib):
     p["X"] = synth.layer_input(wl)
     p["dY"] = synth.upstream_grad(wl)
     run_and_check(cuda_lib, p, wl.M, check_bf16=True)
+
+
+def test_repeated_calls_are_bit_identical(cuda_lib):
+    """Split reductions sum in a fixed order: repeated calls give identical bits."""
+    import torch
+    ft = cuda_lib
+    wl = synth.WORKLOADS["flux-linear-3072"]
+    p = synth.layer_params(wl.layers[0])
+    lay = _device_layer(ft, p)
+    X, dY = to_dev_bf16(synth.layer_input(wl)), to_dev_bf16(synth.upstream_grad(wl))
+    outs = []
+    for _ in range(3):
+        Y, L, ws = ft.linear_fwd(lay, X, torch.bfloat16)
+        dX, dA, dB, wsb = ft.linear_bwd(lay, dY, X, L, torch.bfloat16)
+        torch.cuda.synchronize()
+        outs.append([t.clone() for t in (Y, L, dX, dA, dB)])
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
