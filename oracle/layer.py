@@ -20,9 +20,11 @@ Readings of what the pages leave open (each is also listed in the design notes):
   * dA = X^T P[:, r_s:]   and   dB = L[:, r_s:]^T G   (straight-through: Q has
     no derivative of its own).
   * MLP: h = bf16(FC1(X) + b1) is the saved hidden; a = GELU_tanh(h);
-    FC2's 4-bit input is Q(a) of float32 a; its low-rank input is bf16(a).
-    Backward: d_a from FC2, d_h = d_a * GELU'(h); FC1's 4-bit gradient is
-    Q(d_h) of float32 d_h and its low-rank gradient input is bf16(d_h).
+    FC2's 4-bit input is Q(a) of float32 a (the quantizer consumes the
+    activation as it is produced, never stored in bf16); its low-rank input is
+    bf16(a).  Backward: d_a from FC2, d_h = bf16(d_a * GELU'(h)) -- the
+    gradient reaching FC1 is a bf16 tensor like any layer's incoming gradient,
+    and all three of FC1's branches take it (Q(d_h) for the 4-bit branch).
 
 All GEMMs run in float64 on the exactly dequantized operands; a library matmul
 is the only primitive used.
@@ -129,10 +131,11 @@ def mlp_fwd(X, fc1, fc2, a_f32=None):
                 qa_codes=Qa[0], qa_scales=Qa[1])
 
 
-def mlp_bwd(G, X, h, L1, L2, fc1, fc2, dh_f32=None, a_bf=None):
+def mlp_bwd(G, X, h, L1, L2, fc1, fc2, dh_bf=None, a_bf=None):
     """Backward of mlp_fwd.  G = dL/dy [M, N2].  h, L1, L2 as saved by the forward.
 
-    `dh_f32` optionally overrides the float32 d_h that FC1's backward quantizes.
+    `dh_bf` optionally overrides the bf16 d_h that FC1's backward consumes (the
+    GPU's own, so that FC1's results compare on identical operands).
     `a_bf` optionally overrides FC2's low-rank input bf16(a) (else recomputed
     from h as in the forward).
     Returns dict(dX, dA1, dB1, dA2, dB2, d_a, d_h, ...).
@@ -144,12 +147,11 @@ def mlp_bwd(G, X, h, L1, L2, fc1, fc2, dh_f32=None, a_bf=None):
                     fc2["A"], fc2["B"])
     d_a = b2["dX"]
     d_h = d_a * gelu_tanh_grad(h)
-    dh32 = d_h.astype(np.float32) if dh_f32 is None else np.asarray(dh_f32, dtype=np.float32)
-    dh_bf = formats.bf16_round(dh32.astype(np.float64))
-    Qdh = block16.quantize(dh32)
-    b1 = linear_bwd(dh_bf, X, L1, fc1["R_codes"], fc1["R_scales"], fc1["S_dn"], fc1["S_up"],
+    dh = formats.bf16_round(d_h) if dh_bf is None else np.asarray(dh_bf, dtype=np.float64)
+    Qdh = block16.quantize(dh.astype(np.float32))
+    b1 = linear_bwd(dh, X, L1, fc1["R_codes"], fc1["R_scales"], fc1["S_dn"], fc1["S_up"],
                     fc1["A"], fc1["B"], Qg=Qdh)
     return dict(dX=b1["dX"], dA1=b1["dA"], dB1=b1["dB"], dA2=b2["dA"], dB2=b2["dB"],
-                d_a=d_a, d_h=d_h, dh32=dh32, P1=b1["P"], P2=b2["P"],
+                d_a=d_a, d_h=d_h, dh_bf=dh, a_bf=a_bf, P1=b1["P"], P2=b2["P"],
                 qdh_codes=Qdh[0], qdh_scales=Qdh[1], qg_codes=b2["qg_codes"],
                 qg_scales=b2["qg_scales"])

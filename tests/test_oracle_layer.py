@@ -195,8 +195,7 @@ def test_mlp_chain_rule_vs_autograd(monkeypatch):
     X = rng.standard_normal((M, K))
     G = rng.standard_normal((M, N))
     f = layer.mlp_fwd(X, fc1, fc2)
-    b = layer.mlp_bwd(G, X, f["h"], f["L1"], f["L2"], fc1, fc2, a_bf=f["a32"].astype(np.float64),
-                      dh_f32=None)
+    b = layer.mlp_bwd(G, X, f["h"], f["L1"], f["L2"], fc1, fc2, a_bf=f["a32"].astype(np.float64))
 
     T = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)
     tX = T(X)
