@@ -99,6 +99,7 @@ int num_sms_or_default() {
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
 
 int check_layer(const ft_linear_t* L, bool need_t) {
   if (!L || !L->R_codes || !L->R_scales || !L->D || !L->U) return FT_ERR_INVALID_ARG;
@@ -112,6 +113,13 @@ int check_layer(const ft_linear_t* L, bool need_t) {
     return FT_ERR_ALIGN;
   return FT_OK;
 }
+int check_mlp(const ft_linear_t* fc1, const ft_linear_t* fc2, bool need_t) {
+  int st = check_layer(fc1, need_t);
+  if (st) return st;
+  if ((st = check_layer(fc2, need_t))) return st;
+  return fc1->N == fc2->K ? FT_OK : FT_ERR_SHAPE;
+}
+inline int64_t rank_all(const ft_linear_t* L) { return L->r_s + L->r; }
 
 // ---------------------------------------------------------------- split choice
 struct RowSplit {
@@ -135,63 +143,125 @@ MSplit m_split(int64_t M, int64_t P, int ctas) {
   return {cdiv(MT, per), per};
 }
 
-// ---------------------------------------------------------------- workspace
-// Every layout starts with a header (status word + split counters) that each
-// call clears before its first kernel.
-struct FwdWs {
-  size_t header, counters, codes, scales, part, total;
-  RowSplit rs;
+// ---------------------------------------------------------------- workspace carving
+struct Carver {
+  size_t o = 0;
+  size_t take(size_t bytes) {
+    const size_t at = o;
+    o = up256(o + bytes);
+    return at;
+  }
 };
-FwdWs fwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
+// block16 activations of a [M, C] matrix
+struct Q16 {
+  size_t codes, scales;
+  void carve(Carver& c, int64_t M, int64_t C) {
+    codes = c.take(static_cast<size_t>(M * C / 2));
+    scales = c.take(static_cast<size_t>((M / 16) * (C / 16)));
+  }
+};
+// dA/dB launch of one layer: splits, counters (in the header) and partials
+struct GradPair {
+  MSplit sA, sB;
+  size_t cntA, cntB;
+  size_t partA, partB;
+};
+size_t grad_counter_words(const ft_linear_t* L) { return cdiv(L->K, 128) + cdiv(L->N, 128); }
+void plan_grads(GradPair& g, const ft_linear_t* L, int64_t M, int num_sms) {
+  g.sA = m_split(M, L->K, std::max(1, num_sms / 2));
+  g.sB = m_split(M, L->N, std::max(1, num_sms / 2));
+}
+size_t grad_partial_bytes(const GradPair& g, const ft_linear_t* L) {
+  const size_t a = g.sA.nsplit > 1 ? static_cast<size_t>(g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0;
+  const size_t b = g.sB.nsplit > 1 ? static_cast<size_t>(g.sB.nsplit) * cdiv(L->N, 128) * 128 * 64 * 4 : 0;
+  return a + b;
+}
+
+// Each layout starts with a header of `header` bytes (status word, split
+// counters) that every call clears first.
+// Linear forward: header (status) | Q(X)
+struct FwdWs {
+  size_t header, total;
+  Q16 qx;
+};
+FwdWs fwd_layout(const ft_linear_t* L, int64_t M) {
   FwdWs w{};
-  const int64_t R = L->r_s + L->r;
-  w.rs = row_split(M, L->K, R, 1, num_sms, ft::kRowpassMaxClusterSplit);
-  w.counters = 16;
-  w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
-  size_t o = w.header;
-  w.codes = o;
-  o = up256(o + static_cast<size_t>(M * L->K / 2));
-  w.scales = o;
-  o = up256(o + static_cast<size_t>((M / 16) * (L->K / 16)));
-  w.part = o;  // unused: split partials are reduced inside the cluster
-  w.total = o;
+  Carver c;
+  c.take(w.header = 256);
+  w.qx.carve(c, M, L->K);
+  w.total = c.o;
   return w;
 }
 
+// Linear backward: header (status, dA/dB counters) | Q(G) | P | dA/dB partials
 struct BwdWs {
-  size_t header, cnt_rp, cnt_dA, cnt_dB, codes, scales, P, part_rp, part_dA, part_dB, total;
-  RowSplit rs;
-  MSplit sA, sB;
+  size_t header, P, total;
+  Q16 qg;
+  GradPair g;
 };
 BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   BwdWs w{};
-  const int64_t R = L->r_s + L->r;
-  w.rs = row_split(M, L->N, R, 0, num_sms, ft::kRowpassMaxClusterSplit);
-  w.sA = m_split(M, L->K, std::max(1, num_sms / 2));
-  w.sB = m_split(M, L->N, std::max(1, num_sms / 2));
-  const int MT = cdiv(M, 128), KTl = cdiv(L->K, 128), NTl = cdiv(L->N, 128);
-  w.cnt_rp = 16;
-  w.cnt_dA = w.cnt_rp + 4 * static_cast<size_t>(MT);
-  w.cnt_dB = w.cnt_dA + 4 * static_cast<size_t>(KTl);
-  w.header = up256(w.cnt_dB + 4 * static_cast<size_t>(NTl));
-  size_t o = w.header;
-  w.codes = o;
-  o = up256(o + static_cast<size_t>(M * L->N / 2));
-  w.scales = o;
-  o = up256(o + static_cast<size_t>((M / 16) * (L->N / 16)));
-  w.P = o;
-  o = up256(o + static_cast<size_t>(M * R * 2));
-  w.part_rp = o;  // unused: split partials are reduced inside the cluster
-  w.part_dA = o;
-  if (w.sA.nsplit > 1) o = up256(o + static_cast<size_t>(w.sA.nsplit) * KTl * 128 * 64 * 4);
-  w.part_dB = o;
-  if (w.sB.nsplit > 1) o = up256(o + static_cast<size_t>(w.sB.nsplit) * NTl * 128 * 64 * 4);
-  w.total = o;
+  plan_grads(w.g, L, M, num_sms);
+  Carver c;
+  w.g.cntA = 16;
+  w.g.cntB = w.g.cntA + 4 * static_cast<size_t>(cdiv(L->K, 128));
+  c.take(w.header = up256(16 + 4 * grad_counter_words(L)));
+  w.qg.carve(c, M, L->N);
+  w.P = c.take(static_cast<size_t>(M * rank_all(L) * 2));
+  w.g.partA = c.take(grad_partial_bytes(w.g, L));
+  w.g.partB = w.g.partA + (w.g.sA.nsplit > 1 ? static_cast<size_t>(w.g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0);
+  w.total = c.o;
   return w;
 }
 
-int cuda_err(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
+// MLP forward: header (status) | Q(X) | Q(a)
+struct MlpFwdWs {
+  size_t header, total;
+  Q16 qx, qa;
+};
+MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, int64_t M) {
+  MlpFwdWs w{};
+  Carver c;
+  c.take(w.header = 256);
+  w.qx.carve(c, M, fc1->K);
+  w.qa.carve(c, M, fc1->N);
+  w.total = c.o;
+  return w;
+}
 
+// MLP backward: header (status, counters of both layers' dA/dB) | Q(G) | P2 |
+// d_h | bf16(GELU(h)) | Q(d_h) | P1 | partials (shared by the two dA/dB launches)
+struct MlpBwdWs {
+  size_t header, P2, dh, abf, P1, total;
+  Q16 qg, qdh;
+  GradPair g2, g1;
+};
+MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, int num_sms) {
+  MlpBwdWs w{};
+  plan_grads(w.g2, fc2, M, num_sms);
+  plan_grads(w.g1, fc1, M, num_sms);
+  const int64_t H = fc1->N;
+  Carver c;
+  w.g2.cntA = 16;
+  w.g2.cntB = w.g2.cntA + 4 * static_cast<size_t>(cdiv(fc2->K, 128));
+  w.g1.cntA = w.g2.cntB + 4 * static_cast<size_t>(cdiv(fc2->N, 128));
+  w.g1.cntB = w.g1.cntA + 4 * static_cast<size_t>(cdiv(fc1->K, 128));
+  c.take(w.header = up256(16 + 4 * (grad_counter_words(fc2) + grad_counter_words(fc1))));
+  w.qg.carve(c, M, fc2->N);
+  w.P2 = c.take(static_cast<size_t>(M * rank_all(fc2) * 2));
+  w.dh = c.take(static_cast<size_t>(M * H * 2));
+  w.abf = c.take(static_cast<size_t>(M * H * 2));
+  w.qdh.carve(c, M, H);
+  w.P1 = c.take(static_cast<size_t>(M * rank_all(fc1) * 2));
+  const size_t part = c.take(std::max(grad_partial_bytes(w.g2, fc2), grad_partial_bytes(w.g1, fc1)));
+  w.g2.partA = w.g1.partA = part;
+  w.g2.partB = part + (w.g2.sA.nsplit > 1 ? static_cast<size_t>(w.g2.sA.nsplit) * cdiv(fc2->K, 128) * 128 * 64 * 4 : 0);
+  w.g1.partB = part + (w.g1.sA.nsplit > 1 ? static_cast<size_t>(w.g1.sA.nsplit) * cdiv(fc1->K, 128) * 128 * 64 * 4 : 0);
+  w.total = c.o;
+  return w;
+}
+
+// ---------------------------------------------------------------- timing hooks
 // Optional per-kernel timing: events[2k] / events[2k+1] are recorded on the
 // launching stream right before / after kernel k of the call (when provided).
 struct Events {
@@ -203,17 +273,147 @@ struct Events {
     return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   }
 };
-#define FT_LAUNCH(k, expr)                                      \
-  do {                                                          \
-    if (evs.mark((k), 0, s) != cudaSuccess) return FT_ERR_CUDA; \
-    if ((expr) != cudaSuccess) return FT_ERR_CUDA;              \
-    if (evs.mark((k), 1, s) != cudaSuccess) return FT_ERR_CUDA; \
-  } while (0)
 
-// scales can come by TMA when every compact scale row is a whole number of 16-byte units
-bool scales_by_tma(int64_t K, int64_t N, const void* a, const void* b) {
-  return K % 256 == 0 && N % 256 == 0 && al16(a) && al16(b);
+// ---------------------------------------------------------------- launch helpers
+// Fused row pass over X [M, K] bf16: Q(X) -> (codes, scales), L = bf16(X W)
+// with W = D [K, R] (w_mn) or W^T [R, K]; gelu: the input is h and the pass
+// quantizes GELU(h).  Split reduction inside a cluster: needs only the status word.
+int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
+                float* dbg_a, uint8_t* codes, uint8_t* scales, void* L, int* status, int num_sms,
+                cudaStream_t s) {
+  CUtensorMap tmX, tmW;
+  if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
+  if (w_mn ? !map_bf16(&tmW, W, R, K, 64) : !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
+  const RowSplit rs = row_split(M, K, R, w_mn ? 1 : 0, num_sms, ft::kRowpassMaxClusterSplit);
+  RowpassParams rp{};
+  rp.M = static_cast<int>(M);
+  rp.K = static_cast<int>(K);
+  rp.R = static_cast<int>(R);
+  rp.w_mn_major = w_mn ? 1 : 0;
+  rp.kt_per_split = rs.kt_per_split;
+  rp.nsplit = rs.nsplit;
+  rp.cluster_reduce = rs.nsplit > 1;
+  rp.gelu_input = gelu ? 1 : 0;
+  rp.dbg_a = dbg_a;
+  rp.codes = codes;
+  rp.scales = scales;
+  rp.L = L;
+  rp.status = status;
+  return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
+
+// FP4 GEMM.  Forward form: A = Q(act) [M, K], B = layer's R [N, K], B2 = U [R2, N]
+// (MN-major).  Transposed form (dX): B = R^T from R_codes_t, scales read
+// transposed, B2 = D [N_out, R2] (K-major).
+struct GemmArgs {
+  int64_t M, N, K, R2;
+  const uint8_t* a_codes;
+  const uint8_t* a_scales;
+  const uint8_t* b_codes;       // R_codes [N, K/2] or R_codes_t [N, K/2] (transposed form)
+  const uint8_t* r_scales;      // the layer's R_scales
+  bool transposed;
+  const void* A2;               // bf16 [M, R2]
+  const void* B2;               // U [R2, N] (forward) or D [N, R2] (transposed)
+  const void* bias;
+  void* out;
+  bool out_bf16;
+  const void* h;                // GELU-backward epilogue: saved hidden [M, N]
+  void* out2;                   // GELU-backward epilogue: bf16(GELU(h)) [M, N]
+};
+int run_gemm(const GemmArgs& a, int* status, cudaStream_t s) {
+  CUtensorMap tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, tmO2;
+  // compact scale tiles by TMA when every scale row is a whole number of 16-byte units
+  const bool sf_tma = a.K % 256 == 0 && a.N % 256 == 0 && al16(a.a_scales) && al16(a.r_scales);
+  if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, ft::kGemmBN) ||
+      !map_bf16(&tmA2, a.A2, a.R2, a.M, 128))
+    return FT_ERR_CUDA;
+  if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, ft::kGemmBN) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
+    return FT_ERR_CUDA;
+  if (sf_tma) {
+    if (!map_scales(&tmSA, a.a_scales, a.K / 16, a.M / 16, 8)) return FT_ERR_CUDA;
+    // R_scales is [N_R/16, K_R/16]; transposed form: N_R = this GEMM's K, K_R = its N
+    if (a.transposed ? !map_scales(&tmSB, a.r_scales, a.N / 16, a.K / 16, 16)
+                     : !map_scales(&tmSB, a.r_scales, a.K / 16, a.N / 16, ft::kGemmBN / 16))
+      return FT_ERR_CUDA;
+  } else {
+    tmSA = tmSB = tmA;  // unused
+  }
+  if (!map_out(&tmO, a.out, a.N, a.M, a.out_bf16)) return FT_ERR_CUDA;
+  if (a.out2) {
+    if (!map_out(&tmO2, a.out2, a.N, a.M, true)) return FT_ERR_CUDA;
+  } else {
+    tmO2 = tmO;  // unused
+  }
+  GemmParams gp{};
+  gp.M = static_cast<int>(a.M);
+  gp.N = static_cast<int>(a.N);
+  gp.K = static_cast<int>(a.K);
+  gp.R2 = static_cast<int>(a.R2);
+  gp.b2_mn_major = a.transposed ? 0 : 1;
+  gp.sf_tma = sf_tma ? 1 : 0;
+  gp.sfb_transposed = a.transposed ? 1 : 0;
+  gp.sfa = a.a_scales;
+  gp.sfa_rs = a.K / 16;
+  gp.sfa_gs = 1;
+  gp.sfb = a.r_scales;
+  if (a.transposed) {  // scale of (row n of R^T, group g) = R_scales[g, n/16]
+    gp.sfb_rs = 1;
+    gp.sfb_gs = a.N / 16;
+  } else {
+    gp.sfb_rs = a.K / 16;
+    gp.sfb_gs = 1;
+  }
+  gp.bias = a.bias;
+  gp.out = a.out;
+  gp.ldo = a.N;
+  gp.out_bf16 = a.out_bf16 ? 1 : 0;
+  gp.epi_gelu_bwd = a.h ? 1 : 0;
+  gp.h = a.h;
+  gp.status = status;
+  return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, tmO2, gp, s));
+}
+
+// dA = T_A^T V_A[:, r_s:] ([K, r]) and dB = (L[:, r_s:]^T G) ([r, N]) of one layer, one launch
+int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, const void* G, const void* Lsaved,
+              float* dA, float* dB, bool accumulate, const GradPair& g, uint8_t* base, int* status,
+              cudaStream_t s) {
+  const int64_t R = rank_all(L);
+  CUtensorMap tmTa, tmVa, tmTb, tmVb;
+  if (!map_bf16(&tmTa, X, L->K, M, 128) || !map_bf16(&tmVa, P, R, M, 128) || !map_bf16(&tmTb, G, L->N, M, 128) ||
+      !map_bf16(&tmVb, Lsaved, R, M, 128))
+    return FT_ERR_CUDA;
+  TgradParams ta{}, tb{};
+  ta.M = tb.M = static_cast<int>(M);
+  ta.r = tb.r = static_cast<int>(L->r);
+  ta.v0 = tb.v0 = static_cast<int>(L->r_s);
+  ta.accumulate = tb.accumulate = accumulate ? 1 : 0;
+  ta.status = tb.status = status;
+  ta.P = static_cast<int>(L->K);
+  ta.mt_per_split = g.sA.mt_per_split;
+  ta.nsplit = g.sA.nsplit;
+  ta.out = dA;
+  ta.out_sp = L->r;
+  ta.out_sj = 1;
+  ta.part = reinterpret_cast<float*>(base + g.partA);
+  ta.counters = reinterpret_cast<int*>(base + g.cntA);
+  tb.P = static_cast<int>(L->N);
+  tb.mt_per_split = g.sB.mt_per_split;
+  tb.nsplit = g.sB.nsplit;
+  tb.out = dB;
+  tb.out_sp = 1;
+  tb.out_sj = L->N;
+  tb.part = reinterpret_cast<float*>(base + g.partB);
+  tb.counters = reinterpret_cast<int*>(base + g.cntB);
+  return cuda_err(ft::launch_tgrad2(tmTa, tmVa, ta, tmTb, tmVb, tb, s));
+}
+
+#define FT_TRY(k, expr)                                          \
+  do {                                                           \
+    if (evs.mark((k), 0, s) != cudaSuccess) return FT_ERR_CUDA;  \
+    const int rc_ = (expr);                                      \
+    if (rc_ != FT_OK) return rc_;                                \
+    if (evs.mark((k), 1, s) != cudaSuccess) return FT_ERR_CUDA;  \
+  } while (0)
 
 }  // namespace
 
@@ -261,9 +461,10 @@ int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, u
                                              static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------- linear
 size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M) {
   if (check_layer(layer, false) || M <= 0 || M % 16) return 0;
-  return fwd_layout(layer, M, num_sms_or_default()).total;
+  return fwd_layout(layer, M).total;
 }
 
 size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M) {
@@ -274,9 +475,9 @@ size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M) {
 int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off) {
   int st = check_layer(layer, false);
   if (st) return st;
-  FwdWs w = fwd_layout(layer, M, num_sms_or_default());
-  if (codes_off) *codes_off = w.codes;
-  if (scales_off) *scales_off = w.scales;
+  const FwdWs w = fwd_layout(layer, M);
+  if (codes_off) *codes_off = w.qx.codes;
+  if (scales_off) *scales_off = w.qx.scales;
   return FT_OK;
 }
 
@@ -284,9 +485,9 @@ int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* 
                                    size_t* P_off) {
   int st = check_layer(layer, true);
   if (st) return st;
-  BwdWs w = bwd_layout(layer, M, num_sms_or_default());
-  if (codes_off) *codes_off = w.codes;
-  if (scales_off) *scales_off = w.scales;
+  const BwdWs w = bwd_layout(layer, M, num_sms_or_default());
+  if (codes_off) *codes_off = w.qg.codes;
+  if (scales_off) *scales_off = w.qg.scales;
   if (P_off) *P_off = w.P;
   return FT_OK;
 }
@@ -309,69 +510,34 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   if (!al16(X) || !al16(Y) || !al16(L_saved) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return FT_ERR_ALIGN;
   DevInfo di;
   if ((st = device_info(&di))) return st;
-  const FwdWs w = fwd_layout(layer, M, di.num_sms);
+  const FwdWs w = fwd_layout(layer, M);
   if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const int64_t K = layer->K, N = layer->N, R = layer->r_s + layer->r;
   int* status = reinterpret_cast<int*>(base);
   if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
-
-  // X pass: Q(X) and L = bf16(X D), D = [S_dn | A] read MN-major
-  CUtensorMap tmX, tmW;
-  if (!map_bf16(&tmX, X, K, M, 128) || !map_bf16(&tmW, layer->D, R, K, 64)) return FT_ERR_CUDA;
-  RowpassParams rp{};
-  rp.M = static_cast<int>(M);
-  rp.K = static_cast<int>(K);
-  rp.R = static_cast<int>(R);
-  rp.w_mn_major = 1;
-  rp.kt_per_split = w.rs.kt_per_split;
-  rp.nsplit = w.rs.nsplit;
-  rp.cluster_reduce = w.rs.nsplit > 1;
-  rp.codes = base + w.codes;
-  rp.scales = base + w.scales;
-  rp.L = L_saved;
-  rp.part = reinterpret_cast<float*>(base + w.part);
-  rp.counters = reinterpret_cast<int*>(base + w.counters);
-  rp.status = status;
-  FT_LAUNCH(0, ft::launch_rowpass(tmX, tmW, rp, s));
-
-  // 4-bit GEMM + L U + bias, U = [S_up ; B] read MN-major
-  CUtensorMap tmA, tmB, tmA2, tmB2, tmSA, tmSB;
-  const bool sf_tma = scales_by_tma(K, N, base + w.scales, layer->R_scales);
-  if (!map_codes(&tmA, base + w.codes, K, M, 128) || !map_codes(&tmB, layer->R_codes, K, N, ft::kGemmBN) ||
-      !map_bf16(&tmA2, L_saved, R, M, 128) || !map_bf16(&tmB2, layer->U, N, R, 64))
-    return FT_ERR_CUDA;
-  if (sf_tma) {
-    if (!map_scales(&tmSA, base + w.scales, K / 16, M / 16, 8) ||
-        !map_scales(&tmSB, layer->R_scales, K / 16, N / 16, ft::kGemmBN / 16))
-      return FT_ERR_CUDA;
-  } else {
-    tmSA = tmA;  // unused
-    tmSB = tmA;
-  }
-  GemmParams gp{};
-  gp.M = static_cast<int>(M);
-  gp.N = static_cast<int>(N);
-  gp.K = static_cast<int>(K);
-  gp.R2 = static_cast<int>(R);
-  gp.b2_mn_major = 1;
-  gp.sf_tma = sf_tma ? 1 : 0;
-  gp.sfb_transposed = 0;
-  gp.sfa = base + w.scales;
-  gp.sfa_rs = K / 16;
-  gp.sfa_gs = 1;
-  gp.sfb = layer->R_scales;
-  gp.sfb_rs = K / 16;
-  gp.sfb_gs = 1;
-  gp.bias = layer->bias;
-  gp.out = Y;
-  gp.ldo = N;
-  gp.out_bf16 = y_dtype == FT_DTYPE_BF16;
-  gp.status = status;
-  CUtensorMap tmO;
-  if (!map_out(&tmO, Y, N, M, gp.out_bf16 != 0)) return FT_ERR_CUDA;
-  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, gp, s));
+  const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
+  uint8_t* qc = base + w.qx.codes;
+  uint8_t* qs = base + w.qx.scales;
+  // X pass: Q(X) and L = bf16(X D)
+  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, L_saved, status, di.num_sms, s));
+  // 4-bit GEMM + L U + bias
+  GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.R2 = R;
+  g.a_codes = qc;
+  g.a_scales = qs;
+  g.b_codes = layer->R_codes;
+  g.r_scales = layer->R_scales;
+  g.transposed = false;
+  g.A2 = L_saved;
+  g.B2 = layer->U;
+  g.bias = layer->bias;
+  g.out = Y;
+  g.out_bf16 = y_dtype == FT_DTYPE_BF16;
+  FT_TRY(1, run_gemm(g, status, s));
   return FT_OK;
 }
 
@@ -402,99 +568,203 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const int64_t K = layer->K, N = layer->N, R = layer->r_s + layer->r;
   int* status = reinterpret_cast<int*>(base);
   if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
-
-  // G pass: Q(G) and P = bf16(G U^T), U = [S_up ; B] [R, N] read K-major
-  CUtensorMap tmG, tmU;
-  if (!map_bf16(&tmG, dY, N, M, 128) || !map_bf16(&tmU, layer->U, N, R, static_cast<uint32_t>(R)))
-    return FT_ERR_CUDA;
-  RowpassParams rp{};
-  rp.M = static_cast<int>(M);
-  rp.K = static_cast<int>(N);
-  rp.R = static_cast<int>(R);
-  rp.w_mn_major = 0;
-  rp.kt_per_split = w.rs.kt_per_split;
-  rp.nsplit = w.rs.nsplit;
-  rp.cluster_reduce = w.rs.nsplit > 1;
-  rp.codes = base + w.codes;
-  rp.scales = base + w.scales;
-  rp.L = base + w.P;
-  rp.part = reinterpret_cast<float*>(base + w.part_rp);
-  rp.counters = reinterpret_cast<int*>(base + w.cnt_rp);
-  rp.status = status;
-  FT_LAUNCH(0, ft::launch_rowpass(tmG, tmU, rp, s));
-
-  // dX = deq(Q(G)) deq(Q(R)) + P D^T : B operand = R^T codes, R's scales read transposed,
-  // D = [S_dn | A] [K, R] read K-major
-  CUtensorMap tmA, tmB, tmA2, tmB2, tmSA, tmSB;
-  const bool sf_tma = scales_by_tma(K, N, base + w.scales, layer->R_scales);
-  if (!map_codes(&tmA, base + w.codes, N, M, 128) || !map_codes(&tmB, layer->R_codes_t, N, K, ft::kGemmBN) ||
-      !map_bf16(&tmA2, base + w.P, R, M, 128) || !map_bf16(&tmB2, layer->D, R, K, ft::kGemmBN))
-    return FT_ERR_CUDA;
-  if (sf_tma) {
-    if (!map_scales(&tmSA, base + w.scales, N / 16, M / 16, 8) ||
-        !map_scales(&tmSB, layer->R_scales, K / 16, N / 16, 16))
-      return FT_ERR_CUDA;
-  } else {
-    tmSA = tmA;  // unused
-    tmSB = tmA;
-  }
-  GemmParams gp{};
-  gp.M = static_cast<int>(M);
-  gp.N = static_cast<int>(K);
-  gp.K = static_cast<int>(N);
-  gp.R2 = static_cast<int>(R);
-  gp.b2_mn_major = 0;
-  gp.sf_tma = sf_tma ? 1 : 0;
-  gp.sfb_transposed = 1;
-  gp.sfa = base + w.scales;
-  gp.sfa_rs = N / 16;
-  gp.sfa_gs = 1;
-  gp.sfb = layer->R_scales;  // scale of (row k of R^T, group g over N) = R_scales[g, k/16]
-  gp.sfb_rs = 1;
-  gp.sfb_gs = K / 16;
-  gp.bias = nullptr;
-  gp.out = dX;
-  gp.ldo = K;
-  gp.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  gp.status = status;
-  CUtensorMap tmO;
-  if (!map_out(&tmO, dX, K, M, gp.out_bf16 != 0)) return FT_ERR_CUDA;
-  FT_LAUNCH(1, ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, gp, s));
-
-  // dA = X^T P[:, r_s:] and dB = L[:, r_s:]^T G (computed as dB^T, stored transposed), one launch
-  CUtensorMap tmTa, tmVa, tmTb, tmVb;
-  if (!map_bf16(&tmTa, X, K, M, 128) || !map_bf16(&tmVa, base + w.P, R, M, 128) ||
-      !map_bf16(&tmTb, dY, N, M, 128) || !map_bf16(&tmVb, L_saved, R, M, 128))
-    return FT_ERR_CUDA;
-  TgradParams ta{}, tb{};
-  ta.M = tb.M = static_cast<int>(M);
-  ta.r = tb.r = static_cast<int>(layer->r);
-  ta.v0 = tb.v0 = static_cast<int>(layer->r_s);
-  ta.accumulate = tb.accumulate = accumulate ? 1 : 0;
-  ta.status = tb.status = status;
-  ta.P = static_cast<int>(K);
-  ta.mt_per_split = w.sA.mt_per_split;
-  ta.nsplit = w.sA.nsplit;
-  ta.out = dA;
-  ta.out_sp = layer->r;
-  ta.out_sj = 1;
-  ta.part = reinterpret_cast<float*>(base + w.part_dA);
-  ta.counters = reinterpret_cast<int*>(base + w.cnt_dA);
-  tb.P = static_cast<int>(N);
-  tb.mt_per_split = w.sB.mt_per_split;
-  tb.nsplit = w.sB.nsplit;
-  tb.out = dB;
-  tb.out_sp = 1;
-  tb.out_sj = N;
-  tb.part = reinterpret_cast<float*>(base + w.part_dB);
-  tb.counters = reinterpret_cast<int*>(base + w.cnt_dB);
-  FT_LAUNCH(2, ft::launch_tgrad2(tmTa, tmVa, ta, tmTb, tmVb, tb, s));
+  const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
+  uint8_t* gc = base + w.qg.codes;
+  uint8_t* gs = base + w.qg.scales;
+  void* P = base + w.P;
+  // G pass: Q(G) and P = bf16(G U^T), U [R, N] read K-major
+  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, P, status, di.num_sms, s));
+  // dX = deq(Q(G)) deq(Q(R)) + P D^T
+  GemmArgs g{};
+  g.M = M;
+  g.N = K;
+  g.K = N;
+  g.R2 = R;
+  g.a_codes = gc;
+  g.a_scales = gs;
+  g.b_codes = layer->R_codes_t;
+  g.r_scales = layer->R_scales;
+  g.transposed = true;
+  g.A2 = P;
+  g.B2 = layer->D;
+  g.out = dX;
+  g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
+  FT_TRY(1, run_gemm(g, status, s));
+  // dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G
+  FT_TRY(2, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, s));
   return FT_OK;
 }
 
+// ---------------------------------------------------------------- MLP
+size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
+  if (check_mlp(fc1, fc2, false) || M <= 0 || M % 16) return 0;
+  return mlp_fwd_layout(fc1, M).total;
+}
+
+size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
+  if (check_mlp(fc1, fc2, true) || M <= 0 || M % 16) return 0;
+  return mlp_bwd_layout(fc1, fc2, M, num_sms_or_default()).total;
+}
+
+int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* qa_codes,
+                                size_t* qa_scales) {
+  int st = check_mlp(fc1, fc2, false);
+  if (st) return st;
+  const MlpFwdWs w = mlp_fwd_layout(fc1, M);
+  if (qa_codes) *qa_codes = w.qa.codes;
+  if (qa_scales) *qa_scales = w.qa.scales;
+  return FT_OK;
+}
+
+int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* dh_off,
+                                size_t* a_off, size_t* qdh_codes, size_t* qdh_scales) {
+  int st = check_mlp(fc1, fc2, true);
+  if (st) return st;
+  const MlpBwdWs w = mlp_bwd_layout(fc1, fc2, M, num_sms_or_default());
+  if (dh_off) *dh_off = w.dh;
+  if (a_off) *a_off = w.abf;
+  if (qdh_codes) *qdh_codes = w.qdh.codes;
+  if (qdh_scales) *qdh_scales = w.qdh.scales;
+  return FT_OK;
+}
+
+int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
+                     int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a, void* ws,
+                     size_t ws_bytes, void* stream) {
+  const Events evs{nullptr, 0};
+  int st = check_mlp(fc1, fc2, false);
+  if (st) return st;
+  if (!X || !Y || !h_saved || !L1_saved || !L2_saved || !ws) return FT_ERR_INVALID_ARG;
+  if (y_dtype != FT_DTYPE_F32 && y_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(X) || !al16(Y) || !al16(h_saved) || !al16(L1_saved) || !al16(L2_saved) || (dbg_a && !al16(dbg_a)) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const MlpFwdWs w = mlp_fwd_layout(fc1, M);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
+  // FC1: X pass, then 4-bit GEMM + L1 U1 + b1 -> h (bf16, saved)
+  FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
+                        L1_saved, status, di.num_sms, s));
+  GemmArgs g{};
+  g.M = M;
+  g.N = H;
+  g.K = K1;
+  g.R2 = R1;
+  g.a_codes = base + w.qx.codes;
+  g.a_scales = base + w.qx.scales;
+  g.b_codes = fc1->R_codes;
+  g.r_scales = fc1->R_scales;
+  g.A2 = L1_saved;
+  g.B2 = fc1->U;
+  g.bias = fc1->bias;
+  g.out = h_saved;
+  g.out_bf16 = true;
+  FT_TRY(1, run_gemm(g, status, s));
+  // GELU pass over h: Q(a) of a = GELU(h) and L2 = bf16(bf16(a) D2)
+  FT_TRY(2, run_rowpass(h_saved, M, H, fc2->D, R2, true, true, dbg_a, base + w.qa.codes, base + w.qa.scales,
+                        L2_saved, status, di.num_sms, s));
+  // FC2: 4-bit GEMM + L2 U2 + b2 -> Y
+  GemmArgs g2{};
+  g2.M = M;
+  g2.N = N2;
+  g2.K = H;
+  g2.R2 = R2;
+  g2.a_codes = base + w.qa.codes;
+  g2.a_scales = base + w.qa.scales;
+  g2.b_codes = fc2->R_codes;
+  g2.r_scales = fc2->R_scales;
+  g2.A2 = L2_saved;
+  g2.B2 = fc2->U;
+  g2.bias = fc2->bias;
+  g2.out = Y;
+  g2.out_bf16 = y_dtype == FT_DTYPE_BF16;
+  FT_TRY(3, run_gemm(g2, status, s));
+  return FT_OK;
+}
+
+int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY, const ft_bf16* X,
+                     const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M, void* dX,
+                     int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate, void* ws,
+                     size_t ws_bytes, void* stream) {
+  const Events evs{nullptr, 0};
+  int st = check_mlp(fc1, fc2, true);
+  if (st) return st;
+  if (!dY || !X || !h_saved || !L1_saved || !L2_saved || !dX || !dA1 || !dB1 || !dA2 || !dB2 || !ws)
+    return FT_ERR_INVALID_ARG;
+  if (dx_dtype != FT_DTYPE_F32 && dx_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(dY) || !al16(X) || !al16(h_saved) || !al16(L1_saved) || !al16(L2_saved) || !al16(dX) || !al16(dA1) ||
+      !al16(dB1) || !al16(dA2) || !al16(dB2) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const MlpBwdWs w = mlp_bwd_layout(fc1, fc2, M, di.num_sms);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
+  void* P2 = base + w.P2;
+  void* dh = base + w.dh;
+  void* abf = base + w.abf;
+  void* P1 = base + w.P1;
+  // FC2 backward: G pass (Q(G), P2), dX GEMM with the GELU-backward epilogue
+  FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales, P2,
+                        status, di.num_sms, s));
+  GemmArgs g{};
+  g.M = M;
+  g.N = H;
+  g.K = N2;
+  g.R2 = R2;
+  g.a_codes = base + w.qg.codes;
+  g.a_scales = base + w.qg.scales;
+  g.b_codes = fc2->R_codes_t;
+  g.r_scales = fc2->R_scales;
+  g.transposed = true;
+  g.A2 = P2;
+  g.B2 = fc2->D;
+  g.out = dh;
+  g.out_bf16 = true;
+  g.h = h_saved;
+  g.out2 = abf;
+  FT_TRY(1, run_gemm(g, status, s));
+  // FC2 adapter gradients on bf16(GELU(h)) and G
+  FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, base, status, s));
+  // FC1 backward on d_h: G pass, dX GEMM, adapter gradients
+  FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales, P1,
+                        status, di.num_sms, s));
+  GemmArgs g1{};
+  g1.M = M;
+  g1.N = K1;
+  g1.K = H;
+  g1.R2 = R1;
+  g1.a_codes = base + w.qdh.codes;
+  g1.a_scales = base + w.qdh.scales;
+  g1.b_codes = fc1->R_codes_t;
+  g1.r_scales = fc1->R_scales;
+  g1.transposed = true;
+  g1.A2 = P1;
+  g1.B2 = fc1->D;
+  g1.out = dX;
+  g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
+  FT_TRY(4, run_gemm(g1, status, s));
+  FT_TRY(5, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status, s));
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------- static-scratch row pass
 int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
                                uint8_t* codes, uint8_t* scales, ft_bf16* L, void* stream) {
   if (!X || !W || !codes || !scales || !L) return FT_ERR_INVALID_ARG;
@@ -504,7 +774,7 @@ int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_
   DevInfo di;
   int st = device_info(&di);
   if (st) return st;
-  // W^T [R, K] read K-major (the backward pass's layout) with its own split choice
+  // W^T [R, K] read K-major; split partials in the library's static array
   const RowSplit rs = row_split(M, K, R, 0, di.num_sms, 1 << 20);
   const size_t header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
   const size_t need = header + (rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * M * R * 4 : 0);

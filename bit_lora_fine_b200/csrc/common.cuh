@@ -346,6 +346,38 @@ __device__ __forceinline__ void quantize_2blocks(const float* v, const float* am
   }
 }
 
+// Block16 quantization of 32 float32 values (two 16-column blocks) with the
+// IEEE division v / dec(scale) per element -- for inputs with more significant
+// bits than bf16 (the GELU output), where the division-free shortcut above does
+// not apply.  Same outputs as quantize_2blocks.
+__device__ __forceinline__ void quantize_2blocks_div(const float* v, const float* amax, uint32_t* packed,
+                                                     uint32_t* sc) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
+    const float d = e4m3_to_f32(sc[j]);
+    float q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + e], d);
+    packed[2 * j] = f32x8_to_e2m1(q);
+    packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
+  }
+}
+
+// GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))), and its
+// derivative 0.5 (1 + t) + 0.5 h (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 h^2).
+constexpr float kGeluC = 0.7978845608028654f;  // sqrt(2/pi)
+constexpr float kGeluK = 0.044715f;
+__device__ __forceinline__ float gelu_tanh(float h) {
+  const float t = tanhf(kGeluC * (h + kGeluK * h * h * h));
+  return 0.5f * h * (1.0f + t);
+}
+__device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg) {
+  const float t = tanhf(kGeluC * (h + kGeluK * h * h * h));
+  *g = 0.5f * h * (1.0f + t);
+  *dg = 0.5f * (1.0f + t) + 0.5f * h * (1.0f - t * t) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
 }  // namespace ft

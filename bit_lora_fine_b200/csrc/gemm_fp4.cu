@@ -24,7 +24,9 @@
 //                  reads (one 16-byte pattern per 16 rows)
 //   warps 4..7     epilogue: TMEM -> registers (+ bias) -> fp32/bf16 rows staged
 //                  in the now idle pipeline smem (128-byte swizzled boxes of 32
-//                  rows) -> TMA tensor stores, which clip rows/columns past M, N
+//                  rows) -> TMA tensor stores, which clip rows/columns past M, N.
+//                  MLP backward variant (FourTune §3.3 MLP): reads the saved
+//                  hidden h and writes d_h = bf16(acc * GELU'(h)) and bf16(GELU(h))
 #include "common.cuh"
 #include "kernels.h"
 
@@ -56,7 +58,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                    const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmOut2,
+                    const GemmParams p) {
   using Lay = GemmLayout<BN>;
   static_assert(Lay::kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(Lay::kTmemUsed <= 512, "TMEM budget");
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
     tma_prefetch(&tmOut);
+    if (p.epi_gelu_bwd) tma_prefetch(&tmOut2);
     if (EB) {
       tma_prefetch(&tmA2);
       tma_prefetch(&tmB2);
@@ -276,6 +280,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
       const int ebox = p.out_bf16 ? 64 : 32;               // elements per 128-byte box row
       uint8_t* region = smem + q * (BN / ebox) * 4096;
+      // GELU-backward: second bf16 tile (GELU(h)) staged after the first four warps' regions
+      uint8_t* region2 = smem + 4 * (BN / 64) * 4096 + q * (BN / 64) * 4096;
+      const int row = m0 + 32 * q + lane;
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c0, v);
@@ -289,7 +296,34 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           for (int e = 0; e < 32; ++e)
             if (nb + e < p.N) f[e] += __bfloat162float(bias[nb + e]);
         }
-        uint8_t* row = region + (c0 / ebox) * 4096 + lane * 128;
+        float g[32];
+        if (p.epi_gelu_bwd) {
+          // d_h = d_a * GELU'(h) and GELU(h), h read for this row's 32 columns
+          float hv[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) hv[e] = 0.0f;
+          if (row < p.M && nb < p.N) {
+            const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
+                                                             static_cast<long long>(row) * p.N + nb);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint4 u = hp[k];
+              const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                hv[8 * k + 2 * e] = bf16_bits_to_f32(wd[e] & 0xFFFFu);
+                hv[8 * k + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float dg;
+            gelu_tanh_and_grad(hv[e], &g[e], &dg);
+            f[e] *= dg;
+          }
+        }
+        uint8_t* rowp = region + (c0 / ebox) * 4096 + lane * 128;
         if (p.out_bf16) {
           const int j0 = (c0 % 64) / 8;                    // first 16-byte chunk of this 32-column slice
 #pragma unroll
@@ -300,12 +334,25 @@ __global__ void __launch_bounds__(kGmThreads, 1)
               const __nv_bfloat162 b = __floats2bfloat162_rn(f[8 * k + 2 * e], f[8 * k + 2 * e + 1]);
               w[e] = *reinterpret_cast<const uint32_t*>(&b);
             }
-            *reinterpret_cast<uint4*>(row + (((j0 + k) ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(rowp + (((j0 + k) ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          if (p.epi_gelu_bwd) {
+            uint8_t* rowg = region2 + (c0 / 64) * 4096 + lane * 128;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(g[8 * k + 2 * e], g[8 * k + 2 * e + 1]);
+                w[e] = *reinterpret_cast<const uint32_t*>(&b);
+              }
+              *reinterpret_cast<uint4*>(rowg + (((j0 + k) ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         } else {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(row + ((k ^ (lane & 7)) * 16)) =
+            *reinterpret_cast<uint4*>(rowp + ((k ^ (lane & 7)) * 16)) =
                 make_uint4(__float_as_uint(f[4 * k]), __float_as_uint(f[4 * k + 1]), __float_as_uint(f[4 * k + 2]),
                            __float_as_uint(f[4 * k + 3]));
         }
@@ -316,6 +363,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         for (int b = 0; b < BN / ebox; ++b) {
           const int x = n0 + b * ebox;
           if (x < p.N) tma_store_2d(&tmOut, region + b * 4096, x, m0 + 32 * q);
+          if (x < p.N && p.epi_gelu_bwd) tma_store_2d(&tmOut2, region2 + b * 4096, x, m0 + 32 * q);
         }
         bulk_commit();
         bulk_wait_read_all();
@@ -335,14 +383,16 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
-                            const CUtensorMap& tmOut, const GemmParams& p, cudaStream_t stream) {
+                            const CUtensorMap& tmOut, const CUtensorMap& tmOut2, const GemmParams& p,
+                            cudaStream_t stream) {
   constexpr int BN = kGemmBN;
   using Lay = GemmLayout<BN>;
   cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Lay::kSmem));
   if (e != cudaSuccess) return e;
   dim3 grid((p.N + BN - 1) / BN, (p.M + 127) / 128);
-  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, tmSFA, tmSFB, tmOut, p);
+  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, tmSFA, tmSFB, tmOut,
+                                                                  tmOut2, p);
   return cudaGetLastError();
 }
 

@@ -15,6 +15,8 @@ struct RowpassParams {
   int w_mn_major;                        // 1: D [K, R]; 0: W^T [R, K]
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
   int cluster_reduce;                    // splits of a row tile form a cluster and reduce through DSMEM
+  int gelu_input;                        // input is h: quantize a = GELU(h) (fp32) and project bf16(a)
+  float* dbg_a;                          // gelu_input: optional fp32 copy of a [M, K] (null = none)
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
   void* L;                               // bf16 [M, R]
@@ -43,6 +45,10 @@ struct GemmParams {
   void* out;
   long long ldo;
   int out_bf16;
+  // GELU-backward epilogue: out = bf16(acc * GELU'(h)), out2 = bf16(GELU(h)),
+  // h bf16 [M, N] with row stride N (both outputs bf16, out2 through tmOut2)
+  int epi_gelu_bwd;
+  const void* h;
   int* status;
 };
 
@@ -68,7 +74,8 @@ int rowpass_ctas_per_sm(int R, int w_mn_major);
 // tmOut: the output [M, N] (fp32 or bf16) with 128-byte x 32-row boxes, 128-byte swizzle
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
-                            const CUtensorMap& tmOut, const GemmParams& p, cudaStream_t stream);
+                            const CUtensorMap& tmOut, const CUtensorMap& tmOut2, const GemmParams& p,
+                            cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
                           const CUtensorMap& tmT1, const CUtensorMap& tmV1, const TgradParams& p1,
                           cudaStream_t stream);

@@ -64,7 +64,8 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRpStages * stage_bytes);
   uint64_t* empty = full + kRpStages;
   uint64_t* acc_full = empty + kRpStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* ready = acc_full + 1;  // [kRpStages] GELU mode: transformed tile written back
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + kRpStages);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
   volatile int* s_ok = s_last + 1;  // [kRpQuantWarps]
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       mbar_init(&empty[s], 1 + kRpQuantWarps);  // MMA commit + one arrive per quantizer warp
     }
     mbar_init(acc_full, 1);
+    for (int s = 0; s < kRpStages; ++s) mbar_init(&ready[s], kRpQuantWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         const int s = i % kRpStages;
         const uint32_t ph = (i / kRpStages) & 1;
         if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
+        if (p.gelu_input && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(smem + s * stage_bytes);
         const uint32_t wa = xa + kRpXBytes;
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         ok = false;
         break;
       }
-      const uint8_t* tile = smem + s * stage_bytes;
+      uint8_t* tile = smem + s * stage_bytes;
       float v[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -172,8 +175,31 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
+      if (p.gelu_input) {
+        // a = GELU(h) in fp32; bf16(a) goes back into the tile for the down-projection
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = gelu_tanh(v[e]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t wd[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
+            wd[e] = *reinterpret_cast<const uint32_t*>(&b);
+          }
+          const int phys = (4 * h + q) ^ (r & 7);
+          *reinterpret_cast<uint4*>(tile + r * 128 + phys * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ready[s]);
+          mbar_arrive(&empty[s]);
+        }
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
+      }
       float amax[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -187,13 +213,21 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       const int cstart = (kt0 + i) * 64 + 32 * h;
       if (block_row_ok && cstart < p.K) {
         uint32_t packed[4], sc[2];
-        quantize_2blocks(v, amax, packed, sc);
+        if (p.gelu_input)
+          quantize_2blocks_div(v, amax, packed, sc);
+        else
+          quantize_2blocks(v, amax, packed, sc);
         *reinterpret_cast<uint4*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
             make_uint4(packed[0], packed[1], packed[2], packed[3]);
         if ((lane >> 1) == 0) {
           const long long srow = (m0 / 16 + w8) * static_cast<long long>(kblocks);
           p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
           p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
+        }
+        if (p.dbg_a) {
+          float4* dst = reinterpret_cast<float4*>(p.dbg_a + static_cast<long long>(m0 + r) * p.K + cstart);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
         }
       }
     }

@@ -24,7 +24,9 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_linear_bwd_workspace_size", "fourtune_linear_fwd", "fourtune_linear_bwd",
             "fourtune_linear_fwd_ws_offsets", "fourtune_linear_bwd_ws_offsets", "fourtune_device_status",
             "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed",
-            "fourtune_quant_down_static")
+            "fourtune_quant_down_static", "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_fwd",
+            "fourtune_mlp_bwd_workspace_size", "fourtune_mlp_bwd", "fourtune_mlp_fwd_ws_offsets",
+            "fourtune_mlp_bwd_ws_offsets")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
@@ -73,8 +75,19 @@ def load():
     L.fourtune_device_status.argtypes = [vp, vp]
     L.fourtune_error_string.argtypes = [ctypes.c_int]
     L.fourtune_error_string.restype = ctypes.c_char_p
+    PL = P(ft_linear_t)
+    L.fourtune_mlp_fwd_workspace_size.argtypes = [PL, PL, i64]
+    L.fourtune_mlp_fwd_workspace_size.restype = sz
+    L.fourtune_mlp_bwd_workspace_size.argtypes = [PL, PL, i64]
+    L.fourtune_mlp_bwd_workspace_size.restype = sz
+    L.fourtune_mlp_fwd.argtypes = [PL, PL, vp, i64, vp, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
+    L.fourtune_mlp_bwd.argtypes = [PL, PL, vp, vp, vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, vp, vp,
+                                   ctypes.c_int, vp, sz, vp]
+    L.fourtune_mlp_fwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz)]
+    L.fourtune_mlp_bwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz), P(sz), P(sz)]
     for f in EXPORTED:
         if f not in ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size",
+                     "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
                      "fourtune_error_string"):
             getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -226,6 +239,78 @@ def linear_bwd(layer, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumu
         arr, n = _events(events)
         _check(load().fourtune_linear_bwd_timed(*args, arr, n), "fourtune_linear_bwd_timed")
     return dX, dA, dB, ws
+
+
+class MLP:
+    """FC1 -> GELU(tanh) -> FC2, two Linear layers with fc1.N == fc2.K (FourTune §3.3)."""
+
+    def __init__(self, fc1, fc2):
+        if fc1.N != fc2.K:
+            raise ValueError("fc1.N must equal fc2.K")
+        self.fc1, self.fc2 = fc1, fc2
+        self.H = fc1.N
+
+    def _ws(self, fn, M):
+        n = fn(ctypes.byref(self.fc1.c), ctypes.byref(self.fc2.c), M)
+        if n == 0:
+            raise FourtuneError(-2, "fourtune_mlp_*_workspace_size")
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def fwd_workspace(self, M):
+        return self._ws(load().fourtune_mlp_fwd_workspace_size, M)
+
+    def bwd_workspace(self, M):
+        return self._ws(load().fourtune_mlp_bwd_workspace_size, M)
+
+    def fwd_ws_offsets(self, M):
+        c, s = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().fourtune_mlp_fwd_ws_offsets(ctypes.byref(self.fc1.c), ctypes.byref(self.fc2.c), M,
+                                                  ctypes.byref(c), ctypes.byref(s)), "fourtune_mlp_fwd_ws_offsets")
+        return c.value, s.value
+
+    def bwd_ws_offsets(self, M):
+        o = [ctypes.c_size_t() for _ in range(4)]
+        _check(load().fourtune_mlp_bwd_ws_offsets(ctypes.byref(self.fc1.c), ctypes.byref(self.fc2.c), M,
+                                                  *[ctypes.byref(x) for x in o]), "fourtune_mlp_bwd_ws_offsets")
+        return tuple(x.value for x in o)
+
+
+def mlp_fwd(mlp, X, y_dtype=torch.float32, ws=None, dbg_a=False):
+    """Returns (Y, h, L1, L2, ws, a) -- a is the fp32 activation when dbg_a, else None."""
+    _need(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    dev = X.device
+    Y = torch.empty((M, mlp.fc2.N), dtype=y_dtype, device=dev)
+    h = torch.empty((M, mlp.H), dtype=torch.bfloat16, device=dev)
+    L1 = torch.empty((M, mlp.fc1.R_all), dtype=torch.bfloat16, device=dev)
+    L2 = torch.empty((M, mlp.fc2.R_all), dtype=torch.bfloat16, device=dev)
+    a = torch.empty((M, mlp.H), dtype=torch.float32, device=dev) if dbg_a else None
+    ws = mlp.fwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if y_dtype == torch.float32 else FT_DTYPE_BF16
+    _check(load().fourtune_mlp_fwd(ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(X), M, _ptr(Y), code,
+                                   _ptr(h), _ptr(L1), _ptr(L2), _ptr(a), _ptr(ws), ws.numel(), _stream()),
+           "fourtune_mlp_fwd")
+    return Y, h, L1, L2, ws, a
+
+
+def mlp_bwd(mlp, dY, X, h, L1, L2, dx_dtype=torch.float32, accumulate=False, grads=None, ws=None):
+    """Returns (dX, dA1, dB1, dA2, dB2, ws)."""
+    _need(dY, torch.bfloat16, "dY")
+    M = dY.shape[0]
+    dev = dY.device
+    dX = torch.empty((M, mlp.fc1.K), dtype=dx_dtype, device=dev)
+    if grads is None:
+        grads = (torch.zeros((mlp.fc1.K, mlp.fc1.r), dtype=torch.float32, device=dev),
+                 torch.zeros((mlp.fc1.r, mlp.fc1.N), dtype=torch.float32, device=dev),
+                 torch.zeros((mlp.fc2.K, mlp.fc2.r), dtype=torch.float32, device=dev),
+                 torch.zeros((mlp.fc2.r, mlp.fc2.N), dtype=torch.float32, device=dev))
+    dA1, dB1, dA2, dB2 = grads
+    ws = mlp.bwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if dx_dtype == torch.float32 else FT_DTYPE_BF16
+    _check(load().fourtune_mlp_bwd(ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(dY), _ptr(X), _ptr(h),
+                                   _ptr(L1), _ptr(L2), M, _ptr(dX), code, _ptr(dA1), _ptr(dB1), _ptr(dA2), _ptr(dB2),
+                                   int(accumulate), _ptr(ws), ws.numel(), _stream()), "fourtune_mlp_bwd")
+    return dX, dA1, dB1, dA2, dB2, ws
 
 
 def quant_down_static(X, W, codes=None, scales=None, L=None):

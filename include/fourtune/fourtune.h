@@ -139,6 +139,39 @@ FT_API int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY
                                      float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
 
+/* The MLP pair (§3.3 "MLP Fusion"): y = FC2(GELU_tanh(FC1(X))), both layers
+ * triple-branch, fc1 [K1 -> H], fc2 [H -> N2] (fc1->N == fc2->K).
+ * Forward: the X pass and FC1's 4-bit GEMM (+ bias b1) give the hidden
+ * h = bf16(FC1(X)) [M, H] (saved).  One fused pass over h then computes
+ * a = GELU_tanh(h) in fp32, quantizes it (Q(a), block16 of the fp32 values)
+ * and projects bf16(a) onto FC2's D: L2 = bf16(bf16(a) D2) -- a is never
+ * stored.  FC2's 4-bit GEMM adds L2 U2 and b2.  Writes Y [M, N2], h_saved
+ * [M, H], L1_saved [M, r_s1 + r1], L2_saved [M, r_s2 + r2]; dbg_a, when not
+ * NULL, receives the fp32 a [M, H] that was quantized (for inspection). */
+FT_API size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
+FT_API int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
+                            int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* MLP backward.  FC2's dX GEMM ends in the GELU backward: it reads h and writes
+ * d_h = bf16(d_a * GELU'(h)) and bf16(GELU(h)) into the workspace; FC2's dA2
+ * uses the latter, FC1's backward takes d_h as its incoming gradient (all
+ * three branches).  Writes dX [M, K1] and the four adapter gradients (fp32;
+ * accumulate = 1 adds). */
+FT_API size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
+FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY, const ft_bf16* X,
+                            const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
+                            void* dX, int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace byte offsets of the MLP's intermediate tensors (inspection, tests):
+ * forward: Q(a) codes [M, H/2] and scales [M/16, H/16]; backward: d_h and
+ * bf16(GELU(h)) (both bf16 [M, H]) and Q(d_h) codes and scales. */
+FT_API int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* qa_codes,
+                                       size_t* qa_scales);
+FT_API int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* dh_off,
+                                       size_t* a_off, size_t* qdh_codes, size_t* qdh_scales);
+
 /* Byte offsets, inside the workspace of the last fwd / bwd call with these sizes,
  * of the block16 activation (fwd: Q(X)) or gradient (bwd: Q(G)) codes and scales,
  * and (bwd) of P [M, r_s + r] bf16.  For inspection and tests; unused -> NULL. */
