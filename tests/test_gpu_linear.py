@@ -147,3 +147,59 @@ def test_repeated_calls_are_bit_identical(cuda_lib):
     for other in outs[1:]:
         for a, b in zip(outs[0], other):
             assert torch.equal(a, b)
+
+
+def run_sampled(ft, p, X, dY, rows):
+    """Full-size linear fwd+bwd; y, Q(X), Q(G), dX, L, P on sampled 16-row blocks
+    against the oracle; dA and dB in full from the GPU's own L and P."""
+    import torch
+    M = X.shape[0]
+    lay = _device_layer(ft, p)
+    K, N, r_s = lay.K, lay.N, lay.r_s
+    Rc, Rs = block16.quantize(p["R"])
+    Xd, dYd = to_dev_bf16(X), to_dev_bf16(dY)
+    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32)
+    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32)
+    ft.device_status(ws)
+    ft.device_status(wsb)
+    co, so = lay.fwd_ws_offsets(M)
+    gc, gs, po = lay.bwd_ws_offsets(M)
+    blocks = np.unique(rows // 16)
+    qx = ws[co:co + M * K // 2].view(M, K // 2).cpu().numpy()[rows]
+    qxs = ws[so:so + (M // 16) * (K // 16)].view(M // 16, K // 16).cpu().numpy()[blocks]
+    qg = wsb[gc:gc + M * N // 2].view(M, N // 2).cpu().numpy()[rows]
+    qgs = wsb[gs:gs + (M // 16) * (N // 16)].view(M // 16, N // 16).cpu().numpy()[blocks]
+    Lh = to_host(L)
+    P = to_host(wsb[po:po + M * lay.R_all * 2].view(torch.bfloat16).view(M, lay.R_all))
+
+    ref = olayer.linear_fwd(X[rows], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
+    np.testing.assert_array_equal(qxs, ref["qx_scales"])
+    np.testing.assert_array_equal(qx, ref["qx_codes"])
+    D = np.concatenate([p["S_dn"], p["A"]], axis=1).astype(np.float64)
+    check_bf16_dot(Lh[rows], ref["L"], np.abs(X[rows]) @ np.abs(D), K)
+    assert normwise(to_host(Y)[rows], ref["y"]) <= TOL
+    b = olayer.linear_bwd(dY[rows], X[rows], Lh[rows], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"])
+    np.testing.assert_array_equal(qgs, b["qg_scales"])
+    np.testing.assert_array_equal(qg, b["qg_codes"])
+    U = np.concatenate([p["S_up"], p["B"]], axis=0).astype(np.float64)
+    check_bf16_dot(P[rows], b["P"], np.abs(dY[rows]) @ np.abs(U).T, N)
+    assert normwise(to_host(dX)[rows], b["dX"]) <= TOL
+    assert normwise(to_host(dA), X.astype(np.float64).T @ P[:, r_s:]) <= TOL
+    assert normwise(to_host(dB), Lh[:, r_s:].T @ dY.astype(np.float64)) <= TOL
+
+
+def _sample_rows(M, nblocks=8, seed=0):
+    rng = np.random.default_rng(seed)
+    blocks = np.sort(rng.choice(M // 16, size=nblocks, replace=False))
+    return (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+
+
+@pytest.mark.parametrize("layer", [0, 1], ids=["in-proj-3072x21504", "out-proj-15360x3072"])
+def test_config_flux_single_stream_linears(cuda_lib, layer):
+    """FLUX single-stream block linears at full size (M=4608, ranks 64/64, log-normal
+    channel scales sigma 1.5): fused in-proj 3072 -> 21504 and out-proj 15360 -> 3072."""
+    wl = synth.WORKLOADS["flux-single-stream"]
+    p = synth.layer_params(wl.layers[layer], layer=layer)
+    X = synth.layer_input(wl, layer=layer)
+    dY = synth.upstream_grad(wl, layer=layer)
+    run_sampled(cuda_lib, p, X, dY, _sample_rows(wl.M, seed=layer))

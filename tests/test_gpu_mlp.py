@@ -129,3 +129,17 @@ def test_flux_mlp_3072_sampled_rows(cuda_lib):
     blocks = np.sort(rng.choice(wl.M // 16, size=8, replace=False))
     rows = (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
     run_mlp(cuda_lib, p1, p2, X, dY, rows=rows)
+
+
+def test_video_mlp_5120_sampled_rows(cuda_lib):
+    """Video-DiT-width MLP at full size (M=32768, 5120 -> 13824 -> 5120, ranks 64/64,
+    2% outlier channels x30, weights N(0, 0.015)): sampled rows, gradients in full."""
+    wl = synth.WORKLOADS["video-mlp-5120"]
+    p1 = synth.layer_params(wl.layers[0], layer=0)
+    p2 = synth.layer_params(wl.layers[1], layer=1)
+    X = synth.layer_input(wl)
+    dY = synth.upstream_grad(wl, layer=1)
+    rng = np.random.default_rng(1)
+    blocks = np.sort(rng.choice(wl.M // 16, size=6, replace=False))
+    rows = (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+    run_mlp(cuda_lib, p1, p2, X, dY, rows=rows)
