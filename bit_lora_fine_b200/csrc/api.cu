@@ -61,9 +61,10 @@ bool map_out(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, boo
               : make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, cols, rows, cols * 4, 32, 32,
                          CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// compact scales [rows, cols] bytes, unswizzled boxes of 16 bytes x box_rows
-bool map_scales(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, cols, 16, box_rows,
+// compact scales [rows, cols] bytes, unswizzled boxes of box_cols bytes x box_rows
+bool map_scales(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, cols, box_cols, box_rows,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -330,10 +331,12 @@ int run_gemm(const GemmArgs& a, int* status, cudaStream_t s) {
   if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, ft::kGemmBN) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
     return FT_ERR_CUDA;
   if (sf_tma) {
-    if (!map_scales(&tmSA, a.a_scales, a.K / 16, a.M / 16, 8)) return FT_ERR_CUDA;
+    // one box = the scales of ft::kGemmSfGroups K-groups (several K-blocks) of the tile's rows
+    const uint32_t G = ft::kGemmSfGroups;
+    if (!map_scales(&tmSA, a.a_scales, a.K / 16, a.M / 16, G, 8)) return FT_ERR_CUDA;
     // R_scales is [N_R/16, K_R/16]; transposed form: N_R = this GEMM's K, K_R = its N
-    if (a.transposed ? !map_scales(&tmSB, a.r_scales, a.N / 16, a.K / 16, 16)
-                     : !map_scales(&tmSB, a.r_scales, a.K / 16, a.N / 16, ft::kGemmBN / 16))
+    if (a.transposed ? !map_scales(&tmSB, a.r_scales, a.N / 16, a.K / 16, ft::kGemmBN / 16, G)
+                     : !map_scales(&tmSB, a.r_scales, a.K / 16, a.N / 16, G, ft::kGemmBN / 16))
       return FT_ERR_CUDA;
   } else {
     tmSA = tmSB = tmA;  // unused

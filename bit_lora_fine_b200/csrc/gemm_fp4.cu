@@ -12,10 +12,12 @@
 //
 // CTA tile 128 x BN (BN = 256), K-block = 256 FP4 elements (one 128-byte
 // swizzle row per operand row).  Warp roles:
-//   warp 0 lane 0  TMA: A codes [128 x 128 B], B codes [BN x 128 B] and the
-//                  K-block's compact 16x16 scale tiles; for the bf16 extra
-//                  blocks A2 [128 x 64] and B2 (K-major [BN x 64] or MN-major
-//                  [64 x BN] in four boxes) into the same slots
+//   warp 0 lane 0  TMA: A codes [128 x 128 B] and B codes [BN x 128 B] per
+//                  K-block; every kSfChunk K-blocks the compact 16x16 scale
+//                  tiles of those K-blocks (two small boxes into a 2-slot ring,
+//                  so that a K-block costs two TMA boxes, not four); for the
+//                  bf16 extra blocks A2 [128 x 64] and B2 (K-major [BN x 64] or
+//                  MN-major [64 x BN] in four boxes) into the same slots
 //   warp 1         TMEM owner; lane 0 copies the stage's scale vectors smem->TMEM
 //                  (tcgen05.cp 32x128b.warpx4) and issues
 //                  tcgen05.mma kind::mxf4nvf4.block_scale.block16 (M=128, N=BN,
@@ -34,6 +36,8 @@ namespace ft {
 
 constexpr int kGmStages = 4;
 constexpr int kGmThreads = 256;
+constexpr int kSfChunk = kGemmSfGroups / 16;  // K-blocks per compact-scale load
+constexpr int kSfSlots = 2;
 
 template <int BN>
 struct GemmLayout {
@@ -43,10 +47,12 @@ struct GemmLayout {
   static constexpr uint32_t kSFA = 4 * 512;                  // 4 MMA K-steps x 512 B
   static constexpr uint32_t kSFB = 4 * kNC * 512;
   static constexpr uint32_t kStage = kA + kB + kSFA + kSFB;  // multiple of 1024
-  static constexpr uint32_t kCA = 8 * 16;                    // compact A scales: 8 row-blocks x 16 groups
-  static constexpr uint32_t kCB = (BN / 16) * 16;            // compact B scales: BN/16 row-blocks x 16 groups
-  static constexpr uint32_t kCStage = kCA + kCB;
-  static constexpr uint32_t kSmem = 1024 + kGmStages * (kStage + kCStage) + 256;
+  // compact scales of kSfChunk K-blocks: A 8 row-blocks x 64 groups; B BN/16
+  // row-blocks x 64 groups (or, read transposed, 64 groups x BN/16 row-blocks)
+  static constexpr uint32_t kCA = 8 * 16 * kSfChunk;
+  static constexpr uint32_t kCB = (BN / 16) * 16 * kSfChunk;
+  static constexpr uint32_t kCSlot = kCA + kCB;
+  static constexpr uint32_t kSmem = 1024 + kGmStages * kStage + kSfSlots * kCSlot + 256;
   // TMEM columns: accumulator, then per stage 16 (SFA) + 16*kNC (SFB)
   static constexpr uint32_t kSfColsPerStage = 16 + 16 * kNC;
   static constexpr uint32_t kTmemUsed = BN + kGmStages * kSfColsPerStage;
@@ -66,13 +72,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* compact = smem + kGmStages * Lay::kStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(compact + kGmStages * Lay::kCStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(compact + kSfSlots * Lay::kCSlot);
   uint64_t* sf_ready = full + kGmStages;
   uint64_t* empty = sf_ready + kGmStages;
   uint64_t* acc_full = empty + kGmStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* sf_full = acc_full + 1;       // [kSfSlots] compact scales landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kSfSlots);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   volatile int* abortp = abort_flag;
+  static_assert((3 * kGmStages + 1 + kSfSlots) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;
@@ -90,6 +98,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       mbar_init(&empty[s], 1);     // MMA commit
     }
     mbar_init(acc_full, 1);
+    for (int c = 0; c < kSfSlots; ++c) mbar_init(&sf_full[c], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -118,24 +127,31 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
+      int issued = 0, chunks = 0;
       for (int i = 0; i < T; ++i) {
         const int s = i % kGmStages;
         const uint32_t ph = (i / kGmStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
         uint8_t* st = smem + s * Lay::kStage;
         if (i < KB) {
-          mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + (p.sf_tma ? Lay::kCStage : 0u));
+          if (p.sf_tma && i % kSfChunk == 0) {
+            // The slot of chunk c was last read for K-block kSfChunk (c - 1) - 1,
+            // before the MMA of K-block i - kGmStages, whose commit released
+            // stage s: the slot is free.
+            const int c = i / kSfChunk;
+            uint8_t* cs = compact + (c % kSfSlots) * Lay::kCSlot;
+            uint64_t* bar = &sf_full[c % kSfSlots];
+            mbar_arrive_expect_tx(bar, Lay::kCSlot);
+            tma_load_2d(cs, &tmSFA, bar, c * 16 * kSfChunk, m0 / 16);
+            if (p.sfb_transposed)
+              tma_load_2d(cs + Lay::kCA, &tmSFB, bar, n0 / 16, c * 16 * kSfChunk);
+            else
+              tma_load_2d(cs + Lay::kCA, &tmSFB, bar, c * 16 * kSfChunk, n0 / 16);
+            chunks = c + 1;
+          }
+          mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
           tma_load_2d(st, &tmA, &full[s], i * 128, m0);
           tma_load_2d(st + Lay::kA, &tmB, &full[s], i * 128, n0);
-          if (p.sf_tma) {
-            uint8_t* cs = compact + s * Lay::kCStage;
-            tma_load_2d(cs, &tmSFA, &full[s], i * 16, m0 / 16);
-            if (p.sfb_transposed)
-              tma_load_2d(cs + Lay::kCA, &tmSFB, &full[s], n0 / 16, i * 16);
-            else
-              tma_load_2d(cs + Lay::kCA, &tmSFB, &full[s], i * 16, n0 / 16);
-          }
         } else {
           const int e = i - KB;
           mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
@@ -152,6 +168,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       if (*abortp) {
         for (int i = max(0, issued - kGmStages); i < issued; ++i)
           mbar_wait_drain(&full[i % kGmStages], (i / kGmStages) & 1, 100000000ull);
+        for (int c = max(0, chunks - kSfSlots); c < chunks; ++c)
+          mbar_wait_drain(&sf_full[c % kSfSlots], (c / kSfSlots) & 1, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -210,10 +228,12 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const uint32_t ph = (i / kGmStages) & 1;
       if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
       if (i < KB) {
-        if (p.sf_tma && !mbar_wait(&full[s], ph, p.status, abortp)) break;
+        const int c = i / kSfChunk, kk = i % kSfChunk;   // chunk, K-block within it
+        if (p.sf_tma && kk == 0 && !mbar_wait(&sf_full[c % kSfSlots], (c / kSfSlots) & 1, p.status, abortp))
+          break;
         uint8_t* sfa = smem + s * Lay::kStage + Lay::kA + Lay::kB;
         uint8_t* sfb = sfa + Lay::kSFA;
-        const uint8_t* cA = compact + s * Lay::kCStage;
+        const uint8_t* cA = compact + (c % kSfSlots) * Lay::kCSlot;
         const uint8_t* cB = cA + Lay::kCA;
         if (lane < nA + nB) {
           const bool isA = lane < nA;
@@ -226,14 +246,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const int rb = c * 8 + hh + 2 * w;   // row-block within the tile
+              const int g = 16 * kk + 4 * t;     // first K-group of this MMA step within the chunk
               if (isA) {
-                word[w] = *reinterpret_cast<const uint32_t*>(cA + rb * 16 + 4 * t);
+                word[w] = *reinterpret_cast<const uint32_t*>(cA + rb * (16 * kSfChunk) + g);
               } else if (!p.sfb_transposed) {
-                word[w] = *reinterpret_cast<const uint32_t*>(cB + rb * 16 + 4 * t);
+                word[w] = *reinterpret_cast<const uint32_t*>(cB + rb * (16 * kSfChunk) + g);
               } else {
                 uint32_t wv = 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) wv |= static_cast<uint32_t>(cB[(4 * t + j) * 16 + rb]) << (8 * j);
+                for (int j = 0; j < 4; ++j) wv |= static_cast<uint32_t>(cB[(g + j) * (BN / 16) + rb]) << (8 * j);
                 word[w] = wv;
               }
             }

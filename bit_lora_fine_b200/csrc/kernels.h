@@ -88,5 +88,7 @@ cudaError_t rowpass_static_scratch(void** out);
 // tile sizes the host needs for tensor-map boxes and workspace sizing
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
+// K-groups (of 16) per compact-scale TMA box: the scales of four 256-wide K-blocks
+constexpr int kGemmSfGroups = 64;
 
 }  // namespace ft

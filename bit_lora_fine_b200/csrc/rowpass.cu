@@ -50,8 +50,8 @@ __host__ __device__ constexpr uint32_t rp_smem_bytes(int R, int mn) {
   return 1024 + kRpStages * rp_stage_bytes(R, mn) + 256;
 }
 
-template <int RCOLS>
-__global__ void __launch_bounds__(kRpThreads, 1)
+template <int RCOLS, bool GELU>
+__global__ void __launch_bounds__(kRpThreads, 2)  // two CTAs per SM: registers <= 80
     rowpass_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const RowpassParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         const int s = i % kRpStages;
         const uint32_t ph = (i / kRpStages) & 1;
         if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
-        if (p.gelu_input && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
+        if (GELU && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(smem + s * stage_bytes);
         const uint32_t wa = xa + kRpXBytes;
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
         }
       }
-      if (p.gelu_input) {
+      if (GELU) {
         // a = GELU(h) in fp32; bf16(a) goes back into the tile for the down-projection
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = gelu_tanh(v[e]);
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       const int cstart = (kt0 + i) * 64 + 32 * h;
       if (block_row_ok && cstart < p.K) {
         uint32_t packed[4], sc[2];
-        if (p.gelu_input)
+        if (GELU)
           quantize_2blocks_div(v, amax, packed, sc);
         else
           quantize_2blocks(v, amax, packed, sc);
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
           p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
         }
-        if (p.dbg_a) {
+        if (GELU && p.dbg_a) {
           float4* dst = reinterpret_cast<float4*>(p.dbg_a + static_cast<long long>(m0 + r) * p.K + cstart);
 #pragma unroll
           for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
@@ -366,11 +366,11 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   }
 }
 
-template <int RCOLS>
+template <int RCOLS, bool GELU>
 static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                                     cudaStream_t stream) {
   const uint32_t smem = rp_smem_bytes(p.R, p.w_mn_major);
-  cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS, GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -385,15 +385,20 @@ static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& t
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, rowpass_kernel<RCOLS>, tmX, tmW, p);
+  return cudaLaunchKernelEx(&cfg, rowpass_kernel<RCOLS, GELU>, tmX, tmW, p);
 }
 
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream) {
   const int n = rp_n_mma(p.R, p.w_mn_major);
-  if (n <= 32) return launch_rowpass_t<32>(tmX, tmW, p, stream);
-  if (n <= 64) return launch_rowpass_t<64>(tmX, tmW, p, stream);
-  return launch_rowpass_t<128>(tmX, tmW, p, stream);
+  if (p.gelu_input) {
+    if (n <= 32) return launch_rowpass_t<32, true>(tmX, tmW, p, stream);
+    if (n <= 64) return launch_rowpass_t<64, true>(tmX, tmW, p, stream);
+    return launch_rowpass_t<128, true>(tmX, tmW, p, stream);
+  }
+  if (n <= 32) return launch_rowpass_t<32, false>(tmX, tmW, p, stream);
+  if (n <= 64) return launch_rowpass_t<64, false>(tmX, tmW, p, stream);
+  return launch_rowpass_t<128, false>(tmX, tmW, p, stream);
 }
 
 int rowpass_ctas_per_sm(int R, int w_mn_major) {
