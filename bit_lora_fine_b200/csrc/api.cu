@@ -55,18 +55,6 @@ bool map_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // GEMM output [rows, cols] fp32 or bf16: boxes of 128 bytes x 32 rows, 128-byte swizzle
-bool map_out(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, bool bf16) {
-  return bf16 ? make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, cols * 2, 64, 32,
-                         CU_TENSOR_MAP_SWIZZLE_128B)
-              : make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, cols, rows, cols * 4, 32, 32,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-}
-// compact scales [rows, cols] bytes, unswizzled boxes of box_cols bytes x box_rows
-bool map_scales(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
-                uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, cols, box_cols, box_rows,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
-}
 
 struct DevInfo {
   int ok = 0;  // 1 = sm_100, -1 = other
@@ -103,14 +91,14 @@ inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b)
 int cuda_err(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
 
 int check_layer(const ft_linear_t* L, bool need_t) {
-  if (!L || !L->R_codes || !L->R_scales || !L->D || !L->U) return FT_ERR_INVALID_ARG;
-  if (need_t && !L->R_codes_t) return FT_ERR_INVALID_ARG;
+  if (!L || !L->R_codes || !L->R_scales || !L->R_sf || !L->D || !L->U) return FT_ERR_INVALID_ARG;
+  if (need_t && (!L->R_codes_t || !L->R_sf_t)) return FT_ERR_INVALID_ARG;
   if (L->K <= 0 || L->N <= 0 || L->K % 32 || L->N % 32) return FT_ERR_SHAPE;
   if (L->r_s < 0 || L->r < 16 || L->r_s % 16 || L->r % 16 || L->r > 64 || L->r_s + L->r > 128)
     return FT_ERR_UNSUPPORTED;
   if (L->K > (1 << 30) || L->N > (1 << 30)) return FT_ERR_UNSUPPORTED;
-  if (!al16(L->R_codes) || !al16(L->D) || !al16(L->U) || (L->R_codes_t && !al16(L->R_codes_t)) ||
-      (L->bias && !al16(L->bias)))
+  if (!al16(L->R_codes) || !al16(L->R_sf) || !al16(L->D) || !al16(L->U) || (L->R_codes_t && !al16(L->R_codes_t)) ||
+      (L->R_sf_t && !al16(L->R_sf_t)) || (L->bias && !al16(L->bias)))
     return FT_ERR_ALIGN;
   return FT_OK;
 }
@@ -153,12 +141,14 @@ struct Carver {
     return at;
   }
 };
-// block16 activations of a [M, C] matrix
+// block16 activations of a [M, C] matrix: codes, compact scales and the same
+// scales in the MMA-ready layout the GEMM loads
 struct Q16 {
-  size_t codes, scales;
+  size_t codes, scales, sf;
   void carve(Carver& c, int64_t M, int64_t C) {
     codes = c.take(static_cast<size_t>(M * C / 2));
     scales = c.take(static_cast<size_t>((M / 16) * (C / 16)));
+    sf = c.take(ft::sf_mma_bytes(M, C));
   }
 };
 // dA/dB launch of one layer: splits, counters (in the header) and partials
@@ -280,7 +270,7 @@ struct Events {
 // with W = D [K, R] (w_mn) or W^T [R, K]; gelu: the input is h and the pass
 // quantizes GELU(h).  Split reduction inside a cluster: needs only the status word.
 int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
-                float* dbg_a, uint8_t* codes, uint8_t* scales, void* L, int* status, int num_sms,
+                float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, int* status, int num_sms,
                 cudaStream_t s) {
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
@@ -298,20 +288,22 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.dbg_a = dbg_a;
   rp.codes = codes;
   rp.scales = scales;
+  rp.sf_mma = sf_mma;
   rp.L = L;
   rp.status = status;
   return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
 
-// FP4 GEMM.  Forward form: A = Q(act) [M, K], B = layer's R [N, K], B2 = U [R2, N]
-// (MN-major).  Transposed form (dX): B = R^T from R_codes_t, scales read
-// transposed, B2 = D [N_out, R2] (K-major).
+// FP4 GEMM.  Forward form: A = Q(act) [M, K], B = layer's R [N, K] with R_sf,
+// B2 = U [R2, N] (MN-major).  Transposed form (dX): B = R^T from R_codes_t with
+// R_sf_t, B2 = D [N_out, R2] (K-major).  Scales of both operands in the
+// MMA-ready layout.
 struct GemmArgs {
   int64_t M, N, K, R2;
   const uint8_t* a_codes;
-  const uint8_t* a_scales;
+  const uint8_t* a_sf;          // MMA-ready scales of A (rows M, cols K)
   const uint8_t* b_codes;       // R_codes [N, K/2] or R_codes_t [N, K/2] (transposed form)
-  const uint8_t* r_scales;      // the layer's R_scales
+  const uint8_t* b_sf;          // R_sf or R_sf_t (rows N, cols K)
   bool transposed;
   const void* A2;               // bf16 [M, R2]
   const void* B2;               // U [R2, N] (forward) or D [N, R2] (transposed)
@@ -321,59 +313,30 @@ struct GemmArgs {
   const void* h;                // GELU-backward epilogue: saved hidden [M, N]
   void* out2;                   // GELU-backward epilogue: bf16(GELU(h)) [M, N]
 };
-int run_gemm(const GemmArgs& a, int* status, cudaStream_t s) {
-  CUtensorMap tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, tmO2;
-  // compact scale tiles by TMA when every scale row is a whole number of 16-byte units
-  const bool sf_tma = a.K % 256 == 0 && a.N % 256 == 0 && al16(a.a_scales) && al16(a.r_scales);
+int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
+  CUtensorMap tmA, tmB, tmA2, tmB2;
   if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, ft::kGemmBN) ||
       !map_bf16(&tmA2, a.A2, a.R2, a.M, 128))
     return FT_ERR_CUDA;
   if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, ft::kGemmBN) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
     return FT_ERR_CUDA;
-  if (sf_tma) {
-    // one box = the scales of ft::kGemmSfGroups K-groups (several K-blocks) of the tile's rows
-    const uint32_t G = ft::kGemmSfGroups;
-    if (!map_scales(&tmSA, a.a_scales, a.K / 16, a.M / 16, G, 8)) return FT_ERR_CUDA;
-    // R_scales is [N_R/16, K_R/16]; transposed form: N_R = this GEMM's K, K_R = its N
-    if (a.transposed ? !map_scales(&tmSB, a.r_scales, a.N / 16, a.K / 16, ft::kGemmBN / 16, G)
-                     : !map_scales(&tmSB, a.r_scales, a.K / 16, a.N / 16, G, ft::kGemmBN / 16))
-      return FT_ERR_CUDA;
-  } else {
-    tmSA = tmSB = tmA;  // unused
-  }
-  if (!map_out(&tmO, a.out, a.N, a.M, a.out_bf16)) return FT_ERR_CUDA;
-  if (a.out2) {
-    if (!map_out(&tmO2, a.out2, a.N, a.M, true)) return FT_ERR_CUDA;
-  } else {
-    tmO2 = tmO;  // unused
-  }
   GemmParams gp{};
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
   gp.K = static_cast<int>(a.K);
   gp.R2 = static_cast<int>(a.R2);
   gp.b2_mn_major = a.transposed ? 0 : 1;
-  gp.sf_tma = sf_tma ? 1 : 0;
-  gp.sfb_transposed = a.transposed ? 1 : 0;
-  gp.sfa = a.a_scales;
-  gp.sfa_rs = a.K / 16;
-  gp.sfa_gs = 1;
-  gp.sfb = a.r_scales;
-  if (a.transposed) {  // scale of (row n of R^T, group g) = R_scales[g, n/16]
-    gp.sfb_rs = 1;
-    gp.sfb_gs = a.N / 16;
-  } else {
-    gp.sfb_rs = a.K / 16;
-    gp.sfb_gs = 1;
-  }
+  gp.sfa = a.a_sf;
+  gp.sfb = a.b_sf;
   gp.bias = a.bias;
   gp.out = a.out;
   gp.ldo = a.N;
   gp.out_bf16 = a.out_bf16 ? 1 : 0;
   gp.epi_gelu_bwd = a.h ? 1 : 0;
   gp.h = a.h;
+  gp.out2 = a.out2;
   gp.status = status;
-  return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, tmSA, tmSB, tmO, tmO2, gp, s));
+  return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
 }
 
 // dA = T_A^T V_A[:, r_s:] ([K, r]) and dB = (L[:, r_s:]^T G) ([r, N]) of one layer, one launch
@@ -464,6 +427,24 @@ int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, u
                                              static_cast<cudaStream_t>(stream)));
 }
 
+size_t fourtune_mma_scales_size(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || rows > (1 << 30) || cols > (1 << 30)) return 0;
+  return ft::sf_mma_bytes(rows, cols);
+}
+
+int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int transposed, uint8_t* out,
+                        void* stream) {
+  if (!scales || !out || (transposed != 0 && transposed != 1)) return FT_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return FT_ERR_SHAPE;
+  if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(out)) return FT_ERR_ALIGN;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  return cuda_err(ft::launch_sf_mma(scales, static_cast<int>(rows), static_cast<int>(cols), transposed, out,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- linear
 size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M) {
   if (check_layer(layer, false) || M <= 0 || M % 16) return 0;
@@ -522,8 +503,9 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   uint8_t* qc = base + w.qx.codes;
   uint8_t* qs = base + w.qx.scales;
+  uint8_t* qf = base + w.qx.sf;
   // X pass: Q(X) and L = bf16(X D)
-  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, L_saved, status, di.num_sms, s));
+  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, qf, L_saved, status, di.num_sms, s));
   // 4-bit GEMM + L U + bias
   GemmArgs g{};
   g.M = M;
@@ -531,16 +513,16 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   g.K = K;
   g.R2 = R;
   g.a_codes = qc;
-  g.a_scales = qs;
+  g.a_sf = qf;
   g.b_codes = layer->R_codes;
-  g.r_scales = layer->R_scales;
+  g.b_sf = layer->R_sf;
   g.transposed = false;
   g.A2 = L_saved;
   g.B2 = layer->U;
   g.bias = layer->bias;
   g.out = Y;
   g.out_bf16 = y_dtype == FT_DTYPE_BF16;
-  FT_TRY(1, run_gemm(g, status, s));
+  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   return FT_OK;
 }
 
@@ -576,9 +558,10 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   uint8_t* gc = base + w.qg.codes;
   uint8_t* gs = base + w.qg.scales;
+  uint8_t* gf = base + w.qg.sf;
   void* P = base + w.P;
   // G pass: Q(G) and P = bf16(G U^T), U [R, N] read K-major
-  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, P, status, di.num_sms, s));
+  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P, status, di.num_sms, s));
   // dX = deq(Q(G)) deq(Q(R)) + P D^T
   GemmArgs g{};
   g.M = M;
@@ -586,15 +569,15 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   g.K = N;
   g.R2 = R;
   g.a_codes = gc;
-  g.a_scales = gs;
+  g.a_sf = gf;
   g.b_codes = layer->R_codes_t;
-  g.r_scales = layer->R_scales;
+  g.b_sf = layer->R_sf_t;
   g.transposed = true;
   g.A2 = P;
   g.B2 = layer->D;
   g.out = dX;
   g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(1, run_gemm(g, status, s));
+  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   // dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G
   FT_TRY(2, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, s));
   return FT_OK;
@@ -657,25 +640,25 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   // FC1: X pass, then 4-bit GEMM + L1 U1 + b1 -> h (bf16, saved)
   FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
-                        L1_saved, status, di.num_sms, s));
+                        base + w.qx.sf, L1_saved, status, di.num_sms, s));
   GemmArgs g{};
   g.M = M;
   g.N = H;
   g.K = K1;
   g.R2 = R1;
   g.a_codes = base + w.qx.codes;
-  g.a_scales = base + w.qx.scales;
+  g.a_sf = base + w.qx.sf;
   g.b_codes = fc1->R_codes;
-  g.r_scales = fc1->R_scales;
+  g.b_sf = fc1->R_sf;
   g.A2 = L1_saved;
   g.B2 = fc1->U;
   g.bias = fc1->bias;
   g.out = h_saved;
   g.out_bf16 = true;
-  FT_TRY(1, run_gemm(g, status, s));
+  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   // GELU pass over h: Q(a) of a = GELU(h) and L2 = bf16(bf16(a) D2)
   FT_TRY(2, run_rowpass(h_saved, M, H, fc2->D, R2, true, true, dbg_a, base + w.qa.codes, base + w.qa.scales,
-                        L2_saved, status, di.num_sms, s));
+                        base + w.qa.sf, L2_saved, status, di.num_sms, s));
   // FC2: 4-bit GEMM + L2 U2 + b2 -> Y
   GemmArgs g2{};
   g2.M = M;
@@ -683,15 +666,15 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   g2.K = H;
   g2.R2 = R2;
   g2.a_codes = base + w.qa.codes;
-  g2.a_scales = base + w.qa.scales;
+  g2.a_sf = base + w.qa.sf;
   g2.b_codes = fc2->R_codes;
-  g2.r_scales = fc2->R_scales;
+  g2.b_sf = fc2->R_sf;
   g2.A2 = L2_saved;
   g2.B2 = fc2->U;
   g2.bias = fc2->bias;
   g2.out = Y;
   g2.out_bf16 = y_dtype == FT_DTYPE_BF16;
-  FT_TRY(3, run_gemm(g2, status, s));
+  FT_TRY(3, run_gemm(g2, status, di.num_sms, s));
   return FT_OK;
 }
 
@@ -724,17 +707,17 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   void* abf = base + w.abf;
   void* P1 = base + w.P1;
   // FC2 backward: G pass (Q(G), P2), dX GEMM with the GELU-backward epilogue
-  FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales, P2,
-                        status, di.num_sms, s));
+  FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales,
+                        base + w.qg.sf, P2, status, di.num_sms, s));
   GemmArgs g{};
   g.M = M;
   g.N = H;
   g.K = N2;
   g.R2 = R2;
   g.a_codes = base + w.qg.codes;
-  g.a_scales = base + w.qg.scales;
+  g.a_sf = base + w.qg.sf;
   g.b_codes = fc2->R_codes_t;
-  g.r_scales = fc2->R_scales;
+  g.b_sf = fc2->R_sf_t;
   g.transposed = true;
   g.A2 = P2;
   g.B2 = fc2->D;
@@ -742,27 +725,27 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   g.out_bf16 = true;
   g.h = h_saved;
   g.out2 = abf;
-  FT_TRY(1, run_gemm(g, status, s));
+  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   // FC2 adapter gradients on bf16(GELU(h)) and G
   FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, base, status, s));
   // FC1 backward on d_h: G pass, dX GEMM, adapter gradients
-  FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales, P1,
-                        status, di.num_sms, s));
+  FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales,
+                        base + w.qdh.sf, P1, status, di.num_sms, s));
   GemmArgs g1{};
   g1.M = M;
   g1.N = K1;
   g1.K = H;
   g1.R2 = R1;
   g1.a_codes = base + w.qdh.codes;
-  g1.a_scales = base + w.qdh.scales;
+  g1.a_sf = base + w.qdh.sf;
   g1.b_codes = fc1->R_codes_t;
-  g1.r_scales = fc1->R_scales;
+  g1.b_sf = fc1->R_sf_t;
   g1.transposed = true;
   g1.A2 = P1;
   g1.B2 = fc1->D;
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(4, run_gemm(g1, status, s));
+  FT_TRY(4, run_gemm(g1, status, di.num_sms, s));
   FT_TRY(5, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status, s));
   return FT_OK;
 }

@@ -19,6 +19,7 @@ struct RowpassParams {
   float* dbg_a;                          // gelu_input: optional fp32 copy of a [M, K] (null = none)
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
+  uint8_t* sf_mma;                       // the same scales in the MMA-ready layout (null = not written)
   void* L;                               // bf16 [M, R]
   float* part;                           // fp32 [nsplit, M, R] when nsplit > 1 and no cluster
   int* counters;                         // [ceil(M/128)], zero on entry, left zero (no cluster)
@@ -27,28 +28,37 @@ struct RowpassParams {
 // largest split count the cluster reduction handles (portable cluster size)
 constexpr int kRowpassMaxClusterSplit = 8;
 
-// out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1.
-// Scales: with sf_tma the compact [rows/16, K/16] tiles come by TMA (B's read
-// transposed when sfb_transposed: B's scale(row, g) = array[g, row/16]);
-// otherwise scale(row, g) = sf[(row/16)*rs + g*gs] by plain loads.
+// MMA-ready scale layout of a block16 operand with `rows` rows (along M or N)
+// and `cols` columns along K: for each 128-row chunk c and each 64-column
+// k-step t, one 512-byte block at byte ((c * KS) + t) * 512, KS = ceil(cols/64).
+// Inside a block, the scale of row r (r % 128 = 32 q + l) and of the step's
+// 16-column group j (0..3) sits at byte 16 l + 4 q + j -- the order in which
+// tcgen05.cp 32x128b.warpx4 moves 512 bytes into the TMEM columns that the
+// block-scaled MMA reads.  Rows past `rows` and groups past cols/16 hold 0.
+__host__ __device__ constexpr size_t sf_mma_bytes(long long rows, long long cols) {
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((cols + 63) / 64) * 512u;
+}
+__host__ __device__ constexpr long long sf_mma_offset(long long r, long long g, long long ks) {
+  return ((r / 128) * ks + g / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (g % 4);
+}
+
+// out = deq(A) deq(B)^T (+ A2 * B2^T) (+ bias); A [M, K], B [N, K] packed E2M1,
+// their scales in the MMA-ready layout (sfa: rows = M, sfb: rows = N, cols = K).
 // A2 [M, R2] bf16; B2 is [N, R2] (K-major) or U [R2, N] (b2_mn_major).
 struct GemmParams {
   int M, N, K, R2;
   int b2_mn_major;
-  int sf_tma;
-  int sfb_transposed;
   const uint8_t* sfa;
-  long long sfa_rs, sfa_gs;
   const uint8_t* sfb;
-  long long sfb_rs, sfb_gs;
   const void* bias;                      // bf16 [N] or null
   void* out;
   long long ldo;
   int out_bf16;
   // GELU-backward epilogue: out = bf16(acc * GELU'(h)), out2 = bf16(GELU(h)),
-  // h bf16 [M, N] with row stride N (both outputs bf16, out2 through tmOut2)
+  // h bf16 [M, N] with row stride N (both outputs bf16, row stride ldo)
   int epi_gelu_bwd;
   const void* h;
+  void* out2;
   int* status;
 };
 
@@ -71,11 +81,14 @@ cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uin
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream);
 int rowpass_ctas_per_sm(int R, int w_mn_major);
-// tmOut: the output [M, N] (fp32 or bf16) with 128-byte x 32-row boxes, 128-byte swizzle
+// persistent: min(tiles, num_sms) CTAs
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
-                            const CUtensorMap& tmB2, const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
-                            const CUtensorMap& tmOut, const CUtensorMap& tmOut2, const GemmParams& p,
-                            cudaStream_t stream);
+                            const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream);
+// compact block16 scales -> MMA-ready layout of the operand [rows, cols]; with
+// `transposed`, the operand is the transpose of the quantized matrix, whose
+// compact scales are [cols/16, rows/16]
+cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
+                          cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
                           const CUtensorMap& tmT1, const CUtensorMap& tmV1, const TgradParams& p1,
                           cudaStream_t stream);
@@ -88,7 +101,5 @@ cudaError_t rowpass_static_scratch(void** out);
 // tile sizes the host needs for tensor-map boxes and workspace sizing
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
-// K-groups (of 16) per compact-scale TMA box: the scales of four 256-wide K-blocks
-constexpr int kGemmSfGroups = 64;
 
 }  // namespace ft

@@ -131,4 +131,37 @@ cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uin
   return cudaGetLastError();
 }
 
+// Compact block16 scales -> MMA-ready layout (kernels.h), one thread per byte.
+// Non-transposed: operand [rows, cols] = the quantized matrix, scale(rb, g) =
+// scales[rb * (cols/16) + g].  Transposed: operand = the quantized matrix's
+// transpose (FourTune §3.2: same scale bytes), scale(rb, g) = scales[g * (rows/16) + rb].
+__global__ void sf_mma_kernel(const uint8_t* __restrict__ scales, int rows, int cols, int transposed,
+                              uint8_t* __restrict__ out, long long n) {
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= n) return;
+  const int ks = (cols + 63) / 64;
+  const long long blk = i / 512;
+  const int b = static_cast<int>(i % 512);
+  const long long chunk = blk / ks;
+  const int t = static_cast<int>(blk % ks);
+  const long long r = chunk * 128 + ((b % 16) / 4) * 32 + b / 16;
+  const int g = 4 * t + (b % 4);
+  uint8_t v = 0;
+  if (r < rows && g < cols / 16) {
+    const long long rb = r / 16;
+    v = transposed ? scales[static_cast<long long>(g) * (rows / 16) + rb] : scales[rb * (cols / 16) + g];
+  }
+  out[i] = v;
+}
+
+cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
+                          cudaStream_t stream) {
+  const long long n = static_cast<long long>(sf_mma_bytes(rows, cols));
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  sf_mma_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, stream>>>(scales, rows, cols,
+                                                                                          transposed, out, n);
+  return cudaGetLastError();
+}
+
 }  // namespace ft

@@ -211,23 +211,32 @@ __global__ void __launch_bounds__(kRpThreads, 2)  // two CTAs per SM: registers 
         amax[j] = a;
       }
       const int cstart = (kt0 + i) * 64 + 32 * h;
-      if (block_row_ok && cstart < p.K) {
+      const bool inside = block_row_ok && cstart < p.K;
+      if (inside || p.sf_mma) {
+        // rows past M and columns past K were zero-filled by the TMA: their scale is 0
         uint32_t packed[4], sc[2];
         if (GELU)
           quantize_2blocks_div(v, amax, packed, sc);
         else
           quantize_2blocks(v, amax, packed, sc);
-        *reinterpret_cast<uint4*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
-            make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        if ((lane >> 1) == 0) {
-          const long long srow = (m0 / 16 + w8) * static_cast<long long>(kblocks);
-          p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
-          p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
-        }
-        if (GELU && p.dbg_a) {
-          float4* dst = reinterpret_cast<float4*>(p.dbg_a + static_cast<long long>(m0 + r) * p.K + cstart);
+        if (inside) {
+          *reinterpret_cast<uint4*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          if ((lane >> 1) == 0) {
+            const long long srow = (m0 / 16 + w8) * static_cast<long long>(kblocks);
+            p.scales[srow + cstart / 16] = static_cast<uint8_t>(sc[0]);
+            p.scales[srow + cstart / 16 + 1] = static_cast<uint8_t>(sc[1]);
+          }
+          if (GELU && p.dbg_a) {
+            float4* dst = reinterpret_cast<float4*>(p.dbg_a + static_cast<long long>(m0 + r) * p.K + cstart);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+            for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+        }
+        if (p.sf_mma) {
+          // MMA-ready copy: groups 2h, 2h+1 of k-step kt0+i for row r of chunk blockIdx.x
+          const size_t o = (static_cast<size_t>(blockIdx.x) * KT + (kt0 + i)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + 2 * h;
+          *reinterpret_cast<uint16_t*>(p.sf_mma + o) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
         }
       }
     }

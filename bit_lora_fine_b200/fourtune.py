@@ -26,7 +26,7 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed",
             "fourtune_quant_down_static", "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_fwd",
             "fourtune_mlp_bwd_workspace_size", "fourtune_mlp_bwd", "fourtune_mlp_fwd_ws_offsets",
-            "fourtune_mlp_bwd_ws_offsets")
+            "fourtune_mlp_bwd_ws_offsets", "fourtune_mma_scales_size", "fourtune_mma_scales")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
@@ -42,7 +42,8 @@ class FourtuneError(RuntimeError):
 class ft_linear_t(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int64), ("N", ctypes.c_int64), ("r_s", ctypes.c_int64), ("r", ctypes.c_int64),
                 ("R_codes", ctypes.c_void_p), ("R_scales", ctypes.c_void_p), ("R_codes_t", ctypes.c_void_p),
-                ("D", ctypes.c_void_p), ("U", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+                ("D", ctypes.c_void_p), ("U", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("R_sf", ctypes.c_void_p), ("R_sf_t", ctypes.c_void_p)]
 
 
 _lib = None
@@ -60,6 +61,9 @@ def load():
     P = ctypes.POINTER
     L.fourtune_quantize_block16.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
     L.fourtune_transpose_codes.argtypes = [vp, i64, i64, vp, vp]
+    L.fourtune_mma_scales_size.argtypes = [i64, i64]
+    L.fourtune_mma_scales_size.restype = sz
+    L.fourtune_mma_scales.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp]
     L.fourtune_linear_fwd_workspace_size.argtypes = [P(ft_linear_t), i64]
     L.fourtune_linear_fwd_workspace_size.restype = sz
     L.fourtune_linear_bwd_workspace_size.argtypes = [P(ft_linear_t), i64]
@@ -87,6 +91,7 @@ def load():
     L.fourtune_mlp_bwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz), P(sz), P(sz)]
     for f in EXPORTED:
         if f not in ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size",
+                     "fourtune_mma_scales_size",
                      "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
                      "fourtune_error_string"):
             getattr(L, f).restype = ctypes.c_int
@@ -126,6 +131,20 @@ def quantize_block16(x, transposed=False):
     return codes, scales, codes_t
 
 
+def mma_scales(scales, rows, cols, transposed=False):
+    """Block16 scales of an operand [rows, cols] rearranged for the block-scaled MMA (u8 tensor).
+    transposed: the operand is the transpose of the matrix whose scales are given
+    ([cols/16, rows/16]); otherwise scales is [rows/16, cols/16]."""
+    _need(scales, torch.uint8, "scales")
+    n = load().fourtune_mma_scales_size(rows, cols)
+    if n == 0:
+        raise FourtuneError(-2, "fourtune_mma_scales_size")
+    out = torch.empty(n, dtype=torch.uint8, device=scales.device)
+    _check(load().fourtune_mma_scales(_ptr(scales), rows, cols, int(transposed), _ptr(out), _stream()),
+           "fourtune_mma_scales")
+    return out
+
+
 def transpose_codes(codes, rows, cols):
     out = torch.empty((cols, rows // 2), dtype=torch.uint8, device=codes.device)
     _check(load().fourtune_transpose_codes(_ptr(codes), rows, cols, _ptr(out), _stream()),
@@ -135,7 +154,8 @@ def transpose_codes(codes, rows, cols):
 
 class Linear:
     """Device tensors of one triple-branch layer: frozen R codes/scales/codes_t and bias,
-    D = [S_dn | A] [K, r_s + r] and U = [S_up ; B] [r_s + r, N] (bf16).  The LoRA factors
+    D = [S_dn | A] [K, r_s + r] and U = [S_up ; B] [r_s + r, N] (bf16), and R's scales
+    in the MMA-ready layouts of R and R^T (prepared here once).  The LoRA factors
     are views: A = D[:, r_s:], B = U[r_s:, :].  Holds references so pointers stay valid."""
 
     def __init__(self, R_codes, R_scales, R_codes_t, D, U, r_s, bias=None):
@@ -147,9 +167,12 @@ class Linear:
             _need(t, torch.uint8, n)
         for t, n in ((D, "D"), (U, "U"), (bias, "bias")):
             _need(t, torch.bfloat16, n)
-        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_codes_t=R_codes_t, D=D, U=U, bias=bias)
+        R_sf = mma_scales(R_scales, self.N, self.K)
+        R_sf_t = mma_scales(R_scales, self.K, self.N, transposed=True)
+        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_codes_t=R_codes_t, D=D, U=U, bias=bias,
+                      R_sf=R_sf, R_sf_t=R_sf_t)
         self.c = ft_linear_t(self.K, self.N, self.r_s, self.r, *[
-            _ptr(self.t[k]) for k in ("R_codes", "R_scales", "R_codes_t", "D", "U", "bias")])
+            _ptr(self.t[k]) for k in ("R_codes", "R_scales", "R_codes_t", "D", "U", "bias", "R_sf", "R_sf_t")])
 
     @classmethod
     def from_weights(cls, R, S_dn, S_up, A, B, bias=None):

@@ -70,6 +70,10 @@ enum { FT_DTYPE_F32 = 0, FT_DTYPE_BF16 = 1 };
  *   R_codes_t [K, N/2]  the same codes nibble-transposed (codes of R^T); the
  *                       scales of R^T are R_scales read transposed.  Required by
  *                       the backward (fourtune_quantize_block16 writes it).
+ *   R_sf      R_scales rearranged for the tensor cores: fourtune_mma_scales of
+ *             R_scales with rows = N, cols = K, transposed = 0
+ *   R_sf_t    the same for R^T: rows = K, cols = N, transposed = 1.  Required
+ *             by the backward.  Both are frozen like R and prepared once.
  *   D [K, r_s + r] = [S_dn | A]   down-projections, bf16 row-major: the frozen
  *                       stabilizer's S_dn in columns 0..r_s-1, the LoRA A after it
  *   U [r_s + r, N] = [S_up ; B]   up-projections, bf16 row-major: S_up rows first,
@@ -87,6 +91,8 @@ typedef struct {
   const ft_bf16* D;
   const ft_bf16* U;
   const ft_bf16* bias;
+  const uint8_t* R_sf;
+  const uint8_t* R_sf_t;
 } ft_linear_t;
 
 /* Block16 quantization of a bf16 matrix x [rows, cols] with row stride `ld`
@@ -102,6 +108,21 @@ FT_API int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t col
 /* Nibble transpose of block16 codes: codes [rows, cols/2] -> codes_t [cols, rows/2]
  * (§3.2: the transposed operand keeps its codes and scales). */
 FT_API int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, uint8_t* codes_t, void* stream);
+
+/* The block16 scales of an operand rearranged in the order the block-scaled
+ * tensor-core MMA consumes them (§3.1: the 4-bit products run on 4-bit tensor
+ * cores).  The operand is a [rows, cols] matrix with cols along the reduction
+ * dimension; its scales are `scales` [rows/16, cols/16], or, with transposed =
+ * 1, the operand is the transpose of the quantized matrix and `scales` is that
+ * matrix's [cols/16, rows/16] array (§3.2: the transposed operand keeps its
+ * scales).  Output: fourtune_mma_scales_size(rows, cols) bytes, 16-byte
+ * aligned: for each 128-row chunk c and 64-column step t a 512-byte block at
+ * ((c * ceil(cols/64)) + t) * 512 holding the scale of row r = 128 c + 32 q + l
+ * and column group 4 t + j at byte 16 l + 4 q + j (0 past the matrix).
+ * rows, cols multiples of 16. */
+FT_API size_t fourtune_mma_scales_size(int64_t rows, int64_t cols);
+FT_API int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int transposed, uint8_t* out,
+                               void* stream);
 
 /* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
 FT_API size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M);

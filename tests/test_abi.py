@@ -43,7 +43,7 @@ def test_error_strings(lib):
 
 def _layer(K=64, N=64, r_s=16, r=16, ptr=256):
     p = ctypes.c_void_p(ptr)
-    return fourtune.ft_linear_t(K, N, r_s, r, p, p, p, p, p, None)
+    return fourtune.ft_linear_t(K, N, r_s, r, p, p, p, p, p, None, p, p)
 
 
 def test_argument_checks_without_device(lib):
@@ -74,3 +74,18 @@ def test_argument_checks_without_device(lib):
     L.R_codes_t = None
     assert lib.fourtune_linear_bwd(ctypes.byref(L), p, p, p, 16, p, 0, p, p, 0, p, 1 << 20, s) == -1
     assert lib.fourtune_linear_bwd_workspace_size(ctypes.byref(L), 16) == 0
+    # ... and R's scales in the transposed MMA-ready layout; the forward needs R_sf
+    L = _layer()
+    L.R_sf_t = None
+    assert lib.fourtune_linear_bwd(ctypes.byref(L), p, p, p, 16, p, 0, p, p, 0, p, 1 << 20, s) == -1
+    L = _layer()
+    L.R_sf = None
+    assert lib.fourtune_linear_fwd(ctypes.byref(L), p, 16, p, 0, p, p, 1 << 20, s) == -1
+    # MMA-ready scale layout: size formula, argument checks
+    assert lib.fourtune_mma_scales_size(128, 64) == 512
+    assert lib.fourtune_mma_scales_size(144, 96) == 2 * 2 * 512
+    assert lib.fourtune_mma_scales_size(20, 64) == 0
+    assert lib.fourtune_mma_scales(None, 16, 16, 0, p, s) == -1
+    assert lib.fourtune_mma_scales(p, 16, 16, 2, p, s) == -1
+    assert lib.fourtune_mma_scales(p, 16, 24, 0, p, s) == -2
+    assert lib.fourtune_mma_scales(p, 16, 16, 0, ctypes.c_void_p(264), s) == -3

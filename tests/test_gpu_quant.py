@@ -83,3 +83,32 @@ def test_row_stride(cuda_lib):
     rc_, rs_ = block16.quantize(np.ascontiguousarray(big[:, 16:80]))
     np.testing.assert_array_equal(s.cpu().numpy(), rs_)
     np.testing.assert_array_equal(c.cpu().numpy(), rc_)
+
+
+def _mma_layout(scales, rows, cols, transposed):
+    """The MMA-ready scale order written out from its definition (the 512-byte
+    block of 128-row chunk c and 64-column step t holds the scale of row
+    128 c + 32 q + l and group 4 t + j at byte 16 l + 4 q + j; zero elsewhere)."""
+    ks = (cols + 63) // 64
+    out = np.zeros(((rows + 127) // 128) * ks * 512, np.uint8)
+    r = np.arange(rows)[:, None]
+    g = np.arange(cols // 16)[None, :]
+    off = ((r // 128) * ks + g // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + g % 4
+    src = scales.T if transposed else scales
+    out[off.ravel()] = src[np.arange(rows) // 16][:, np.arange(cols // 16)].ravel()
+    return out
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 32), (144, 96), (400, 320), (3072, 3072)])
+def test_mma_scale_layout(cuda_lib, rows, cols):
+    """fourtune_mma_scales on the oracle's scales of R [rows, cols] (forward operand)
+    and of R^T (backward operand, transposed read of the same bytes)."""
+    import torch
+    rng = np.random.default_rng(rows + cols)
+    R = synth.to_bf16((rng.standard_normal((rows, cols)) * 0.02).astype(np.float32))
+    _, rs = block16.quantize(R)
+    sd = torch.from_numpy(rs).to("cuda")
+    got = cuda_lib.mma_scales(sd, rows, cols).cpu().numpy()
+    np.testing.assert_array_equal(got, _mma_layout(rs, rows, cols, False))
+    got_t = cuda_lib.mma_scales(sd, cols, rows, transposed=True).cpu().numpy()
+    np.testing.assert_array_equal(got_t, _mma_layout(rs, cols, rows, True))
