@@ -112,15 +112,21 @@ inline int64_t rank_all(const ft_linear_t* L) { return L->r_s + L->r; }
 
 // ---------------------------------------------------------------- split choice
 struct RowSplit {
-  int nsplit, kt_per_split;
+  int nsplit, kt_per_split, stages;
 };
-// enough CTAs for every SM (two per SM when they fit), never more splits than tiles
+// One CTA per SM with the deepest ring: enough CTAs for every SM (split-K when
+// the 128-row tiles alone are too few), never more splits than K tiles.
+constexpr int kRowMaxSplit = 16;
 RowSplit row_split(int64_t M, int64_t K, int64_t R, int mn, int num_sms, int max_split) {
   const int MT = cdiv(M, 128), KT = cdiv(K, 64);
-  const int target = num_sms * ft::rowpass_ctas_per_sm(static_cast<int>(R), mn);
-  const int ns = MT >= target ? 1 : std::max(1, std::min({KT, target / MT, max_split}));
+  const int ns = MT >= num_sms ? 1 : std::max(1, std::min({KT, num_sms / MT, max_split}));
   const int per = cdiv(KT, ns);
-  return {cdiv(KT, per), per};
+  return {cdiv(KT, per), per, ft::rowpass_stages(static_cast<int>(R), mn)};
+}
+// fp32 split partials of one row pass (0 without a split)
+size_t rp_part_bytes(int64_t M, int64_t K, int64_t R, int mn, int num_sms) {
+  const RowSplit rs = row_split(M, K, R, mn, num_sms, kRowMaxSplit);
+  return rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * static_cast<size_t>(M) * static_cast<size_t>(R) * 4 : 0;
 }
 struct MSplit {
   int nsplit, mt_per_split;
@@ -170,23 +176,26 @@ size_t grad_partial_bytes(const GradPair& g, const ft_linear_t* L) {
 
 // Each layout starts with a header of `header` bytes (status word, split
 // counters) that every call clears first.
-// Linear forward: header (status) | Q(X)
+// Linear forward: header (status, row-pass split counters) | Q(X) | row-pass partials
 struct FwdWs {
-  size_t header, total;
+  size_t header, rp_cnt, rp_part, total;
   Q16 qx;
 };
-FwdWs fwd_layout(const ft_linear_t* L, int64_t M) {
+FwdWs fwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   FwdWs w{};
   Carver c;
-  c.take(w.header = 256);
+  w.rp_cnt = 16;
+  c.take(w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qx.carve(c, M, L->K);
+  w.rp_part = c.take(rp_part_bytes(M, L->K, rank_all(L), 1, num_sms));
   w.total = c.o;
   return w;
 }
 
-// Linear backward: header (status, dA/dB counters) | Q(G) | P | dA/dB partials
+// Linear backward: header (status, dA/dB and row-pass counters) | Q(G) | P |
+// dA/dB partials | row-pass partials
 struct BwdWs {
-  size_t header, P, total;
+  size_t header, P, rp_cnt, rp_part, total;
   Q16 qg;
   GradPair g;
 };
@@ -196,34 +205,41 @@ BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   Carver c;
   w.g.cntA = 16;
   w.g.cntB = w.g.cntA + 4 * static_cast<size_t>(cdiv(L->K, 128));
-  c.take(w.header = up256(16 + 4 * grad_counter_words(L)));
+  w.rp_cnt = 16 + 4 * grad_counter_words(L);
+  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qg.carve(c, M, L->N);
   w.P = c.take(static_cast<size_t>(M * rank_all(L) * 2));
   w.g.partA = c.take(grad_partial_bytes(w.g, L));
   w.g.partB = w.g.partA + (w.g.sA.nsplit > 1 ? static_cast<size_t>(w.g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0);
+  w.rp_part = c.take(rp_part_bytes(M, L->N, rank_all(L), 0, num_sms));
   w.total = c.o;
   return w;
 }
 
-// MLP forward: header (status) | Q(X) | Q(a)
+// MLP forward: header (status, row-pass counters) | Q(X) | Q(a) | row-pass
+// partials (shared by the two row passes, which run one after the other)
 struct MlpFwdWs {
-  size_t header, total;
+  size_t header, rp_cnt, rp_part, total;
   Q16 qx, qa;
 };
-MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, int64_t M) {
+MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, int num_sms) {
   MlpFwdWs w{};
   Carver c;
-  c.take(w.header = 256);
+  w.rp_cnt = 16;
+  c.take(w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qx.carve(c, M, fc1->K);
   w.qa.carve(c, M, fc1->N);
+  w.rp_part = c.take(std::max(rp_part_bytes(M, fc1->K, rank_all(fc1), 1, num_sms),
+                              rp_part_bytes(M, fc1->N, rank_all(fc2), 1, num_sms)));
   w.total = c.o;
   return w;
 }
 
-// MLP backward: header (status, counters of both layers' dA/dB) | Q(G) | P2 |
-// d_h | bf16(GELU(h)) | Q(d_h) | P1 | partials (shared by the two dA/dB launches)
+// MLP backward: header (status, counters of both layers' dA/dB, row-pass
+// counters) | Q(G) | P2 | d_h | bf16(GELU(h)) | Q(d_h) | P1 | dA/dB partials
+// (shared by the two dA/dB launches) | row-pass partials (shared likewise)
 struct MlpBwdWs {
-  size_t header, P2, dh, abf, P1, total;
+  size_t header, P2, dh, abf, P1, rp_cnt, rp_part, total;
   Q16 qg, qdh;
   GradPair g2, g1;
 };
@@ -237,7 +253,8 @@ MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
   w.g2.cntB = w.g2.cntA + 4 * static_cast<size_t>(cdiv(fc2->K, 128));
   w.g1.cntA = w.g2.cntB + 4 * static_cast<size_t>(cdiv(fc2->N, 128));
   w.g1.cntB = w.g1.cntA + 4 * static_cast<size_t>(cdiv(fc1->K, 128));
-  c.take(w.header = up256(16 + 4 * (grad_counter_words(fc2) + grad_counter_words(fc1))));
+  w.rp_cnt = 16 + 4 * (grad_counter_words(fc2) + grad_counter_words(fc1));
+  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qg.carve(c, M, fc2->N);
   w.P2 = c.take(static_cast<size_t>(M * rank_all(fc2) * 2));
   w.dh = c.take(static_cast<size_t>(M * H * 2));
@@ -248,6 +265,8 @@ MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
   w.g2.partA = w.g1.partA = part;
   w.g2.partB = part + (w.g2.sA.nsplit > 1 ? static_cast<size_t>(w.g2.sA.nsplit) * cdiv(fc2->K, 128) * 128 * 64 * 4 : 0);
   w.g1.partB = part + (w.g1.sA.nsplit > 1 ? static_cast<size_t>(w.g1.sA.nsplit) * cdiv(fc1->K, 128) * 128 * 64 * 4 : 0);
+  w.rp_part = c.take(std::max(rp_part_bytes(M, fc2->N, rank_all(fc2), 0, num_sms),
+                              rp_part_bytes(M, H, rank_all(fc1), 0, num_sms)));
   w.total = c.o;
   return w;
 }
@@ -270,12 +289,12 @@ struct Events {
 // with W = D [K, R] (w_mn) or W^T [R, K]; gelu: the input is h and the pass
 // quantizes GELU(h).  Split reduction inside a cluster: needs only the status word.
 int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
-                float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, int* status, int num_sms,
-                cudaStream_t s) {
+                float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
+                int* status, int num_sms, cudaStream_t s) {
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
   if (w_mn ? !map_bf16(&tmW, W, R, K, 64) : !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
-  const RowSplit rs = row_split(M, K, R, w_mn ? 1 : 0, num_sms, ft::kRowpassMaxClusterSplit);
+  const RowSplit rs = row_split(M, K, R, w_mn ? 1 : 0, num_sms, kRowMaxSplit);
   RowpassParams rp{};
   rp.M = static_cast<int>(M);
   rp.K = static_cast<int>(K);
@@ -283,13 +302,15 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.w_mn_major = w_mn ? 1 : 0;
   rp.kt_per_split = rs.kt_per_split;
   rp.nsplit = rs.nsplit;
-  rp.cluster_reduce = rs.nsplit > 1;
+  rp.stages = rs.stages;
   rp.gelu_input = gelu ? 1 : 0;
   rp.dbg_a = dbg_a;
   rp.codes = codes;
   rp.scales = scales;
   rp.sf_mma = sf_mma;
   rp.L = L;
+  rp.part = part;
+  rp.counters = counters;
   rp.status = status;
   return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
@@ -448,7 +469,7 @@ int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int t
 // ---------------------------------------------------------------- linear
 size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M) {
   if (check_layer(layer, false) || M <= 0 || M % 16) return 0;
-  return fwd_layout(layer, M).total;
+  return fwd_layout(layer, M, num_sms_or_default()).total;
 }
 
 size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M) {
@@ -459,7 +480,7 @@ size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M) {
 int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off) {
   int st = check_layer(layer, false);
   if (st) return st;
-  const FwdWs w = fwd_layout(layer, M);
+  const FwdWs w = fwd_layout(layer, M, num_sms_or_default());
   if (codes_off) *codes_off = w.qx.codes;
   if (scales_off) *scales_off = w.qx.scales;
   return FT_OK;
@@ -494,7 +515,7 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   if (!al16(X) || !al16(Y) || !al16(L_saved) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return FT_ERR_ALIGN;
   DevInfo di;
   if ((st = device_info(&di))) return st;
-  const FwdWs w = fwd_layout(layer, M);
+  const FwdWs w = fwd_layout(layer, M, di.num_sms);
   if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -505,7 +526,9 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   uint8_t* qs = base + w.qx.scales;
   uint8_t* qf = base + w.qx.sf;
   // X pass: Q(X) and L = bf16(X D)
-  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, qf, L_saved, status, di.num_sms, s));
+  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, qf, L_saved,
+                        reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                        di.num_sms, s));
   // 4-bit GEMM + L U + bias
   GemmArgs g{};
   g.M = M;
@@ -561,7 +584,9 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   uint8_t* gf = base + w.qg.sf;
   void* P = base + w.P;
   // G pass: Q(G) and P = bf16(G U^T), U [R, N] read K-major
-  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P, status, di.num_sms, s));
+  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P,
+                        reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                        di.num_sms, s));
   // dX = deq(Q(G)) deq(Q(R)) + P D^T
   GemmArgs g{};
   g.M = M;
@@ -586,7 +611,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
 // ---------------------------------------------------------------- MLP
 size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
   if (check_mlp(fc1, fc2, false) || M <= 0 || M % 16) return 0;
-  return mlp_fwd_layout(fc1, M).total;
+  return mlp_fwd_layout(fc1, fc2, M, num_sms_or_default()).total;
 }
 
 size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
@@ -598,7 +623,7 @@ int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, 
                                 size_t* qa_scales) {
   int st = check_mlp(fc1, fc2, false);
   if (st) return st;
-  const MlpFwdWs w = mlp_fwd_layout(fc1, M);
+  const MlpFwdWs w = mlp_fwd_layout(fc1, fc2, M, num_sms_or_default());
   if (qa_codes) *qa_codes = w.qa.codes;
   if (qa_scales) *qa_scales = w.qa.scales;
   return FT_OK;
@@ -631,7 +656,7 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
     return FT_ERR_ALIGN;
   DevInfo di;
   if ((st = device_info(&di))) return st;
-  const MlpFwdWs w = mlp_fwd_layout(fc1, M);
+  const MlpFwdWs w = mlp_fwd_layout(fc1, fc2, M, di.num_sms);
   if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -640,7 +665,8 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   // FC1: X pass, then 4-bit GEMM + L1 U1 + b1 -> h (bf16, saved)
   FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
-                        base + w.qx.sf, L1_saved, status, di.num_sms, s));
+                        base + w.qx.sf, L1_saved, reinterpret_cast<float*>(base + w.rp_part),
+                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   GemmArgs g{};
   g.M = M;
   g.N = H;
@@ -658,7 +684,8 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   // GELU pass over h: Q(a) of a = GELU(h) and L2 = bf16(bf16(a) D2)
   FT_TRY(2, run_rowpass(h_saved, M, H, fc2->D, R2, true, true, dbg_a, base + w.qa.codes, base + w.qa.scales,
-                        base + w.qa.sf, L2_saved, status, di.num_sms, s));
+                        base + w.qa.sf, L2_saved, reinterpret_cast<float*>(base + w.rp_part),
+                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   // FC2: 4-bit GEMM + L2 U2 + b2 -> Y
   GemmArgs g2{};
   g2.M = M;
@@ -708,7 +735,8 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   void* P1 = base + w.P1;
   // FC2 backward: G pass (Q(G), P2), dX GEMM with the GELU-backward epilogue
   FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales,
-                        base + w.qg.sf, P2, status, di.num_sms, s));
+                        base + w.qg.sf, P2, reinterpret_cast<float*>(base + w.rp_part),
+                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   GemmArgs g{};
   g.M = M;
   g.N = H;
@@ -730,7 +758,8 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
   FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, base, status, s));
   // FC1 backward on d_h: G pass, dX GEMM, adapter gradients
   FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales,
-                        base + w.qdh.sf, P1, status, di.num_sms, s));
+                        base + w.qdh.sf, P1, reinterpret_cast<float*>(base + w.rp_part),
+                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   GemmArgs g1{};
   g1.M = M;
   g1.N = K1;
@@ -780,7 +809,7 @@ int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_
   rp.w_mn_major = 0;
   rp.kt_per_split = rs.kt_per_split;
   rp.nsplit = rs.nsplit;
-  rp.cluster_reduce = 0;  // partials in the static scratch, summed by the last CTA
+  rp.stages = rs.stages;
   rp.codes = codes;
   rp.scales = scales;
   rp.L = L;

@@ -94,32 +94,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// ------------------------------------------------------------------ clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// every thread of every CTA in the cluster arrives and waits (release/acquire).
-// The non-aligned forms: a warp may reach this with its lanes diverged.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-// address of the same shared-memory location in CTA `rank` of this cluster
-__device__ __forceinline__ uint32_t map_cluster(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(caddr)
-               : "memory");
-  return v;
-}
-
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -317,11 +291,9 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
   return r;
 }
 
-// Block16 quantization of 32 consecutive bf16 values of one row (two 16-column
-// blocks) given the two block maxima: scale = E4M3(amax / 6) (IEEE division),
-// code = E2M1(v / dec(scale)) rounded to nearest even, all +0 when the scale
-// decodes to 0.  Writes four 32-bit words of codes (element i of block j in word
-// 2j + i/8) and the two scale bytes.
+// Block16 quantization of consecutive bf16 values of one row, given the block
+// maximum: scale = E4M3(amax / 6) (IEEE division), code = E2M1(v / dec(scale))
+// rounded to nearest even, all +0 when the scale decodes to 0.
 //
 // The per-element division is replaced by an exact equivalent.  v is bf16 (at
 // most 8 significant bits) and d = dec(scale) an E4M3 value (at most 4), so v/d
@@ -336,41 +308,40 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
 __device__ __forceinline__ float snap19(float q) {
   return __uint_as_float((__float_as_uint(q) + 0x8u) & ~0xFu);
 }
+// One block: 16 values of one row and the block maximum -> two words of codes
+// (element i in bits 4(i%8).. of word i/8) and the scale byte.
+__device__ __forceinline__ void quantize_1block(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+  *sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+  const float d = e4m3_to_f32(*sc);
+  if (d == 0.0f) {
+    packed[0] = packed[1] = 0u;
+    return;
+  }
+  const float rd = __frcp_rn(d);
+  float q[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) q[e] = snap19(v[e] * rd);
+  packed[0] = f32x8_to_e2m1(q);
+  packed[1] = f32x8_to_e2m1(q + 8);
+}
 __device__ __forceinline__ void quantize_2blocks(const float* v, const float* amax, uint32_t* packed,
                                                  uint32_t* sc) {
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
-    const float d = e4m3_to_f32(sc[j]);
-    if (d == 0.0f) {
-      packed[2 * j] = packed[2 * j + 1] = 0u;
-      continue;
-    }
-    const float rd = __frcp_rn(d);
-    float q[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) q[e] = snap19(v[16 * j + e] * rd);
-    packed[2 * j] = f32x8_to_e2m1(q);
-    packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
-  }
+  for (int j = 0; j < 2; ++j) quantize_1block(v + 16 * j, amax[j], packed + 2 * j, sc + j);
 }
 
-// Block16 quantization of 32 float32 values (two 16-column blocks) with the
+// Block16 quantization of 16 float32 values (one block) with the
 // IEEE division v / dec(scale) per element -- for inputs with more significant
 // bits than bf16 (the GELU output), where the division-free shortcut above does
-// not apply.  Same outputs as quantize_2blocks.
-__device__ __forceinline__ void quantize_2blocks_div(const float* v, const float* amax, uint32_t* packed,
-                                                     uint32_t* sc) {
+// not apply.  Same outputs as quantize_1block.
+__device__ __forceinline__ void quantize_1block_div(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+  *sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+  const float d = e4m3_to_f32(*sc);
+  float q[16];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    sc[j] = f32_to_e4m3(__fdiv_rn(amax[j], 6.0f));
-    const float d = e4m3_to_f32(sc[j]);
-    float q[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[16 * j + e], d);
-    packed[2 * j] = f32x8_to_e2m1(q);
-    packed[2 * j + 1] = f32x8_to_e2m1(q + 8);
-  }
+  for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[e], d);
+  packed[0] = f32x8_to_e2m1(q);
+  packed[1] = f32x8_to_e2m1(q + 8);
 }
 
 // GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))), and its

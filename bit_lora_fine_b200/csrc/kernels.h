@@ -14,19 +14,17 @@ struct RowpassParams {
   int M, K, R;
   int w_mn_major;                        // 1: D [K, R]; 0: W^T [R, K]
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
-  int cluster_reduce;                    // splits of a row tile form a cluster and reduce through DSMEM
+  int stages;                            // TMA ring depth, 2..rowpass_stages()
   int gelu_input;                        // input is h: quantize a = GELU(h) (fp32) and project bf16(a)
   float* dbg_a;                          // gelu_input: optional fp32 copy of a [M, K] (null = none)
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
   uint8_t* sf_mma;                       // the same scales in the MMA-ready layout (null = not written)
   void* L;                               // bf16 [M, R]
-  float* part;                           // fp32 [nsplit, M, R] when nsplit > 1 and no cluster
-  int* counters;                         // [ceil(M/128)], zero on entry, left zero (no cluster)
+  float* part;                           // fp32 [nsplit, M, R] when nsplit > 1
+  int* counters;                         // [ceil(M/128)], zero on entry, left zero (nsplit > 1)
   int* status;
 };
-// largest split count the cluster reduction handles (portable cluster size)
-constexpr int kRowpassMaxClusterSplit = 8;
 
 // MMA-ready scale layout of a block16 operand with `rows` rows (along M or N)
 // and `cols` columns along K: for each 128-row chunk c and each 64-column
@@ -80,7 +78,8 @@ cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uin
                                    cudaStream_t stream);
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                            cudaStream_t stream);
-int rowpass_ctas_per_sm(int R, int w_mn_major);
+// Deepest TMA ring of the row pass that one CTA's shared memory holds (one CTA per SM).
+int rowpass_stages(int R, int w_mn_major);
 // persistent: min(tiles, num_sms) CTAs
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream);
