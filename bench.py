@@ -10,7 +10,10 @@ rank 32, LoRA rank 32, seeded synthetic bf16 data (synth.py).
 
 Prints one JSON line (rank 0).  `value` is device time from CUDA events summed
 over exactly K steps (L2 flushed before each step, outside the events, by a
-256 MB write followed by a 256 MB read of another buffer), max over ranks; `e2e` repeats the steps through the same C ABI with
+256 MB write followed by a 256 MB read of another buffer), max over ranks, with
+no event between the kernels of a step; K further steps with an event pair
+around every kernel give the per-kernel times (`kernels`, `roofline`);
+`e2e` repeats the steps through the same C ABI with
 inputs in pinned host memory (H2D of X and dY, D2H of dA and dB inside the
 timed region).  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload.  With N > 1 (torchrun) every rank runs an independent
@@ -239,29 +242,37 @@ def run_ours(args, rank, world, local_rank):
     ft.device_status(ws_f)
     ft.device_status(ws_b)
 
-    steps = [(mk_events(2), mk_events(2 * nf), mk_events(2 * nb)) for _ in range(args.steps)]
+    # timed region: K steps with no event between the kernels of a step (the
+    # kernels chain through programmatic dependent launch); then K more steps
+    # with an event pair around every kernel, for the per-kernel breakdown
+    steps = [mk_events(2) for _ in range(args.steps)]
+    ksteps = [(mk_events(2 * nf), mk_events(2 * nb)) for _ in range(args.steps)]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    for se, evf, evb in steps:
+    for se in steps:
         flush.zero_()
         se[0].record()
-        step(evf, evb)
+        step()
         se[1].record()
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    for evf, evb in ksteps:
+        flush.zero_()
+        step(evf, evb)
+    torch.cuda.synchronize()
     ft.device_status(ws_f)
     ft.device_status(ws_b)
 
-    total_ms = sum(se[0].elapsed_time(se[1]) for se, _, _ in steps)
+    total_ms = sum(se[0].elapsed_time(se[1]) for se in steps)
     per_kernel = {n: 0.0 for n in names}
-    for _, evf, evb in steps:
+    for evf, evb in ksteps:
         for i in range(nf):
             per_kernel[names[i]] += evf[2 * i].elapsed_time(evf[2 * i + 1])
         for i in range(nb):
@@ -341,6 +352,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": (fp4 + lr) * args.steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K + 2 * M * N, "d2h_bytes_per_step": 4 * K * r + 4 * r * N},
         "gpu_launches": args.steps * (nf + nb),
+        "kernel_breakdown": "per-kernel times from K separate steps with an event pair around every kernel",
         "roofline": roofline,
         "kernels": kern,
         "clocks": clk,

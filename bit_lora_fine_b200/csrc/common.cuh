@@ -84,6 +84,19 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
+// ------------------------------------------------------------------ dependent launch
+// Programmatic dependent launch (kernels launched with launch_pdl): the next
+// kernel on the stream may be scheduled once every CTA of this grid has issued
+// launch_dependents (its CTAs then run their prologue on SMs this grid has
+// left); wait_prior blocks until the previous grid has completed and its
+// memory operations are visible.  Every kernel here calls both right after
+// its prologue (barriers, TMEM, tensor-map prefetch) and before touching
+// global memory, so no read or write can race the neighbouring kernels.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -359,5 +372,22 @@ __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg)
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Launch with programmatic stream serialization (see pdl_wait_prior).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace ft

@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_prior();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -389,8 +391,7 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
   if (e != cudaSuccess) return e;
   const int tiles = ((p.N + BN - 1) / BN) * ((p.M + 127) / 128);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_fp4_kernel<BN><<<grid, kGmThreads, Lay::kSmem, stream>>>(tmA, tmB, tmA2, tmB2, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_fp4_kernel<BN>, dim3(grid), dim3(kGmThreads), Lay::kSmem, stream, tmA, tmB, tmA2, tmB2, p);
 }
 
 }  // namespace ft

@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_prior();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -349,8 +351,8 @@ static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& t
   cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS, GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  rowpass_kernel<RCOLS, GELU><<<dim3((p.M + 127) / 128, p.nsplit), kRpThreads, smem, stream>>>(tmX, tmW, p);
-  return cudaGetLastError();
+  return launch_pdl(rowpass_kernel<RCOLS, GELU>, dim3((p.M + 127) / 128, p.nsplit), dim3(kRpThreads), smem, stream,
+                    tmX, tmW, p);
 }
 
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,

@@ -77,6 +77,8 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait_prior();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -201,8 +203,8 @@ cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, cons
   if (e != cudaSuccess) return e;
   const int tiles0 = ((p0.P + 127) / 128) * p0.nsplit;
   const int tiles1 = ((p1.P + 127) / 128) * p1.nsplit;
-  tgrad_kernel<<<tiles0 + tiles1, kTgThreads, kTgSmem, stream>>>(tmT0, tmV0, tmT1, tmV1, p0, p1);
-  return cudaGetLastError();
+  return launch_pdl(tgrad_kernel, dim3(tiles0 + tiles1), dim3(kTgThreads), kTgSmem, stream, tmT0, tmV0, tmT1, tmV1,
+                    p0, p1);
 }
 
 }  // namespace ft
