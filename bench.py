@@ -369,14 +369,24 @@ def run_ours(args, rank, world, local_rank):
 
 
 def load_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if any."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summary profiles/traffic.txt; None when there is none or when the kernel's
+    source file has changed since the counters were taken (git blob hash)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            d = json.load(f)
-        return d.get(kernel)
+            for line in f:
+                parts = line.split()
+                if len(parts) != 4 or parts[0].startswith("#") or parts[0] != kernel:
+                    continue
+                with open(os.path.join(ROOT, parts[2]), "rb") as src:
+                    data = src.read()
+                blob = hashlib.sha1(b"blob %d\0" % len(data) + data).hexdigest()
+                return int(parts[1]) if blob == parts[3] else None
     except Exception:
         return None
+    return None
 
 
 def main():
