@@ -282,16 +282,20 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           }
         }
         if (p.nsplit > 1) {
-          // the last CTA of this row tile to finish sums every split's partial, in split order
-          __threadfence();
+          // the last CTA of this row tile to finish sums every split's partial, in
+          // split order.  One thread publishes the CTA's partial writes (ordered
+          // before it by the barrier) with a gpu-scope fence before its counter
+          // increment; the last CTA's fence after reading the counter orders the
+          // partial reads after every other CTA's increment.
           named_bar_sync(1, 32 * kRpEpiWarps);
           if (threadIdx.x == 128) {
+            __threadfence();
             const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
+            __threadfence();
             *s_last = (prev == p.nsplit - 1);
           }
           named_bar_sync(1, 32 * kRpEpiWarps);
           if (*s_last) {
-            __threadfence();
             const int c8n = R / 8;
             for (int idx = threadIdx.x - 128; idx < 128 * c8n; idx += 32 * kRpEpiWarps) {
               const int grow = m0 + idx / c8n;

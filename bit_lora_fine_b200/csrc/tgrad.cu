@@ -144,31 +144,39 @@ __global__ void __launch_bounds__(kTgThreads, 1)
       }
       bool write = true;
       if (p.nsplit > 1) {
+        // only the r columns that are output travel through the partials
+        const int nq = (p.r + 3) / 4;
         float4* dst = reinterpret_cast<float4*>(p.part + (static_cast<long long>(split) * Ppad + prow) * 64);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-        __threadfence();
+        for (int e = 0; e < 16; ++e)
+          if (e < nq) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+        // one thread publishes the CTA's partial (ordered before it by the
+        // barrier) with a gpu-scope fence before the counter increment; the last
+        // CTA's fence after the increment orders its partial reads after all others
         named_bar_sync(1, 128);
         if (threadIdx.x == 128) {
+          __threadfence();
           const int prev = atomicAdd(&p.counters[ptile], 1);
+          __threadfence();
           *s_last = (prev == p.nsplit - 1);
         }
         named_bar_sync(1, 128);
         write = *s_last != 0;
         if (write) {
           // sum every split's partial row in split order (vector loads, registers only)
-          __threadfence();
 #pragma unroll
           for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
           for (int sp = 0; sp < p.nsplit; ++sp) {
             const float4* src = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float4 x = __ldcg(src + e);
-              acc[4 * e] += x.x;
-              acc[4 * e + 1] += x.y;
-              acc[4 * e + 2] += x.z;
-              acc[4 * e + 3] += x.w;
+              if (e < nq) {
+                const float4 x = __ldcg(src + e);
+                acc[4 * e] += x.x;
+                acc[4 * e + 1] += x.y;
+                acc[4 * e + 2] += x.z;
+                acc[4 * e + 3] += x.w;
+              }
             }
           }
           if (threadIdx.x == 128) p.counters[ptile] = 0;
