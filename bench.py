@@ -357,6 +357,9 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kern,
         "clocks": clk,
     }
+    if world == 1 and not args.no_extra:
+        line["configs_extra"] = measure_extra(ft, synth, dev, flush, peaks, steps=max(3, min(args.steps, 10)),
+                                              warmup=max(1, min(args.warmup, 3)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, flop_s = time_oracle(M, repeats=1)
         t = min(times)
@@ -366,6 +369,105 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------------------ other workloads
+EXTRA_WORKLOADS = ("flux-mlp-3072", "flux-single-stream", "video-mlp-5120")
+
+
+def measure_extra(ft, synth, dev, flush, peaks, steps, warmup):
+    """The other workloads (MLP pair, single-stream block linears, video MLP): device
+    time of fwd+bwd steps (L2 flushed before each, no events inside), then one step
+    with an event pair around every kernel for the breakdown."""
+    import torch
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16)
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    out = {}
+    for name in EXTRA_WORKLOADS:
+        wl = synth.WORKLOADS[name]
+        M = wl.M
+        layers = []
+        for li, spec in enumerate(wl.layers):
+            p = synth.layer_params(spec, li)
+            layers.append(ft.Linear.from_weights(up(p["R"]), up(p["S_dn"]), up(p["S_up"]), up(p["A"]), up(p["B"]),
+                                                 up(p["bias"]) if p["bias"] is not None else None))
+        fp4 = lr = 0
+        for spec in wl.layers:
+            a, b = layer_work(M, spec.K, spec.N, spec.r_s, spec.r)
+            fp4, lr = fp4 + a, lr + b
+        if wl.kind == "mlp":
+            mlp = ft.MLP(layers[0], layers[1])
+            X = up(synth.layer_input(wl))
+            dY = up(synth.upstream_grad(wl, layer=1))
+            H, N2 = mlp.H, mlp.fc2.N
+            fo = (torch.empty((M, N2), dtype=torch.bfloat16, device=dev),
+                  torch.empty((M, H), dtype=torch.bfloat16, device=dev),
+                  torch.empty((M, mlp.fc1.R_all), dtype=torch.bfloat16, device=dev),
+                  torch.empty((M, mlp.fc2.R_all), dtype=torch.bfloat16, device=dev))
+            dX = torch.empty((M, mlp.fc1.K), dtype=torch.bfloat16, device=dev)
+            grads = (torch.zeros((mlp.fc1.K, mlp.fc1.r), dtype=torch.float32, device=dev),
+                     torch.zeros((mlp.fc1.r, mlp.fc1.N), dtype=torch.float32, device=dev),
+                     torch.zeros((mlp.fc2.K, mlp.fc2.r), dtype=torch.float32, device=dev),
+                     torch.zeros((mlp.fc2.r, mlp.fc2.N), dtype=torch.float32, device=dev))
+            wsf, wsb = mlp.fwd_workspace(M), mlp.bwd_workspace(M)
+            knames = [f"fwd.{k}" for k in ft.MLP_FWD_KERNELS] + [f"bwd.{k}" for k in ft.MLP_BWD_KERNELS]
+            nf = len(ft.MLP_FWD_KERNELS)
+
+            def step(evs=None, mlp=mlp, X=X, dY=dY, fo=fo, dX=dX, grads=grads, wsf=wsf, wsb=wsb, nf=nf):
+                ft.mlp_fwd(mlp, X, ws=wsf, out=fo, events=None if evs is None else evs[:2 * nf])
+                ft.mlp_bwd(mlp, dY, X, fo[1], fo[2], fo[3], grads=grads, ws=wsb, dX=dX,
+                           events=None if evs is None else evs[2 * nf:])
+        else:
+            specs = wl.layers
+            Xs = [up(synth.layer_input(wl, layer=li)) for li in range(len(specs))]
+            dYs = [up(synth.upstream_grad(wl, layer=li)) for li in range(len(specs))]
+            bufs = []
+            for li, lay in enumerate(layers):
+                bufs.append(dict(Y=torch.empty((M, lay.N), dtype=torch.bfloat16, device=dev),
+                                 L=torch.empty((M, lay.R_all), dtype=torch.bfloat16, device=dev),
+                                 dX=torch.empty((M, lay.K), dtype=torch.bfloat16, device=dev),
+                                 dA=torch.zeros((lay.K, lay.r), dtype=torch.float32, device=dev),
+                                 dB=torch.zeros((lay.r, lay.N), dtype=torch.float32, device=dev),
+                                 wsf=lay.fwd_workspace(M), wsb=lay.bwd_workspace(M)))
+            per = list(ft.FWD_KERNELS) + list(ft.BWD_KERNELS)
+            knames = [f"layer{li}.{k}" for li in range(len(layers)) for k in per]
+            nf = len(ft.FWD_KERNELS)
+
+            def step(evs=None, layers=layers, Xs=Xs, dYs=dYs, bufs=bufs, nf=nf, per=per):
+                for li, lay in enumerate(layers):
+                    b = bufs[li]
+                    e = None if evs is None else evs[2 * len(per) * li:2 * len(per) * (li + 1)]
+                    ft.linear_fwd(lay, Xs[li], ws=b["wsf"], Y=b["Y"], L=b["L"], events=None if e is None else e[:2 * nf])
+                    ft.linear_bwd(lay, dYs[li], Xs[li], b["L"], ws=b["wsb"], dX=b["dX"], dA=b["dA"], dB=b["dB"],
+                                  events=None if e is None else e[2 * nf:])
+        for _ in range(warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        kev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(knames))]
+        for e in kev:
+            e.record()
+        flush.zero_()
+        step(kev)
+        torch.cuda.synchronize()
+        kern = {n: round(kev[2 * i].elapsed_time(kev[2 * i + 1]) * 1e3, 1) for i, n in enumerate(knames)}
+        out[name] = {
+            "M": M, "layers": [[sp.K, sp.N, sp.r_s, sp.r] for sp in wl.layers], "kind": wl.kind, "steps": steps,
+            "ms_per_step": ms, "value": (fp4 + lr) / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "tokens_per_s": M / (ms / 1e3), "fp4_tflops": fp4 / (ms / 1e3) / 1e12,
+            "fp4_peak_frac": fp4 / (ms / 1e3) / 1e12 / fp4_peak, "kernels_us": kern,
+        }
+        del layers, step
+        torch.cuda.empty_cache()
+    return out
 
 
 def load_traffic(kernel):
@@ -396,6 +498,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' timings")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -437,6 +437,19 @@ int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t cols, int6
   return cuda_err(e);
 }
 
+int fourtune_quantize_block16_f32(const float* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                                  uint8_t* scales, void* stream) {
+  if (!x || !codes || !scales) return FT_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols || ld % 4) return FT_ERR_SHAPE;
+  if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(x) || (reinterpret_cast<uintptr_t>(codes) & 7u)) return FT_ERR_ALIGN;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  return cuda_err(ft::launch_quantize_block16_f32(x, static_cast<int>(rows), static_cast<int>(cols), ld, codes, scales,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, uint8_t* codes_t, void* stream) {
   if (!codes || !codes_t) return FT_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return FT_ERR_SHAPE;
@@ -644,7 +657,14 @@ int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, 
 int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
                      int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a, void* ws,
                      size_t ws_bytes, void* stream) {
-  const Events evs{nullptr, 0};
+  return fourtune_mlp_fwd_timed(fc1, fc2, X, M, Y, y_dtype, h_saved, L1_saved, L2_saved, dbg_a, ws, ws_bytes, stream,
+                                nullptr, 0);
+}
+
+int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
+                           int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a,
+                           void* ws, size_t ws_bytes, void* stream, void* const* events, int n_events) {
+  const Events evs{events, n_events};
   int st = check_mlp(fc1, fc2, false);
   if (st) return st;
   if (!X || !Y || !h_saved || !L1_saved || !L2_saved || !ws) return FT_ERR_INVALID_ARG;
@@ -709,7 +729,15 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
                      const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M, void* dX,
                      int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate, void* ws,
                      size_t ws_bytes, void* stream) {
-  const Events evs{nullptr, 0};
+  return fourtune_mlp_bwd_timed(fc1, fc2, dY, X, h_saved, L1_saved, L2_saved, M, dX, dx_dtype, dA1, dB1, dA2, dB2,
+                                accumulate, ws, ws_bytes, stream, nullptr, 0);
+}
+
+int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY, const ft_bf16* X,
+                           const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
+                           void* dX, int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate,
+                           void* ws, size_t ws_bytes, void* stream, void* const* events, int n_events) {
+  const Events evs{events, n_events};
   int st = check_mlp(fc1, fc2, true);
   if (st) return st;
   if (!dY || !X || !h_saved || !L1_saved || !L2_saved || !dX || !dA1 || !dB1 || !dA2 || !dB2 || !ws)

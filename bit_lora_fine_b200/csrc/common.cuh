@@ -343,32 +343,61 @@ __device__ __forceinline__ void quantize_2blocks(const float* v, const float* am
   for (int j = 0; j < 2; ++j) quantize_1block(v + 16 * j, amax[j], packed + 2 * j, sc + j);
 }
 
-// Block16 quantization of 16 float32 values (one block) with the
-// IEEE division v / dec(scale) per element -- for inputs with more significant
-// bits than bf16 (the GELU output), where the division-free shortcut above does
-// not apply.  Same outputs as quantize_1block.
-__device__ __forceinline__ void quantize_1block_div(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+// Block16 quantization of 16 float32 values (one block) of any precision (the
+// GELU output), with the semantics of the IEEE quotient fp32(v / d) but no
+// division per element.  q = v * RN(1/d) lies within 2^-22.4 (relative) of the
+// quotient, so the code of the quotient is the code of q unless an E2M1 rounding
+// threshold lies within [q (1 - 2^-21), q (1 + 2^-21)]: the codes of those two
+// ends (the conversion is monotonic in |x|) detect it, and only then is the
+// quotient computed by IEEE division.  Same outputs as quantize_1block.
+__device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
   *sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
   const float d = e4m3_to_f32(*sc);
-  float q[16];
+  if (d == 0.0f) {
+    packed[0] = packed[1] = 0u;
+    return;
+  }
+  const float rd = __frcp_rn(d);
+  constexpr float kDown = 1.0f - 0x1p-21f, kUp = 1.0f + 0x1p-21f;
+  float lo[16], hi[16];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) q[e] = (d == 0.0f) ? 0.0f : __fdiv_rn(v[e], d);
-  packed[0] = f32x8_to_e2m1(q);
-  packed[1] = f32x8_to_e2m1(q + 8);
+  for (int e = 0; e < 16; ++e) {
+    const float q = v[e] * rd;
+    lo[e] = q * kDown;
+    hi[e] = q * kUp;
+  }
+  uint32_t c0 = f32x8_to_e2m1(lo), c1 = f32x8_to_e2m1(lo + 8);
+  if (c0 != f32x8_to_e2m1(hi) || c1 != f32x8_to_e2m1(hi + 8)) {
+    float q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(v[e], d);
+    c0 = f32x8_to_e2m1(q);
+    c1 = f32x8_to_e2m1(q + 8);
+  }
+  packed[0] = c0;
+  packed[1] = c1;
 }
 
-// GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))), and its
-// derivative 0.5 (1 + t) + 0.5 h (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 h^2).
+// GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))), evaluated
+// through 0.5 (1 + tanh(u)) = 1 / (1 + e^{-2u}) =: s (no cancellation for very
+// negative h), so GELU(h) = h s.  Its derivative, with 1 - tanh(u)^2 = 4 s (1 - s)
+// and 1 - s = s e^{-2u}: GELU'(h) = s + 2 h s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 h^2).
+// u is clamped at -40 (e^{-2u} stays finite; s < 2e-35 there either way).  The
+// exponential and the quotient are the fast hardware forms (__expf, __fdividef):
+// over the range where s is not saturated (|2u| <= 20) e^{-2u} is within ~3e-6
+// (relative), which is the relative error of GELU(h) and of s.
 constexpr float kGeluC = 0.7978845608028654f;  // sqrt(2/pi)
 constexpr float kGeluK = 0.044715f;
 __device__ __forceinline__ float gelu_tanh(float h) {
-  const float t = tanhf(kGeluC * (h + kGeluK * h * h * h));
-  return 0.5f * h * (1.0f + t);
+  const float u = fmaxf(kGeluC * (h + kGeluK * h * h * h), -40.0f);
+  return __fdividef(h, 1.0f + __expf(-2.0f * u));
 }
 __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg) {
-  const float t = tanhf(kGeluC * (h + kGeluK * h * h * h));
-  *g = 0.5f * h * (1.0f + t);
-  *dg = 0.5f * (1.0f + t) + 0.5f * h * (1.0f - t * t) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
+  const float u = fmaxf(kGeluC * (h + kGeluK * h * h * h), -40.0f);
+  const float e = __expf(-2.0f * u);
+  const float s = __fdividef(1.0f, 1.0f + e);
+  *g = h * s;
+  *dg = s + 2.0f * h * s * (e * s) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }

@@ -82,7 +82,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-template <int BN>
+// GELU: the MLP's GELU-backward epilogue (its own instantiation, so that the
+// other epilogues do not carry its registers)
+template <int BN, bool GELU>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -261,9 +263,21 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     uint8_t* buf = epi + (warp - 4) * 1024;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const long long ldb = p.ldo * (p.out_bf16 ? 2 : 4);   // output row stride in bytes
-    const bool fast = p.out_bf16 && !p.epi_gelu_bwd;
+    const bool fast = !GELU && p.out_bf16;
     int j = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
+      // GELU backward: this lane's row of the saved hidden h for the warp's
+      // columns, loaded while the tile's MMAs run (zero past M or N)
+      uint4 hreg[GELU ? BN / 16 : 1];
+      if constexpr (GELU) {
+        const int hrow = (tile / tiles_n) * 128 + 32 * q + lane;
+        const int hcol = (tile % tiles_n) * BN + c_lo;
+        const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
+                                                         static_cast<long long>(hrow) * p.N + hcol);
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          hreg[k] = (hrow < p.M && hcol + 8 * k < p.N) ? hp[k] : make_uint4(0u, 0u, 0u, 0u);
+      }
       if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
       __syncwarp();
       tc_fence_after();
@@ -306,7 +320,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             store_rows32(buf, w, lane, out_rows + static_cast<long long>(nb) * 2, ldb, rows_left);
           }
         }
-      } else if (!p.out_bf16) {
+      } else if constexpr (!GELU) {
         // fp32 rows, 8 columns (32 bytes) at a time
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[16];
@@ -329,37 +343,22 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         if (lane == 0) mbar_arrive(acc_empty);
       } else {
         // GELU backward: d_h = bf16(acc * GELU'(h)) -> out, bf16(GELU(h)) -> out2
-        const int row = row0 + lane;
         uint8_t* out2_rows = static_cast<uint8_t*>(p.out2) + static_cast<long long>(row0) * ldb;
+#pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           const int nb = n0 + 16 * c;
           uint32_t v[16];
           tmem_ld_32x32b_x16(taddr + 16 * c, v);
           tmem_ld_wait();
           if (nb >= p.N || rows_left <= 0) continue;
-          float hv[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) hv[e] = 0.0f;
-          if (row < p.M) {
-            const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
-                                                             static_cast<long long>(row) * p.N + nb);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const uint4 u = hp[k];
-              const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                hv[8 * k + 2 * e] = bf16_bits_to_f32(wd[e] & 0xFFFFu);
-                hv[8 * k + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
-              }
-            }
-          }
+          const uint32_t hw[8] = {hreg[2 * c].x,     hreg[2 * c].y,     hreg[2 * c].z,     hreg[2 * c].w,
+                                  hreg[2 * c + 1].x, hreg[2 * c + 1].y, hreg[2 * c + 1].z, hreg[2 * c + 1].w};
           uint32_t wd_h[8], wg[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             float g0, d0, g1, d1;
-            gelu_tanh_and_grad(hv[2 * e], &g0, &d0);
-            gelu_tanh_and_grad(hv[2 * e + 1], &g1, &d1);
+            gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] & 0xFFFFu), &g0, &d0);
+            gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] >> 16), &g1, &d1);
             wd_h[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
             wg[e] = pack_bf16x2(g0, g1);
           }
@@ -386,12 +385,13 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
   using Lay = GemmLayout<BN>;
-  cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Lay::kSmem));
+  if (p.epi_gelu_bwd && !p.out_bf16) return cudaErrorInvalidValue;
+  auto kernel = p.epi_gelu_bwd ? gemm_fp4_kernel<BN, true> : gemm_fp4_kernel<BN, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Lay::kSmem));
   if (e != cudaSuccess) return e;
   const int tiles = ((p.N + BN - 1) / BN) * ((p.M + 127) / 128);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(gemm_fp4_kernel<BN>, dim3(grid), dim3(kGmThreads), Lay::kSmem, stream, tmA, tmB, tmA2, tmB2, p);
+  return launch_pdl(kernel, dim3(grid), dim3(kGmThreads), Lay::kSmem, stream, tmA, tmB, tmA2, tmB2, p);
 }
 
 }  // namespace ft

@@ -74,6 +74,8 @@ struct TgradParams {
 
 cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long ld, uint8_t* codes,
                                     uint8_t* scales, cudaStream_t stream);
+cudaError_t launch_quantize_block16_f32(const float* x, int rows, int cols, long long ld, uint8_t* codes,
+                                        uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uint8_t* codes_t,
                                    cudaStream_t stream);
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,

@@ -94,6 +94,67 @@ __global__ void __launch_bounds__(256) quantize_block16_kernel(const __nv_bfloat
   }
 }
 
+// The same strip decomposition for float32 input of any precision: two blocks per
+// lane through quantize_1block_f32 (the IEEE-quotient semantics without a division
+// per element).
+__global__ void __launch_bounds__(256) quantize_block16_f32_kernel(const float* __restrict__ x, int rows, int cols,
+                                                                   long long ld, uint8_t* __restrict__ codes,
+                                                                   uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int strips_per_row = (cols + 63) / 64;
+  const long long nstrips = static_cast<long long>(rows / 16) * strips_per_row;
+  if (warp >= nstrips) return;
+  const int rb = static_cast<int>(warp / strips_per_row);
+  const int c0 = static_cast<int>(warp % strips_per_row) * 64;
+  const int r = rb * 16 + (lane >> 1);
+  const int cstart = c0 + 32 * (lane & 1);
+  const int nblk = cstart < cols ? min(2, (cols - cstart) / 16) : 0;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+  const float4* src = reinterpret_cast<const float4*>(x + static_cast<long long>(r) * ld + cstart);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    if (q < 4 * nblk) {
+      const float4 f = src[q];
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  }
+  float amax[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[16 * j + i]));
+#pragma unroll
+    for (int off = 2; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    amax[j] = a;
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    if (j >= nblk) break;
+    uint32_t packed[2], sc;
+    quantize_1block_f32(v + 16 * j, amax[j], packed, &sc);
+    const int cb = cstart + 16 * j;
+    *reinterpret_cast<uint2*>(codes + static_cast<long long>(r) * (cols / 2) + cb / 2) = make_uint2(packed[0], packed[1]);
+    if ((lane >> 1) == 0) scales[static_cast<long long>(rb) * (cols / 16) + cb / 16] = static_cast<uint8_t>(sc);
+  }
+}
+
+cudaError_t launch_quantize_block16_f32(const float* x, int rows, int cols, long long ld, uint8_t* codes,
+                                        uint8_t* scales, cudaStream_t stream) {
+  const long long nstrips = static_cast<long long>(rows / 16) * ((cols + 63) / 64);
+  if (nstrips == 0) return cudaSuccess;
+  const int block = 256;
+  const long long grid = (nstrips * 32 + block - 1) / block;
+  quantize_block16_f32_kernel<<<static_cast<unsigned>(grid), block, 0, stream>>>(x, rows, cols, ld, codes, scales);
+  return cudaGetLastError();
+}
+
 // codes_t[c, r/2] = nibble (r & 1) <- code of element (r, c)
 __global__ void transpose_codes_kernel(const uint8_t* __restrict__ codes, int rows, int cols,
                                        uint8_t* __restrict__ codes_t) {

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         // rows past M and columns past K were zero-filled by the TMA: their scale is 0
         uint32_t packed[2], sc;
         if (GELU)
-          quantize_1block_div(v, amax, packed, &sc);
+          quantize_1block_f32(v, amax, packed, &sc);
         else
           quantize_1block(v, amax, packed, &sc);
         if (inside) {

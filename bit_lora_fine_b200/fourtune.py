@@ -26,11 +26,15 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_error_string", "fourtune_linear_fwd_timed", "fourtune_linear_bwd_timed",
             "fourtune_quant_down_static", "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_fwd",
             "fourtune_mlp_bwd_workspace_size", "fourtune_mlp_bwd", "fourtune_mlp_fwd_ws_offsets",
-            "fourtune_mlp_bwd_ws_offsets", "fourtune_mma_scales_size", "fourtune_mma_scales")
+            "fourtune_mlp_bwd_ws_offsets", "fourtune_mma_scales_size", "fourtune_mma_scales",
+            "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
 BWD_KERNELS = ("gpass_quant_down", "gemm_fp4_dx", "tgrad_dA_dB")
+MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1", "gelu_pass_quant_down", "gemm_fp4_fc2")
+MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_gelu_bwd_fc2", "tgrad_fc2", "dhpass_quant_down_fc1",
+                   "gemm_fp4_dx_fc1", "tgrad_fc1")
 
 
 class FourtuneError(RuntimeError):
@@ -61,6 +65,7 @@ def load():
     P = ctypes.POINTER
     L.fourtune_quantize_block16.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
     L.fourtune_transpose_codes.argtypes = [vp, i64, i64, vp, vp]
+    L.fourtune_quantize_block16_f32.argtypes = [vp, i64, i64, i64, vp, vp, vp]
     L.fourtune_mma_scales_size.argtypes = [i64, i64]
     L.fourtune_mma_scales_size.restype = sz
     L.fourtune_mma_scales.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp]
@@ -87,6 +92,8 @@ def load():
     L.fourtune_mlp_fwd.argtypes = [PL, PL, vp, i64, vp, ctypes.c_int, vp, vp, vp, vp, vp, sz, vp]
     L.fourtune_mlp_bwd.argtypes = [PL, PL, vp, vp, vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, vp, vp,
                                    ctypes.c_int, vp, sz, vp]
+    L.fourtune_mlp_fwd_timed.argtypes = list(L.fourtune_mlp_fwd.argtypes) + [P(vp), ctypes.c_int]
+    L.fourtune_mlp_bwd_timed.argtypes = list(L.fourtune_mlp_bwd.argtypes) + [P(vp), ctypes.c_int]
     L.fourtune_mlp_fwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz)]
     L.fourtune_mlp_bwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz), P(sz), P(sz)]
     for f in EXPORTED:
@@ -129,6 +136,17 @@ def quantize_block16(x, transposed=False):
     _check(load().fourtune_quantize_block16(_ptr(x), rows, cols, x.stride(0), _ptr(codes), _ptr(scales),
                                             _ptr(codes_t), _stream()), "fourtune_quantize_block16")
     return codes, scales, codes_t
+
+
+def quantize_block16_f32(x):
+    """x: float32 [rows, cols] -> (codes u8 [rows, cols/2], scales u8 [rows/16, cols/16])."""
+    _need(x, torch.float32, "x")
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows // 16, cols // 16), dtype=torch.uint8, device=x.device)
+    _check(load().fourtune_quantize_block16_f32(_ptr(x), rows, cols, x.stride(0), _ptr(codes), _ptr(scales),
+                                                _stream()), "fourtune_quantize_block16_f32")
+    return codes, scales
 
 
 def mma_scales(scales, rows, cols, transposed=False):
@@ -298,30 +316,39 @@ class MLP:
         return tuple(x.value for x in o)
 
 
-def mlp_fwd(mlp, X, y_dtype=torch.float32, ws=None, dbg_a=False):
-    """Returns (Y, h, L1, L2, ws, a) -- a is the fp32 activation when dbg_a, else None."""
+def mlp_fwd(mlp, X, y_dtype=torch.float32, ws=None, dbg_a=False, out=None, events=None):
+    """Returns (Y, h, L1, L2, ws, a) -- a is the fp32 activation when dbg_a, else None.
+    out: optional preallocated (Y, h, L1, L2); events: 2*len(MLP_FWD_KERNELS) torch.cuda.Events."""
     _need(X, torch.bfloat16, "X")
     M = X.shape[0]
     dev = X.device
-    Y = torch.empty((M, mlp.fc2.N), dtype=y_dtype, device=dev)
-    h = torch.empty((M, mlp.H), dtype=torch.bfloat16, device=dev)
-    L1 = torch.empty((M, mlp.fc1.R_all), dtype=torch.bfloat16, device=dev)
-    L2 = torch.empty((M, mlp.fc2.R_all), dtype=torch.bfloat16, device=dev)
+    if out is None:
+        Y = torch.empty((M, mlp.fc2.N), dtype=y_dtype, device=dev)
+        h = torch.empty((M, mlp.H), dtype=torch.bfloat16, device=dev)
+        L1 = torch.empty((M, mlp.fc1.R_all), dtype=torch.bfloat16, device=dev)
+        L2 = torch.empty((M, mlp.fc2.R_all), dtype=torch.bfloat16, device=dev)
+    else:
+        Y, h, L1, L2 = out
     a = torch.empty((M, mlp.H), dtype=torch.float32, device=dev) if dbg_a else None
     ws = mlp.fwd_workspace(M) if ws is None else ws
-    code = FT_DTYPE_F32 if y_dtype == torch.float32 else FT_DTYPE_BF16
-    _check(load().fourtune_mlp_fwd(ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(X), M, _ptr(Y), code,
-                                   _ptr(h), _ptr(L1), _ptr(L2), _ptr(a), _ptr(ws), ws.numel(), _stream()),
-           "fourtune_mlp_fwd")
+    code = FT_DTYPE_F32 if Y.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(X), M, _ptr(Y), code, _ptr(h), _ptr(L1),
+            _ptr(L2), _ptr(a), _ptr(ws), ws.numel(), _stream())
+    if events is None:
+        _check(load().fourtune_mlp_fwd(*args), "fourtune_mlp_fwd")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_mlp_fwd_timed(*args, arr, n), "fourtune_mlp_fwd_timed")
     return Y, h, L1, L2, ws, a
 
 
-def mlp_bwd(mlp, dY, X, h, L1, L2, dx_dtype=torch.float32, accumulate=False, grads=None, ws=None):
-    """Returns (dX, dA1, dB1, dA2, dB2, ws)."""
+def mlp_bwd(mlp, dY, X, h, L1, L2, dx_dtype=torch.float32, accumulate=False, grads=None, ws=None, dX=None,
+            events=None):
+    """Returns (dX, dA1, dB1, dA2, dB2, ws).  events: 2*len(MLP_BWD_KERNELS) torch.cuda.Events."""
     _need(dY, torch.bfloat16, "dY")
     M = dY.shape[0]
     dev = dY.device
-    dX = torch.empty((M, mlp.fc1.K), dtype=dx_dtype, device=dev)
+    dX = torch.empty((M, mlp.fc1.K), dtype=dx_dtype, device=dev) if dX is None else dX
     if grads is None:
         grads = (torch.zeros((mlp.fc1.K, mlp.fc1.r), dtype=torch.float32, device=dev),
                  torch.zeros((mlp.fc1.r, mlp.fc1.N), dtype=torch.float32, device=dev),
@@ -329,10 +356,15 @@ def mlp_bwd(mlp, dY, X, h, L1, L2, dx_dtype=torch.float32, accumulate=False, gra
                  torch.zeros((mlp.fc2.r, mlp.fc2.N), dtype=torch.float32, device=dev))
     dA1, dB1, dA2, dB2 = grads
     ws = mlp.bwd_workspace(M) if ws is None else ws
-    code = FT_DTYPE_F32 if dx_dtype == torch.float32 else FT_DTYPE_BF16
-    _check(load().fourtune_mlp_bwd(ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(dY), _ptr(X), _ptr(h),
-                                   _ptr(L1), _ptr(L2), M, _ptr(dX), code, _ptr(dA1), _ptr(dB1), _ptr(dA2), _ptr(dB2),
-                                   int(accumulate), _ptr(ws), ws.numel(), _stream()), "fourtune_mlp_bwd")
+    code = FT_DTYPE_F32 if dX.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(mlp.fc1.c), ctypes.byref(mlp.fc2.c), _ptr(dY), _ptr(X), _ptr(h), _ptr(L1), _ptr(L2), M,
+            _ptr(dX), code, _ptr(dA1), _ptr(dB1), _ptr(dA2), _ptr(dB2), int(accumulate), _ptr(ws), ws.numel(),
+            _stream())
+    if events is None:
+        _check(load().fourtune_mlp_bwd(*args), "fourtune_mlp_bwd")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_mlp_bwd_timed(*args, arr, n), "fourtune_mlp_bwd_timed")
     return dX, dA1, dB1, dA2, dB2, ws
 
 

@@ -105,6 +105,14 @@ typedef struct {
 FT_API int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
                               uint8_t* scales, uint8_t* codes_t, void* stream);
 
+/* The same block16 quantization of a float32 matrix x [rows, cols] (row stride
+ * `ld` elements, a multiple of 4): element codes follow the IEEE float32 quotient
+ * x / dec(scale), exactly as for bf16 input, for inputs of any precision (the
+ * MLP's fp32 GELU output is quantized this way, §3.3).  x 16-byte aligned,
+ * codes 8-byte aligned. */
+FT_API int fourtune_quantize_block16_f32(const float* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                                         uint8_t* scales, void* stream);
+
 /* Nibble transpose of block16 codes: codes [rows, cols/2] -> codes_t [cols, rows/2]
  * (§3.2: the transposed operand keeps its codes and scales). */
 FT_API int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, uint8_t* codes_t, void* stream);
@@ -184,6 +192,20 @@ FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
                             const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
                             void* dX, int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* The MLP calls with per-kernel CUDA events, as fourtune_linear_*_timed.  Kernels,
+ * in order -- forward: 0 X pass, 1 FC1 GEMM (h), 2 GELU pass (Q(a), L2), 3 FC2 GEMM;
+ * backward: 0 G pass (FC2), 1 FC2 dX GEMM with the GELU backward, 2 FC2 dA/dB,
+ * 3 d_h pass (FC1), 4 FC1 dX GEMM, 5 FC1 dA/dB. */
+FT_API int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M,
+                                  void* Y, int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved,
+                                  float* dbg_a, void* ws, size_t ws_bytes, void* stream, void* const* events,
+                                  int n_events);
+FT_API int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY,
+                                  const ft_bf16* X, const ft_bf16* h_saved, const ft_bf16* L1_saved,
+                                  const ft_bf16* L2_saved, int64_t M, void* dX, int dx_dtype, float* dA1, float* dB1,
+                                  float* dA2, float* dB2, int accumulate, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events, int n_events);
 
 /* Workspace byte offsets of the MLP's intermediate tensors (inspection, tests):
  * forward: Q(a) codes [M, H/2] and scales [M/16, H/16]; backward: d_h and

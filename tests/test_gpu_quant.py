@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 
 from bit_lora_fine_b200 import synth
-from oracle import block16
+from oracle import block16, formats
 from tests.helpers import tie_tensor, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
@@ -112,3 +112,39 @@ def test_mma_scale_layout(cuda_lib, rows, cols):
     np.testing.assert_array_equal(got, _mma_layout(rs, rows, cols, False))
     got_t = cuda_lib.mma_scales(sd, cols, rows, transposed=True).cpu().numpy()
     np.testing.assert_array_equal(got_t, _mma_layout(rs, cols, rows, True))
+
+
+def _near_tie_f32(rows, cols, seed):
+    """float32 blocks for the fp32-input quantizer: each 16x16 block gets a chosen
+    E4M3 scale d (one element is +-6 d, so amax / 6 = d exactly) and elements on,
+    and a few float32 ulps either side of, every E2M1 rounding threshold times d,
+    both signs -- the cases where the float32 rounding of the quotient decides the
+    code -- plus random values.  Scales run over subnormal, normal and near-448 codes."""
+    rng = np.random.default_rng(seed)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    codes = np.concatenate([np.arange(1, 8), rng.integers(8, 0x7F, size=64)])
+    x = np.zeros((rows, cols), np.float64)
+    for rb in range(rows // 16):
+        for cb in range(cols // 16):
+            d = float(formats.e4m3_decode(np.array([codes[(rb * 7 + cb) % len(codes)]], np.uint8))[0])
+            t = rng.choice(ties, size=(16, 16)) * rng.choice([-1.0, 1.0], size=(16, 16))
+            k = rng.integers(-6, 7, size=(16, 16))
+            blk = (t * d * (1.0 + k * 2.0 ** -24)).astype(np.float32).astype(np.float64)
+            rnd = rng.random((16, 16)) < 0.25
+            blk[rnd] = (rng.uniform(-6, 6, size=int(rnd.sum())) * d).astype(np.float32)
+            blk[0, 0] = 6.0 * d * rng.choice([-1.0, 1.0])
+            x[rb * 16:(rb + 1) * 16, cb * 16:(cb + 1) * 16] = blk
+    return x.astype(np.float32)
+
+
+@pytest.mark.parametrize("rows,cols,seed", [(64, 256, 0), (160, 96, 1), (512, 1024, 2)])
+def test_fp32_quantizer_near_ties(cuda_lib, rows, cols, seed):
+    """fourtune_quantize_block16_f32 (the division-free IEEE-quotient quantizer used
+    for the MLP's fp32 GELU output) bit for bit against the oracle at the E2M1
+    rounding thresholds."""
+    import torch
+    x = _near_tie_f32(rows, cols, seed)
+    c, s = cuda_lib.quantize_block16_f32(torch.from_numpy(x).to("cuda"))
+    rc, rs = block16.quantize(x)
+    np.testing.assert_array_equal(s.cpu().numpy(), rs)
+    np.testing.assert_array_equal(c.cpu().numpy(), rc)
