@@ -38,7 +38,8 @@
 namespace ft {
 
 constexpr int kGmStages = 4;
-constexpr int kGmThreads = 384;
+constexpr int kGmThreads = 384;      // warps 0-3 roles, 4-11 epilogue
+constexpr int kGmThreadsGelu = 640;  // GELU-backward variant: 16 epilogue warps
 
 template <int BN>
 struct GemmLayout {
@@ -85,7 +86,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // GELU: the MLP's GELU-backward epilogue (its own instantiation, so that the
 // other epilogues do not carry its registers)
 template <int BN, bool GELU>
-__global__ void __launch_bounds__(kGmThreads, 1)
+__global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmParams p) {
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   // fills, and their E4M3 bytes must not be NaN (they multiply zero codes).
   for (int s = 0; s < kGmStages; ++s) {
     uint4* z = reinterpret_cast<uint4*>(smem + s * Lay::kStage + Lay::kA + Lay::kB);
-    for (int k = threadIdx.x; k < static_cast<int>((Lay::kSFA + Lay::kSFB) / 16); k += kGmThreads)
+    for (int k = threadIdx.x; k < static_cast<int>((Lay::kSFA + Lay::kSFB) / 16); k += blockDim.x)
       z[k] = make_uint4(0u, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       mbar_init(&empty[s], 1);     // MMA commit
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);       // one arrive per epilogue warp
+    mbar_init(acc_empty, GELU ? 16 : 8);   // one arrive per epilogue warp
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -255,7 +256,72 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0, kWaitLimitNs);  // every MMA done before TMEM can be freed
     }
-  } else if (warp >= 4) {
+  } else if (GELU && warp >= 4) {
+    // GELU backward (FourTune §3.3 MLP): d_h = bf16(acc * GELU'(h)) -> out and
+    // bf16(GELU(h)) -> out2.  Four warps per TMEM lane quadrant, 64 columns each.
+    // GELU(h) does not need the accumulator: it is computed and stored while the
+    // tile's MMAs run, so the accumulator is held only for the d_h products.
+    // Rows are stored straight from registers (32 bytes per row and chunk).
+    constexpr int kCols = BN / 4;
+    const int q = warp & 3;
+    const int c_lo = ((warp - 4) >> 2) * kCols;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c_lo);
+    int j = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
+      const int m0 = (tile / tiles_n) * 128, n0 = (tile % tiles_n) * BN + c_lo;
+      const int row = m0 + 32 * q + lane;
+      const bool row_ok = row < p.M;
+      uint4 hreg[kCols / 8];
+      const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
+                                                       static_cast<long long>(row) * p.N + n0);
+#pragma unroll
+      for (int k = 0; k < kCols / 8; ++k)
+        hreg[k] = (row_ok && n0 + 8 * k < p.N) ? hp[k] : make_uint4(0u, 0u, 0u, 0u);
+      uint4* g_out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out2) + static_cast<long long>(row) * p.ldo + n0);
+#pragma unroll
+      for (int k = 0; k < kCols / 8; ++k) {
+        const uint32_t hw[4] = {hreg[k].x, hreg[k].y, hreg[k].z, hreg[k].w};
+        uint32_t wg[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          wg[e] = pack_bf16x2(gelu_tanh(bf16_bits_to_f32(hw[e] & 0xFFFFu)), gelu_tanh(bf16_bits_to_f32(hw[e] >> 16)));
+        if (row_ok && n0 + 8 * k < p.N) g_out[k] = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+      }
+      if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
+      __syncwarp();
+      tc_fence_after();
+      uint4* dh_out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(row) * p.ldo + n0);
+#pragma unroll 1
+      for (int c = 0; c < kCols / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(taddr + 16 * c, v);
+        tmem_ld_wait();
+        uint4 h0 = hreg[0], h1 = hreg[1];
+#pragma unroll
+        for (int k = 1; k < kCols / 16; ++k)
+          if (k == c) {
+            h0 = hreg[2 * k];
+            h1 = hreg[2 * k + 1];
+          }
+        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        uint32_t wd[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float g0, d0, g1, d1;
+          gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] & 0xFFFFu), &g0, &d0);
+          gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] >> 16), &g1, &d1);
+          wd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
+        }
+        if (row_ok && n0 + 16 * c < p.N) {
+          dh_out[2 * c] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          dh_out[2 * c + 1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+  } else if (!GELU && warp >= 4) {
     // two warps per TMEM lane quadrant, each owning half of the tile's columns
     const int q = warp & 3;
     const int c_lo = ((warp - 4) >> 2) * (BN / 2);
@@ -266,18 +332,6 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const bool fast = !GELU && p.out_bf16;
     int j = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
-      // GELU backward: this lane's row of the saved hidden h for the warp's
-      // columns, loaded while the tile's MMAs run (zero past M or N)
-      uint4 hreg[GELU ? BN / 16 : 1];
-      if constexpr (GELU) {
-        const int hrow = (tile / tiles_n) * 128 + 32 * q + lane;
-        const int hcol = (tile % tiles_n) * BN + c_lo;
-        const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
-                                                         static_cast<long long>(hrow) * p.N + hcol);
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          hreg[k] = (hrow < p.M && hcol + 8 * k < p.N) ? hp[k] : make_uint4(0u, 0u, 0u, 0u);
-      }
       if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
       __syncwarp();
       tc_fence_after();
@@ -320,7 +374,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             store_rows32(buf, w, lane, out_rows + static_cast<long long>(nb) * 2, ldb, rows_left);
           }
         }
-      } else if constexpr (!GELU) {
+      } else {
         // fp32 rows, 8 columns (32 bytes) at a time
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[16];
@@ -337,33 +391,6 @@ __global__ void __launch_bounds__(kGmThreads, 1)
               w[e] = __float_as_uint(__uint_as_float(v[8 * hlf + e]) + (bias ? __bfloat162float(bias[nb + e]) : 0.0f));
             store_rows32(buf, w, lane, out_rows + static_cast<long long>(nb) * 4, ldb, rows_left);
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
-      } else {
-        // GELU backward: d_h = bf16(acc * GELU'(h)) -> out, bf16(GELU(h)) -> out2
-        uint8_t* out2_rows = static_cast<uint8_t*>(p.out2) + static_cast<long long>(row0) * ldb;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          const int nb = n0 + 16 * c;
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(taddr + 16 * c, v);
-          tmem_ld_wait();
-          if (nb >= p.N || rows_left <= 0) continue;
-          const uint32_t hw[8] = {hreg[2 * c].x,     hreg[2 * c].y,     hreg[2 * c].z,     hreg[2 * c].w,
-                                  hreg[2 * c + 1].x, hreg[2 * c + 1].y, hreg[2 * c + 1].z, hreg[2 * c + 1].w};
-          uint32_t wd_h[8], wg[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float g0, d0, g1, d1;
-            gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] & 0xFFFFu), &g0, &d0);
-            gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] >> 16), &g1, &d1);
-            wd_h[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
-            wg[e] = pack_bf16x2(g0, g1);
-          }
-          store_rows32(buf, wd_h, lane, out_rows + static_cast<long long>(nb) * 2, ldb, rows_left);
-          store_rows32(buf, wg, lane, out2_rows + static_cast<long long>(nb) * 2, ldb, rows_left);
         }
         tc_fence_before();
         __syncwarp();
@@ -391,7 +418,8 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
   if (e != cudaSuccess) return e;
   const int tiles = ((p.N + BN - 1) / BN) * ((p.M + 127) / 128);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(kernel, dim3(grid), dim3(kGmThreads), Lay::kSmem, stream, tmA, tmB, tmA2, tmB2, p);
+  return launch_pdl(kernel, dim3(grid), dim3(p.epi_gelu_bwd ? kGmThreadsGelu : kGmThreads), Lay::kSmem, stream, tmA,
+                    tmB, tmA2, tmB2, p);
 }
 
 }  // namespace ft
