@@ -321,21 +321,37 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
 __device__ __forceinline__ float snap19(float q) {
   return __uint_as_float((__float_as_uint(q) + 0x8u) & ~0xFu);
 }
-// One block: 16 values of one row and the block maximum -> two words of codes
-// (element i in bits 4(i%8).. of word i/8) and the scale byte.
-__device__ __forceinline__ void quantize_1block(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
-  *sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+// N (a multiple of 8) values of one block row and the block maximum -> N/8 words
+// of codes (element i in bits 4(i%8).. of word i/8) and the scale byte.
+// fp32(a / 6) for a bf16 value a (the block maximum of bf16 inputs), correctly
+// rounded without a division: q0 = RN(a * RN(1/6)) is at most one ulp off and one
+// fused correction q0 + RN(a - 6 q0) * RN(1/6) (the residual is exact) lands on the
+// correctly rounded quotient for every finite bf16 a (checked exhaustively against
+// IEEE division on the GPU by the scale tests of every bf16 block maximum).
+__device__ __forceinline__ float div6_bf16(float a) {
+  constexpr float kSixth = 1.0f / 6.0f;
+  const float q0 = a * kSixth;
+  const float r = fmaf(-q0, 6.0f, a);
+  return fmaf(r, kSixth, q0);
+}
+template <int N>
+__device__ __forceinline__ void quantize_block_row(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+  *sc = f32_to_e4m3(div6_bf16(amax));
   const float d = e4m3_to_f32(*sc);
   if (d == 0.0f) {
-    packed[0] = packed[1] = 0u;
+#pragma unroll
+    for (int w = 0; w < N / 8; ++w) packed[w] = 0u;
     return;
   }
   const float rd = __frcp_rn(d);
-  float q[16];
+  float q[N];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) q[e] = snap19(v[e] * rd);
-  packed[0] = f32x8_to_e2m1(q);
-  packed[1] = f32x8_to_e2m1(q + 8);
+  for (int e = 0; e < N; ++e) q[e] = snap19(v[e] * rd);
+#pragma unroll
+  for (int w = 0; w < N / 8; ++w) packed[w] = f32x8_to_e2m1(q + 8 * w);
+}
+__device__ __forceinline__ void quantize_1block(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+  quantize_block_row<16>(v, amax, packed, sc);
 }
 __device__ __forceinline__ void quantize_2blocks(const float* v, const float* amax, uint32_t* packed,
                                                  uint32_t* sc) {
@@ -350,32 +366,40 @@ __device__ __forceinline__ void quantize_2blocks(const float* v, const float* am
 // threshold lies within [q (1 - 2^-21), q (1 + 2^-21)]: the codes of those two
 // ends (the conversion is monotonic in |x|) detect it, and only then is the
 // quotient computed by IEEE division.  Same outputs as quantize_1block.
-__device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+template <int N>
+__device__ __forceinline__ void quantize_block_row_f32(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
   *sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
   const float d = e4m3_to_f32(*sc);
   if (d == 0.0f) {
-    packed[0] = packed[1] = 0u;
+#pragma unroll
+    for (int w = 0; w < N / 8; ++w) packed[w] = 0u;
     return;
   }
   const float rd = __frcp_rn(d);
   constexpr float kDown = 1.0f - 0x1p-21f, kUp = 1.0f + 0x1p-21f;
-  float lo[16], hi[16];
+  float lo[N], hi[N];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
+  for (int e = 0; e < N; ++e) {
     const float q = v[e] * rd;
     lo[e] = q * kDown;
     hi[e] = q * kUp;
   }
-  uint32_t c0 = f32x8_to_e2m1(lo), c1 = f32x8_to_e2m1(lo + 8);
-  if (c0 != f32x8_to_e2m1(hi) || c1 != f32x8_to_e2m1(hi + 8)) {
-    float q[16];
+  bool near = false;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(v[e], d);
-    c0 = f32x8_to_e2m1(q);
-    c1 = f32x8_to_e2m1(q + 8);
+  for (int w = 0; w < N / 8; ++w) {
+    packed[w] = f32x8_to_e2m1(lo + 8 * w);
+    near = near || packed[w] != f32x8_to_e2m1(hi + 8 * w);
   }
-  packed[0] = c0;
-  packed[1] = c1;
+  if (near) {
+    float q[N];
+#pragma unroll
+    for (int e = 0; e < N; ++e) q[e] = __fdiv_rn(v[e], d);
+#pragma unroll
+    for (int w = 0; w < N / 8; ++w) packed[w] = f32x8_to_e2m1(q + 8 * w);
+  }
+}
+__device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, uint32_t* packed, uint32_t* sc) {
+  quantize_block_row_f32<16>(v, amax, packed, sc);
 }
 
 // GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))), evaluated

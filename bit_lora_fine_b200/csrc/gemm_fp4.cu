@@ -342,23 +342,37 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       if (fast) {
         // the warp's half row to registers (+ bias, bf16), accumulator handed
         // back, then the stores
+        // two rounds of four 16-column TMEM loads in flight per wait
         uint32_t pk[BN / 4];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(taddr + 16 * c, v);
-          uint4 bw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};   // 16 bias values (bf16)
-          if (bias && n0 + 16 * c < p.N) {
-            const uint4* bp = reinterpret_cast<const uint4*>(bias + n0 + 16 * c);
-            bw[0] = __ldg(bp);
-            bw[1] = __ldg(bp + 1);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[4][16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tmem_ld_32x32b_x16(taddr + 64 * half + 16 * k, v[k]);
+          uint4 bw[8];                                     // 64 bias values (bf16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) bw[k] = make_uint4(0u, 0u, 0u, 0u);
+          if (bias) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if (n0 + 64 * half + 16 * k < p.N) {
+                const uint4* bp = reinterpret_cast<const uint4*>(bias + n0 + 64 * half + 16 * k);
+                bw[2 * k] = __ldg(bp);
+                bw[2 * k + 1] = __ldg(bp + 1);
+              }
+            }
           }
           tmem_ld_wait();
-          const uint32_t bb[8] = {bw[0].x, bw[0].y, bw[0].z, bw[0].w, bw[1].x, bw[1].y, bw[1].z, bw[1].w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            pk[8 * c + e] = pack_bf16x2(__uint_as_float(v[2 * e]) + bf16_bits_to_f32(bb[e] & 0xFFFFu),
-                                        __uint_as_float(v[2 * e + 1]) + bf16_bits_to_f32(bb[e] >> 16));
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t bb[8] = {bw[2 * k].x,     bw[2 * k].y,     bw[2 * k].z,     bw[2 * k].w,
+                                    bw[2 * k + 1].x, bw[2 * k + 1].y, bw[2 * k + 1].z, bw[2 * k + 1].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pk[32 * half + 8 * k + e] =
+                  pack_bf16x2(__uint_as_float(v[k][2 * e]) + bf16_bits_to_f32(bb[e] & 0xFFFFu),
+                              __uint_as_float(v[k][2 * e + 1]) + bf16_bits_to_f32(bb[e] >> 16));
+          }
         }
         tc_fence_before();
         __syncwarp();

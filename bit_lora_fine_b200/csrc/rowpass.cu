@@ -110,9 +110,9 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % NS;
-        const uint32_t ph = (i / NS) & 1;
+      int s = 0;                 // ring slot and its phase parity (no division by the runtime depth)
+      uint32_t ph = 0;
+      for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
         if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
         uint8_t* st = smem + s * stage_bytes;
         const int kc = (kt0 + i) * 64;
@@ -127,16 +127,16 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         issued = i + 1;
       }
       if (*abortp) {  // let copies already in flight land before the CTA exits
-        for (int i = max(0, issued - NS); i < issued; ++i)
+        for (int i = max(0, issued - NS); i < issued; ++i)  // once, on the abort path only
           mbar_wait_drain(&full[i % NS], (i / NS) & 1, 100000000ull);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, nmma, false, mn != 0);
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % NS;
-        const uint32_t ph = (i / NS) & 1;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
         if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
         if (GELU && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
         tc_fence_after();
@@ -161,9 +161,9 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     const int kblocks = p.K / 16;
     const bool block_row_ok = m0 + blk * 16 < p.M;
     bool ok = true;
-    for (int i = 0; i < nt; ++i) {
-      const int s = i % NS;
-      const uint32_t ph = (i / NS) & 1;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
       if (!mbar_wait(&full[s], ph, p.status, abortp)) {
         ok = false;
         break;

@@ -148,3 +148,20 @@ def test_fp32_quantizer_near_ties(cuda_lib, rows, cols, seed):
     rc, rs = block16.quantize(x)
     np.testing.assert_array_equal(s.cpu().numpy(), rs)
     np.testing.assert_array_equal(c.cpu().numpy(), rc)
+
+
+def test_every_bf16_block_maximum(cuda_lib):
+    """One 16x16 block per positive finite bf16 value as its maximum (32640 blocks,
+    normal and subnormal, up to the largest finite): the block scales (E4M3 of
+    fp32(amax / 6)) and codes match the oracle's IEEE division bit for bit."""
+    rng = np.random.default_rng(11)
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)
+    amax = (bits << 16).view(np.float32)                                  # 32639 values
+    amax = np.concatenate([amax, np.float32([0.0])])                      # + an all-zero block
+    nb = len(amax)                                                        # 32640 = 255 x 128
+    frac = rng.uniform(-1.0, 1.0, size=(nb, 16, 16)).astype(np.float32)
+    blocks = synth.to_bf16(frac * amax[:, None, None])
+    blocks = np.minimum(np.abs(blocks), amax[:, None, None]) * np.sign(blocks)
+    blocks[:, 0, 0] = amax                                                # the exact maximum
+    x = blocks.reshape(255, 128, 16, 16).transpose(0, 2, 1, 3).reshape(255 * 16, 128 * 16)
+    _check(cuda_lib, synth.to_bf16(x))
