@@ -600,6 +600,9 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P,
                         reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                         di.num_sms, s));
+  // dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G -- right after the G pass, while G
+  // (just streamed by it) is still in L2
+  FT_TRY(1, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, s));
   // dX = deq(Q(G)) deq(Q(R)) + P D^T
   GemmArgs g{};
   g.M = M;
@@ -615,9 +618,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   g.B2 = layer->D;
   g.out = dX;
   g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
-  // dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G
-  FT_TRY(2, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, s));
+  FT_TRY(2, run_gemm(g, status, di.num_sms, s));
   return FT_OK;
 }
 
@@ -788,6 +789,8 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales,
                         base + w.qdh.sf, P1, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
+  // FC1 adapter gradients while d_h (just streamed by the d_h pass) is in L2
+  FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status, s));
   GemmArgs g1{};
   g1.M = M;
   g1.N = K1;
@@ -802,8 +805,7 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g1.B2 = fc1->D;
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(4, run_gemm(g1, status, di.num_sms, s));
-  FT_TRY(5, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status, s));
+  FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
   return FT_OK;
 }
 

@@ -158,8 +158,8 @@ FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, cons
  * `stream` around each kernel they launch: events[2k] before and events[2k+1]
  * after kernel k (NULL entries and k >= n_events/2 are skipped).  Kernels, in
  * order -- forward: 0 fused X pass (quantize + X D), 1 FP4 GEMM with
- * up-projection; backward: 0 fused G pass (quantize + G U^T), 1 FP4 dX GEMM,
- * 2 dA and dB.  Used for live per-kernel timing. */
+ * up-projection; backward: 0 fused G pass (quantize + G U^T), 1 dA and dB (run
+ * while G is still in L2), 2 FP4 dX GEMM.  Used for live per-kernel timing. */
 FT_API int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
                                      ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
@@ -196,7 +196,7 @@ FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
 /* The MLP calls with per-kernel CUDA events, as fourtune_linear_*_timed.  Kernels,
  * in order -- forward: 0 X pass, 1 FC1 GEMM (h), 2 GELU pass (Q(a), L2), 3 FC2 GEMM;
  * backward: 0 G pass (FC2), 1 FC2 dX GEMM with the GELU backward, 2 FC2 dA/dB,
- * 3 d_h pass (FC1), 4 FC1 dX GEMM, 5 FC1 dA/dB. */
+ * 3 d_h pass (FC1), 4 FC1 dA/dB, 5 FC1 dX GEMM. */
 FT_API int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M,
                                   void* Y, int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved,
                                   float* dbg_a, void* ws, size_t ws_bytes, void* stream, void* const* events,
