@@ -164,9 +164,11 @@ struct GradPair {
   size_t partA, partB;
 };
 size_t grad_counter_words(const ft_linear_t* L) { return cdiv(L->K, 128) + cdiv(L->N, 128); }
+// dA reads X from HBM; dB reads G, which the G pass has just streamed through L2,
+// so dA gets two thirds of the SMs
 void plan_grads(GradPair& g, const ft_linear_t* L, int64_t M, int num_sms) {
-  g.sA = m_split(M, L->K, std::max(1, num_sms / 2));
-  g.sB = m_split(M, L->N, std::max(1, num_sms / 2));
+  g.sA = m_split(M, L->K, std::max(1, 2 * num_sms / 3));
+  g.sB = m_split(M, L->N, std::max(1, num_sms / 3));
 }
 size_t grad_partial_bytes(const GradPair& g, const ft_linear_t* L) {
   const size_t a = g.sA.nsplit > 1 ? static_cast<size_t>(g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0;
