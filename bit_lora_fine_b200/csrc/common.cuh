@@ -426,6 +426,14 @@ __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg)
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
+// Maximum of a non-negative float over the 16 lanes of the warp whose lane bit 0
+// equals this lane's (two half-warp groups, reduced at once).  Non-negative
+// IEEE floats order like their bit patterns, so one integer max reduction does it.
+__device__ __forceinline__ float max16_same_parity(float a, int lane) {
+  const unsigned mask = (lane & 1) ? 0xAAAAAAAAu : 0x55555555u;
+  return __uint_as_float(__reduce_max_sync(mask, __float_as_uint(a)));
+}
+
 // Launch with programmatic stream serialization (see pdl_wait_prior).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,

@@ -206,11 +206,14 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
       }
-      float amax = 0.0f;
+      float m[8];                               // this lane's 16 magnitudes, tree-reduced
 #pragma unroll
-      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      for (int e = 0; e < 8; ++e) m[e] = fmaxf(fabsf(v[e]), fabsf(v[e + 8]));
 #pragma unroll
-      for (int off = 2; off < 32; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int e = 0; e < w; ++e) m[e] = fmaxf(m[e], m[e + w]);
+      const float amax = max16_same_parity(m[0], lane);   // over the block's 16 rows
       const int cstart = (kt0 + i) * 64 + colw;
       const bool inside = block_row_ok && cstart < p.K;
       if (inside || p.sf_mma) {
