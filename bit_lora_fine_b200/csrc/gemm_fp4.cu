@@ -13,16 +13,33 @@
 // Persistent kernel: one CTA per SM walks the 128 x BN output tiles (BN = 256)
 // in row-major tile order, so that the CTAs of one wave share the rows of A and
 // all of B in L2.  One pipeline stage = one K-block of 256 FP4 elements: the A
-// and B code boxes (128-byte swizzled rows) plus both operands' scales in the
-// MMA-ready layout (kernels.h), which come as plain bulk copies, so the MMA
-// warp only moves them smem -> TMEM.  Warp roles:
-//   warp 0 lane 0  producer: TMA code boxes + scale bulk copies per K-block;
-//                  then the bf16 low-rank blocks A2 [128 x 64] and B2
-//                  (K-major [BN x 64] or MN-major [64 x BN] in four boxes)
-//   warp 1         TMEM owner; lane 0 copies each stage's scales smem -> TMEM
-//                  (tcgen05.cp 32x128b.warpx4) and issues
+// and B code boxes (128-byte swizzled rows).  Both operands' scales, kept in
+// global memory in the MMA-ready layout (kernels.h), must sit in TMEM when
+// the MMAs run: the MMA reads A's scales of lane quadrant w from column
+// base + w of that quadrant, and B's scales from all four columns of every
+// quadrant, so B's scales are needed four times over.  Moving them with
+// tcgen05.cp 32x128b.warpx4 (which replicates into the four quadrants) costs
+// ~70 cycles a copy, 12 copies per K-block, on the same queue as the MMAs --
+// more than the 4 MMAs of the K-block take.  Instead four scale warps, one per
+// lane quadrant, load each K-block's scale words from global memory (L2) into
+// registers and write them into their quadrant with tcgen05.st, which runs
+// beside the MMAs.  (The GELU-backward variant, which needs all of its warps'
+// registers for its epilogue, keeps the copy path: the scale blocks come into
+// the stage by bulk copies and the MMA warp moves them with tcgen05.cp.)
+// Warp roles:
+//   warp 0 lane 0  producer: TMA code boxes per K-block (+ scale bulk copies in
+//                  the GELU variant); then the bf16 low-rank blocks A2
+//                  [128 x 64] and B2 (K-major [BN x 64] or MN-major [64 x BN]
+//                  in four boxes)
+//   warp 1         TMEM owner; lane 0 issues
 //                  tcgen05.mma kind::mxf4nvf4.block_scale.block16 (M=128,
-//                  N=BN, K=64), then kind::f16 for the low-rank blocks
+//                  N=BN, K=64) once a stage's codes and scales are in, then
+//                  kind::f16 for the low-rank blocks
+//   warps 12..15   scale warps (all but the GELU variant): warp 12+q fills
+//                  quadrant q's scale columns of each stage, one stage ahead
+//                  in registers; a stage's columns are rewritten only after
+//                  the MMAs that read them have completed (the stage's
+//                  empty barrier)
 //   warps 4..11    epilogue, warp w on TMEM lanes 32 (w % 4).. and half of the
 //                  columns.  bf16 output: the warp's accumulator slice goes to
 //                  registers (+ bias, packed to bf16), the accumulator is
@@ -38,16 +55,17 @@
 namespace ft {
 
 constexpr int kGmStages = 4;
-constexpr int kGmThreads = 384;      // warps 0-3 roles, 4-11 epilogue
-constexpr int kGmThreadsGelu = 640;  // GELU-backward variant: 16 epilogue warps
+constexpr int kGmThreads = 512;      // warps 0-3 roles, 4-11 epilogue, 12-15 scale warps
+constexpr int kGmThreadsGelu = 640;  // GELU-backward variant: 16 epilogue warps, copy path for scales
 
-template <int BN>
+template <int BN, bool kSmemScales>
 struct GemmLayout {
   static constexpr int kNC = BN / 128;                       // 128-row scale chunks of the B tile
   static constexpr uint32_t kA = 128 * 128;                  // A codes / A2 bf16 tile
   static constexpr uint32_t kB = BN * 128;                   // B codes / B2 bf16 tile
-  static constexpr uint32_t kSFA = 4 * 512;                  // A scales: 4 k-steps x 512 B
-  static constexpr uint32_t kSFB = kNC * 4 * 512;            // B scales: [chunk][k-step][512 B]
+  // scale blocks in the stage (copy path only): A 4 k-steps x 512 B, B [chunk][k-step][512 B]
+  static constexpr uint32_t kSFA = kSmemScales ? 4 * 512 : 0;
+  static constexpr uint32_t kSFB = kSmemScales ? kNC * 4 * 512 : 0;
   static constexpr uint32_t kStage = kA + kB + kSFA + kSFB;  // multiple of 1024
   static constexpr uint32_t kEpi = 8 * 1024;                 // one transpose buffer per epilogue warp
   static constexpr uint32_t kSmem = 1024 + kGmStages * kStage + kEpi + 256;
@@ -90,7 +108,9 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmParams p) {
-  using Lay = GemmLayout<BN>;
+  constexpr bool kCp = GELU;   // scales through the stage and tcgen05.cp (else scale warps)
+  using Lay = GemmLayout<BN, kCp>;
+  static_assert(kCp || Lay::kNC == 2, "scale warps store the B scales of two 128-row chunks (32 columns)");
   static_assert(Lay::kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(Lay::kTmemUsed <= 512, "TMEM budget");
   static_assert(Lay::kSmem <= 232448, "shared memory budget");
@@ -102,10 +122,11 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
   uint64_t* acc_full = empty + kGmStages;   // MMA -> epilogue: tile accumulated
   uint64_t* acc_empty = acc_full + 1;       // epilogue -> MMA: accumulator read out
   uint64_t* mma_done = acc_empty + 1;       // every MMA of the CTA completed (teardown)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* sf_full = mma_done + 1;         // scale warps -> MMA: a stage's scales are in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kGmStages);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   volatile int* abortp = abort_flag;
-  static_assert((2 * kGmStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
+  static_assert((3 * kGmStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = (p.K + 255) / 256;       // FP4 K-blocks
@@ -128,6 +149,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     for (int s = 0; s < kGmStages; ++s) {
       mbar_init(&full[s], 1);      // producer (expect_tx)
       mbar_init(&empty[s], 1);     // MMA commit
+      mbar_init(&sf_full[s], 4);   // one arrive per scale warp
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, GELU ? 16 : 8);   // one arrive per epilogue warp
@@ -170,20 +192,24 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
           }
           uint8_t* st = smem + s * Lay::kStage;
           if (i < KB) {
-            const int nks = min(4, KS - 4 * i);                 // k-steps of this K-block
-            const uint32_t sfbytes = static_cast<uint32_t>(nks) * 512u;
-            int nb = 0;
+            if (kCp) {
+              const int nks = min(4, KS - 4 * i);                 // k-steps of this K-block
+              const uint32_t sfbytes = static_cast<uint32_t>(nks) * 512u;
+              int nb = 0;
 #pragma unroll
-            for (int c = 0; c < Lay::kNC; ++c) nb += (n0 / 128 + c < nchunk_b) ? 1 : 0;
-            mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + sfbytes * static_cast<uint32_t>(1 + nb));
+              for (int c = 0; c < Lay::kNC; ++c) nb += (n0 / 128 + c < nchunk_b) ? 1 : 0;
+              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + sfbytes * static_cast<uint32_t>(1 + nb));
+              bulk_load(st + Lay::kA + Lay::kB, sfa + static_cast<size_t>(4 * i) * 512, sfbytes, &full[s]);
+#pragma unroll
+              for (int c = 0; c < Lay::kNC; ++c)
+                if (n0 / 128 + c < nchunk_b)
+                  bulk_load(st + Lay::kA + Lay::kB + Lay::kSFA + c * 2048,
+                            p.sfb + (static_cast<size_t>(n0 / 128 + c) * KS + 4 * i) * 512, sfbytes, &full[s]);
+            } else {
+              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
+            }
             tma_load_2d(st, &tmA, &full[s], i * 128, m0);
             tma_load_2d(st + Lay::kA, &tmB, &full[s], i * 128, n0);
-            bulk_load(st + Lay::kA + Lay::kB, sfa + static_cast<size_t>(4 * i) * 512, sfbytes, &full[s]);
-#pragma unroll
-            for (int c = 0; c < Lay::kNC; ++c)
-              if (n0 / 128 + c < nchunk_b)
-                bulk_load(st + Lay::kA + Lay::kB + Lay::kSFA + c * 2048,
-                          p.sfb + (static_cast<size_t>(n0 / 128 + c) * KS + 4 * i) * 512, sfbytes, &full[s]);
           } else {
             const int e = i - KB;
             mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
@@ -217,7 +243,8 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
         for (int i = 0; i < T; ++i) {
           const int s = g % kGmStages;
           const uint32_t ph = (g / kGmStages) & 1;
-          if (!mbar_wait(&full[s], ph, p.status, abortp)) {
+          if (!mbar_wait(&full[s], ph, p.status, abortp) ||
+              (!kCp && !mbar_wait(&sf_full[s], ph, p.status, abortp))) {
             ok = false;
             break;
           }
@@ -229,12 +256,14 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
             const uint32_t sfa_addr = b_addr + Lay::kB;
             const uint32_t sfb_addr = sfa_addr + Lay::kSFA;
             const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
-            for (int t = 0; t < nks; ++t) {
-              tmem_cp_32x128b_x4(tmem + sf_col + 4 * t, desc_sf_copy(sfa_addr + t * 512));
+            if (kCp) {
+              for (int t = 0; t < nks; ++t) {
+                tmem_cp_32x128b_x4(tmem + sf_col + 4 * t, desc_sf_copy(sfa_addr + t * 512));
 #pragma unroll
-              for (int c = 0; c < Lay::kNC; ++c)
-                tmem_cp_32x128b_x4(tmem + sf_col + 16 + (t * Lay::kNC + c) * 4,
-                                   desc_sf_copy(sfb_addr + (c * 4 + t) * 512));
+                for (int c = 0; c < Lay::kNC; ++c)
+                  tmem_cp_32x128b_x4(tmem + sf_col + 16 + (t * Lay::kNC + c) * 4,
+                                     desc_sf_copy(sfb_addr + (c * 4 + t) * 512));
+              }
             }
             for (int t = 0; t < nks; ++t)
               mma_fp4_block16(tmem, desc_kmajor_sw128(a_addr + 32 * t), desc_kmajor_sw128(b_addr + 32 * t), idesc4,
@@ -320,6 +349,75 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
+    }
+  } else if (!kCp && warp >= 12) {
+    // Scale warp of TMEM lane quadrant q.  Stage columns (from sf_col): A's
+    // k-step t at 4t..4t+3, of which the MMA reads 4t+q here (the diagonal
+    // word of the 512-byte block: rows 32q+lane, byte 16*lane + 4q); B's
+    // k-step t, chunk c at 16+8t+4c..+3, all four (the block's words
+    // 16*lane..16*lane+15, i.e. rows 32j+lane of the chunk, j = 0..3).
+    const int q = warp & 3;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    const int bx = static_cast<int>(blockIdx.x), gx = static_cast<int>(gridDim.x);
+    const int G = (bx < tiles ? (tiles - 1 - bx) / gx + 1 : 0) * T;
+    constexpr int NB = 4 * 4 * Lay::kNC;
+    auto fetch = [&](int gg, uint32_t (&a)[4], uint32_t (&b)[NB]) {
+      const int tile = bx + (gg / T) * gx;
+      const int i = gg % T;
+      const int nks = i < KB ? min(4, KS - 4 * i) : 0;
+      const int mc = tile / tiles_n, nc = (tile % tiles_n) * Lay::kNC;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        a[t] = 0u;
+        if (t < nks)
+          a[t] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa + (static_cast<size_t>(mc) * KS + 4 * i + t) * 512 +
+                                                         16 * lane + 4 * q));
+      }
+#pragma unroll
+      for (int c = 0; c < Lay::kNC; ++c) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);   // zero scales past N (their codes are zero)
+          if (t < nks && nc + c < nchunk_b)
+            x = __ldg(reinterpret_cast<const uint4*>(p.sfb + (static_cast<size_t>(nc + c) * KS + 4 * i + t) * 512 +
+                                                     16 * lane));
+          b[4 * (t * Lay::kNC + c)] = x.x;
+          b[4 * (t * Lay::kNC + c) + 1] = x.y;
+          b[4 * (t * Lay::kNC + c) + 2] = x.z;
+          b[4 * (t * Lay::kNC + c) + 3] = x.w;
+        }
+      }
+    };
+    auto put = [&](int gg, const uint32_t (&a)[4], const uint32_t (&b)[NB]) -> bool {
+      const int s = gg % kGmStages;
+      const uint32_t ph = (gg / kGmStages) & 1;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(&empty[s], ph ^ 1, p.status, abortp);   // MMAs that read the slot are done
+      okw = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
+      if (!okw) return false;
+      tc_fence_after();
+      if (gg % T < KB) {
+        const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
+        uint32_t a16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a16[e] = a[e >> 2];
+        tmem_st_32x32b_x16(trow + sf_col, a16);
+        tmem_st_32x32b_x32(trow + sf_col + 16, b);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sf_full[s]);
+      return true;
+    };
+    // two register sets: stage gg+1's loads are in flight while stage gg is stored
+    uint32_t a0[4], b0[NB], a1[4], b1[NB];
+    if (G > 0) fetch(0, a0, b0);
+    for (int gg = 0; gg < G; gg += 2) {
+      if (gg + 1 < G) fetch(gg + 1, a1, b1);
+      if (!put(gg, a0, b0) || gg + 1 >= G) break;
+      if (gg + 2 < G) fetch(gg + 2, a0, b0);
+      if (!put(gg + 1, a1, b1)) break;
     }
   } else if (!GELU && warp >= 4) {
     // two warps per TMEM lane quadrant, each owning half of the tile's columns
@@ -425,14 +523,14 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
-  using Lay = GemmLayout<BN>;
   if (p.epi_gelu_bwd && !p.out_bf16) return cudaErrorInvalidValue;
   auto kernel = p.epi_gelu_bwd ? gemm_fp4_kernel<BN, true> : gemm_fp4_kernel<BN, false>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Lay::kSmem));
+  const uint32_t smem = p.epi_gelu_bwd ? GemmLayout<BN, true>::kSmem : GemmLayout<BN, false>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = ((p.N + BN - 1) / BN) * ((p.M + 127) / 128);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(kernel, dim3(grid), dim3(p.epi_gelu_bwd ? kGmThreadsGelu : kGmThreads), Lay::kSmem, stream, tmA,
+  return launch_pdl(kernel, dim3(grid), dim3(p.epi_gelu_bwd ? kGmThreadsGelu : kGmThreads), smem, stream, tmA,
                     tmB, tmA2, tmB2, p);
 }
 
