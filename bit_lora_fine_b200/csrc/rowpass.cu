@@ -18,11 +18,13 @@
 //                  and the 32-column half w%2 of the smem tile, a lane one
 //                  16x16 block row (block amax by warp shuffles), so that the
 //                  ALU work of the quantizer is spread over enough warps to
-//                  hide its latency.  Warps 4..11 then drain the accumulator
-//                  (two per TMEM lane quadrant).  One split: L in bf16 straight
-//                  from TMEM.  Several splits: each CTA writes its fp32 partial
-//                  to scratch, and the last CTA of the row tile (split counter)
-//                  sums them in split order (deterministic), rounding once.
+//                  hide its latency.  The same sixteen warps then drain the
+//                  accumulator (four per TMEM lane quadrant, 16 columns
+//                  each).  One split: L in bf16 straight from TMEM.  Several
+//                  splits: each CTA writes its fp32 partial to scratch, and
+//                  the last CTA of the row tile (split counter) sums them in
+//                  split order (deterministic), rounding once, with a batch of
+//                  splits of two 4-column pieces in flight per thread.
 // The projection matrix is read either K-major (W^T [R, K], rows of 128 bytes,
 // N = R) or MN-major (D [K, R] with R contiguous: TMA boxes of 64 k-rows x 64
 // r, N = R rounded up to 64, the extra columns zero-filled by the TMA).
@@ -35,10 +37,11 @@ namespace ft {
 
 constexpr int kRpStages = 8;               // largest ring (p.stages <= this)
 constexpr int kRpQuantWarps = 16;
-constexpr int kRpEpiWarps = 8;
 constexpr int kRpThreads = 32 * (4 + kRpQuantWarps);
 constexpr uint32_t kRpXBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kRpSumBatch = 4;             // split partials loaded per batch by the last CTA
+constexpr int kRpSumItems = 2;             // 4-column pieces per thread and pass of that sum
+constexpr uint32_t kRpTail = 512;          // barriers, TMEM slot, flags
 
 __host__ __device__ constexpr int rp_mn_chunks(int R) { return (R + 63) / 64; }
 __host__ __device__ constexpr int rp_n_mma(int R, int mn) { return mn ? 64 * rp_mn_chunks(R) : R; }
@@ -49,7 +52,7 @@ __host__ __device__ constexpr uint32_t rp_stage_bytes(int R, int mn) {
   return kRpXBytes + ((rp_w_bytes(R, mn) + 1023u) & ~1023u);
 }
 __host__ __device__ constexpr uint32_t rp_smem_bytes(int R, int mn, int stages) {
-  return 1024 + stages * rp_stage_bytes(R, mn) + 256;
+  return 1024 + stages * rp_stage_bytes(R, mn) + kRpTail;
 }
 
 template <int RCOLS, bool GELU>
@@ -71,7 +74,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + NS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
-  volatile int* s_ok = s_last + 1;  // [kRpEpiWarps]
+  volatile int* s_ok = s_last + 1;  // [kRpQuantWarps]
   volatile int* abortp = abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -243,16 +246,16 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       }
     }
 
-    // ---- epilogue (warps 4..11): accumulator -> L (bf16) or fp32 partials.
-    // All eight agree on whether to run it, so the named barriers below are
-    // always reached by all of them.
-    if (w16 < kRpEpiWarps) {
+    // ---- epilogue (all sixteen quantizer warps): accumulator -> L (bf16) or
+    // fp32 partials.  All agree on whether to run it, so the named barriers
+    // below are always reached by all of them.
+    {
       const bool mine = ok && mbar_wait(acc_full, 0, p.status, abortp);
       if (lane == 0) s_ok[w16] = mine ? 1 : 0;
-      named_bar_sync(1, 32 * kRpEpiWarps);
+      named_bar_sync(1, 32 * kRpQuantWarps);
       bool go = true;
 #pragma unroll
-      for (int w = 0; w < kRpEpiWarps; ++w) go = go && s_ok[w];
+      for (int w = 0; w < kRpQuantWarps; ++w) go = go && s_ok[w];
       if (go) {
         __syncwarp();
         tc_fence_after();
@@ -260,8 +263,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         const int row = m0 + 32 * q + lane;
         const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
         const bool row_ok = row < p.M;
-        const int half = w16 >> 2;                    // which 16-column chunks this warp drains
-        for (int c0 = 16 * half; c0 < R; c0 += 32) {
+        for (int c0 = 16 * (w16 >> 2); c0 < R; c0 += 64) {   // this warp's 16-column chunks
           uint32_t v[16];
           tmem_ld_32x32b_x16(taddr + c0, v);
           tmem_ld_wait();
@@ -290,50 +292,61 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           // before it by the barrier) with a gpu-scope fence before its counter
           // increment; the last CTA's fence after reading the counter orders the
           // partial reads after every other CTA's increment.
-          named_bar_sync(1, 32 * kRpEpiWarps);
+          named_bar_sync(1, 32 * kRpQuantWarps);
           if (threadIdx.x == 128) {
             __threadfence();
             const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
             __threadfence();
             *s_last = (prev == p.nsplit - 1);
           }
-          named_bar_sync(1, 32 * kRpEpiWarps);
+          named_bar_sync(1, 32 * kRpQuantWarps);
           if (*s_last) {
-            const int c8n = R / 8;
-            for (int idx = threadIdx.x - 128; idx < 128 * c8n; idx += 32 * kRpEpiWarps) {
-              const int grow = m0 + idx / c8n;
-              const int c = 8 * (idx % c8n);
-              if (grow >= p.M) continue;
-              float acc[8];
+            // pieces of 4 columns; a thread takes kRpSumItems of them per pass, with
+            // a batch of splits of all of them in flight before the in-order sums
+            constexpr int kT = 32 * kRpQuantWarps;
+            const int c4n = R / 4;
+            const int npiece = 128 * c4n;
+            const int tid = static_cast<int>(threadIdx.x) - 128;
+            for (int base = tid; base < npiece; base += kRpSumItems * kT) {
+              float4 acc[kRpSumItems];
+              long long off[kRpSumItems];
+              bool live[kRpSumItems];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+              for (int j = 0; j < kRpSumItems; ++j) {
+                const int idx = base + j * kT;
+                const int grow = m0 + idx / c4n;
+                live[j] = idx < npiece && grow < p.M;
+                off[j] = static_cast<long long>(grow) * R + 4 * (idx % c4n);
+                acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              }
               for (int sp0 = 0; sp0 < p.nsplit; sp0 += kRpSumBatch) {
-                float4 a[kRpSumBatch][2];   // a batch of splits in flight, then summed in order
+                float4 a[kRpSumBatch][kRpSumItems];
 #pragma unroll
-                for (int j = 0; j < kRpSumBatch; ++j) {
-                  if (sp0 + j < p.nsplit) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.part + (static_cast<long long>(sp0 + j) * p.M + grow) * R + c);
-                    a[j][0] = __ldcg(src);
-                    a[j][1] = __ldcg(src + 1);
-                  }
-                }
+                for (int b = 0; b < kRpSumBatch; ++b)
 #pragma unroll
-                for (int j = 0; j < kRpSumBatch; ++j) {
-                  if (sp0 + j < p.nsplit) {
-                    acc[0] += a[j][0].x; acc[1] += a[j][0].y; acc[2] += a[j][0].z; acc[3] += a[j][0].w;
-                    acc[4] += a[j][1].x; acc[5] += a[j][1].y; acc[6] += a[j][1].z; acc[7] += a[j][1].w;
-                  }
-                }
+                  for (int j = 0; j < kRpSumItems; ++j)
+                    if (live[j] && sp0 + b < p.nsplit)
+                      a[b][j] = __ldcg(reinterpret_cast<const float4*>(
+                          p.part + static_cast<long long>(sp0 + b) * p.M * R + off[j]));
+#pragma unroll
+                for (int b = 0; b < kRpSumBatch; ++b)
+#pragma unroll
+                  for (int j = 0; j < kRpSumItems; ++j)
+                    if (live[j] && sp0 + b < p.nsplit) {
+                      acc[j].x += a[b][j].x;
+                      acc[j].y += a[b][j].y;
+                      acc[j].z += a[b][j].z;
+                      acc[j].w += a[b][j].w;
+                    }
               }
-              uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 bb = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-                w[e] = *reinterpret_cast<const uint32_t*>(&bb);
+              for (int j = 0; j < kRpSumItems; ++j) {
+                if (!live[j]) continue;
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x, acc[j].y);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z, acc[j].w);
+                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.L) + off[j]) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
               }
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.L) + static_cast<long long>(grow) * R + c) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
             }
             if (threadIdx.x == 128) p.counters[blockIdx.x] = 0;
           }
@@ -378,7 +391,7 @@ cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const
 }
 
 int rowpass_stages(int R, int w_mn_major) {
-  const int fit = (232448 - 1024 - 256) / static_cast<int>(rp_stage_bytes(R, w_mn_major));
+  const int fit = (232448 - 1024 - static_cast<int>(kRpTail)) / static_cast<int>(rp_stage_bytes(R, w_mn_major));
   return fit < kRpStages ? fit : kRpStages;
 }
 
