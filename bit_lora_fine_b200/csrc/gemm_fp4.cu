@@ -439,37 +439,31 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       uint8_t* out_rows = static_cast<uint8_t*>(p.out) + static_cast<long long>(row0) * ldb;
       if (fast) {
         // the warp's half row to registers (+ bias, bf16), accumulator handed
-        // back, then the stores
-        // two rounds of four 16-column TMEM loads in flight per wait
+        // back, then the stores.  Four rounds of 32 columns (two 16-column TMEM
+        // loads in flight per wait): the packed row and one round fit the
+        // register budget without spilling.
         uint32_t pk[BN / 4];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[4][16];
+        for (int rd = 0; rd < BN / 64; ++rd) {
+          uint32_t v[2][16];
+          tmem_ld_32x32b_x16(taddr + 32 * rd, v[0]);
+          tmem_ld_32x32b_x16(taddr + 32 * rd + 16, v[1]);
+          uint4 bw[4];                                     // 32 bias values (bf16)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) tmem_ld_32x32b_x16(taddr + 64 * half + 16 * k, v[k]);
-          uint4 bw[8];                                     // 64 bias values (bf16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) bw[k] = make_uint4(0u, 0u, 0u, 0u);
-          if (bias) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (n0 + 64 * half + 16 * k < p.N) {
-                const uint4* bp = reinterpret_cast<const uint4*>(bias + n0 + 64 * half + 16 * k);
-                bw[2 * k] = __ldg(bp);
-                bw[2 * k + 1] = __ldg(bp + 1);
-              }
-            }
+          for (int k = 0; k < 4; ++k) {
+            bw[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (bias && n0 + 32 * rd + 8 * k < p.N) bw[k] = __ldg(reinterpret_cast<const uint4*>(bias + n0 + 32 * rd) + k);
           }
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t bb[8] = {bw[2 * k].x,     bw[2 * k].y,     bw[2 * k].z,     bw[2 * k].w,
-                                    bw[2 * k + 1].x, bw[2 * k + 1].y, bw[2 * k + 1].z, bw[2 * k + 1].w};
+          for (int k = 0; k < 2; ++k) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              pk[32 * half + 8 * k + e] =
-                  pack_bf16x2(__uint_as_float(v[k][2 * e]) + bf16_bits_to_f32(bb[e] & 0xFFFFu),
-                              __uint_as_float(v[k][2 * e + 1]) + bf16_bits_to_f32(bb[e] >> 16));
+            for (int e = 0; e < 8; ++e) {
+              const uint4 b4 = bw[2 * k + e / 4];
+              const uint32_t bb = (e & 3) == 0 ? b4.x : (e & 3) == 1 ? b4.y : (e & 3) == 2 ? b4.z : b4.w;
+              pk[16 * rd + 8 * k + e] = pack_bf16x2(__uint_as_float(v[k][2 * e]) + bf16_bits_to_f32(bb & 0xFFFFu),
+                                                    __uint_as_float(v[k][2 * e + 1]) + bf16_bits_to_f32(bb >> 16));
+            }
           }
         }
         tc_fence_before();

@@ -163,19 +163,39 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         named_bar_sync(1, 128);
         write = *s_last != 0;
         if (write) {
-          // sum every split's partial row in split order (vector loads, registers only)
+          // sum every split's partial row in split order (vector loads, registers
+          // only), two splits' loads in flight at a time
 #pragma unroll
           for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-          for (int sp = 0; sp < p.nsplit; ++sp) {
-            const float4* src = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
+          for (int sp = 0; sp < p.nsplit; sp += 2) {
+            const float4* src0 = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
+            const float4* src1 = src0 + static_cast<long long>(Ppad) * 16;
+            const bool two = sp + 1 < p.nsplit;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              if (e < nq) {
-                const float4 x = __ldcg(src + e);
-                acc[4 * e] += x.x;
-                acc[4 * e + 1] += x.y;
-                acc[4 * e + 2] += x.z;
-                acc[4 * e + 3] += x.w;
+            for (int h = 0; h < 2; ++h) {   // 8 float4 of each split per round (registers)
+              float4 x0[8], x1[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (8 * h + e < nq) {
+                  x0[e] = __ldcg(src0 + 8 * h + e);
+                  if (two) x1[e] = __ldcg(src1 + 8 * h + e);
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (8 * h + e < nq) {
+                  const int c = 4 * (8 * h + e);
+                  acc[c] += x0[e].x;
+                  acc[c + 1] += x0[e].y;
+                  acc[c + 2] += x0[e].z;
+                  acc[c + 3] += x0[e].w;
+                  if (two) {
+                    acc[c] += x1[e].x;
+                    acc[c + 1] += x1[e].y;
+                    acc[c + 2] += x1[e].z;
+                    acc[c + 3] += x1[e].w;
+                  }
+                }
               }
             }
           }
