@@ -13,9 +13,12 @@ over exactly K steps (L2 flushed before each step, outside the events, by a
 256 MB write followed by a 256 MB read of another buffer), max over ranks, with
 no event between the kernels of a step; K further steps with an event pair
 around every kernel give the per-kernel times (`kernels`, `roofline`);
-`e2e` repeats the steps through the same C ABI with
-inputs in pinned host memory (H2D of X and dY, D2H of dA and dB inside the
-timed region).  `--impl reference` times the CPU oracle on a bounded sample of
+`e2e` runs K steps through the same C ABI with
+inputs in pinned host memory: every step copies its X and dY host -> device and
+its dA and dB device -> host inside one timed region, the way a training loop
+feeds the layer -- the next step's inputs are copied on a second stream into a
+second device buffer while the current step computes, the forward starts when
+its X has landed and the backward when its dY has.  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload.  With N > 1 (torchrun) every rank runs an independent
 replica: the layer has no data-path exchange.
 """
@@ -278,31 +281,57 @@ def run_ours(args, rank, world, local_rank):
         for i in range(nb):
             per_kernel[names[nf + i]] += evb[2 * i].elapsed_time(evb[2 * i + 1])
 
-    # ---- end to end through the C ABI with host-resident inputs and outputs
+    # ---- end to end through the C ABI with host-resident inputs and outputs:
+    # double-buffered device inputs, H2D copies on their own stream one step
+    # ahead, D2H of the gradients on the compute stream
     X_pin = torch.from_numpy(synth.bf16_bits(X_h).view(np.int16)).pin_memory()
     dY_pin = torch.from_numpy(synth.bf16_bits(dY_h).view(np.int16)).pin_memory()
     dA_pin = torch.empty((K, r), dtype=torch.float32).pin_memory()
     dB_pin = torch.empty((r, N), dtype=torch.float32).pin_memory()
-    Xv, dYv = X.view(torch.int16), dY.view(torch.int16)
-    e2e_ev = [mk_events(2) for _ in range(args.steps)]
-    for _ in range(max(args.warmup, 1)):
-        Xv.copy_(X_pin, non_blocking=True)
-        dYv.copy_(dY_pin, non_blocking=True)
-        step()
-        dA_pin.copy_(dA, non_blocking=True)
-        dB_pin.copy_(dB, non_blocking=True)
+    Xb = [X, torch.empty_like(X)]
+    dYb = [dY, torch.empty_like(dY)]
+    main_s = torch.cuda.current_stream()
+    copy_s = torch.cuda.Stream()
+
+    def e2e_run(nsteps):
+        evx = [torch.cuda.Event() for _ in range(nsteps)]
+        evy = [torch.cuda.Event() for _ in range(nsteps)]
+        done = [torch.cuda.Event() for _ in range(nsteps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(main_s)
+        copy_s.wait_stream(main_s)
+
+        def h2d(k):
+            b = k % 2
+            with torch.cuda.stream(copy_s):
+                if k >= 2:
+                    copy_s.wait_event(done[k - 2])          # step k-2 has finished with this buffer
+                Xb[b].view(torch.int16).copy_(X_pin, non_blocking=True)
+                evx[k].record(copy_s)
+                dYb[b].view(torch.int16).copy_(dY_pin, non_blocking=True)
+                evy[k].record(copy_s)
+
+        h2d(0)
+        for k in range(nsteps):
+            if k + 1 < nsteps:
+                h2d(k + 1)
+            b = k % 2
+            main_s.wait_event(evx[k])
+            ft.linear_fwd(lay, Xb[b], ws=ws_f, Y=Y, L=L)
+            main_s.wait_event(evy[k])
+            ft.linear_bwd(lay, dYb[b], Xb[b], L, ws=ws_b, dX=dX, dA=dA, dB=dB)
+            dA_pin.copy_(dA, non_blocking=True)
+            dB_pin.copy_(dB, non_blocking=True)
+            done[k].record(main_s)
+        main_s.wait_stream(copy_s)
+        t1.record(main_s)
+        return t0, t1
+
+    e2e_run(max(args.warmup, 1))
     torch.cuda.synchronize()
-    for ev in e2e_ev:
-        flush.zero_()
-        ev[0].record()
-        Xv.copy_(X_pin, non_blocking=True)
-        dYv.copy_(dY_pin, non_blocking=True)
-        step()
-        dA_pin.copy_(dA, non_blocking=True)
-        dB_pin.copy_(dB, non_blocking=True)
-        ev[1].record()
+    t0, t1 = e2e_run(args.steps)
     torch.cuda.synchronize()
-    e2e_ms = sum(ev[0].elapsed_time(ev[1]) for ev in e2e_ev)
+    e2e_ms = t0.elapsed_time(t1)
 
     if world > 1:
         t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
