@@ -188,6 +188,26 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ------------------------------------------------------------------ replicas
+def max_over_ranks(values, device):
+    """Element-wise maximum of a list of floats over all ranks (every rank
+    gets it); identity on one process.  Timing is the slowest replica's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(work_per_step, steps, world, ms):
+    """Whole-job throughput (work units per second) of `world` replicas that
+    each ran `steps` steps of `work_per_step` in `ms` milliseconds (the
+    maximum over ranks): per-GPU work is fixed, so this is weak scaling."""
+    return work_per_step * steps * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ ours (GPU)
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -333,14 +353,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = t0.elapsed_time(t1)
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     fp4, lr = layer_work(M, K, N, r_s, r)
     sec = total_ms / 1e3
-    value = (fp4 + lr) * args.steps * world / sec / 1e12
+    value = job_throughput(fp4 + lr, args.steps, world, total_ms) / 1e12
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     work = kernel_work(M, K, N, r_s, r)
@@ -378,7 +395,7 @@ def run_ours(args, rank, world, local_rank):
         "fp4_tflops": fp4 * args.steps * world / sec / 1e12,
         "fp4_peak_frac": fp4 * args.steps * world / sec / 1e12 / fp4_peak,
         "fp4_peak_tflops": fp4_peak,
-        "e2e": {"value": (fp4 + lr) * args.steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_throughput(fp4 + lr, args.steps, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K + 2 * M * N, "d2h_bytes_per_step": 4 * K * r + 4 * r * N},
         "gpu_launches": args.steps * (nf + nb),
         "kernel_breakdown": "per-kernel times from K separate steps with an event pair around every kernel",
