@@ -398,7 +398,9 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": job_throughput(fp4 + lr, args.steps, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K + 2 * M * N, "d2h_bytes_per_step": 4 * K * r + 4 * r * N},
         "gpu_launches": args.steps * (nf + nb),
-        "kernel_breakdown": "per-kernel times from K separate steps with an event pair around every kernel",
+        "kernel_breakdown": "per-kernel times from K separate steps with an event pair around every kernel; "
+                            "those steps run every kernel on all SMs one after another, the timed steps run "
+                            "dA/dB on a second stream beside the dX GEMM",
         "roofline": roofline,
         "kernels": kern,
         "clocks": clk,

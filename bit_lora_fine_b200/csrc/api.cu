@@ -157,23 +157,47 @@ struct Q16 {
     sf = c.take(ft::sf_mma_bytes(M, C));
   }
 };
-// dA/dB launch of one layer: splits, counters (in the header) and partials
+// dA/dB launch of one layer: splits (serial run on all SMs; side run beside the
+// dX GEMM on side_sms SMs), counters (in the header) and partials
 struct GradPair {
-  MSplit sA, sB;
+  MSplit sA, sB;   // serial
+  MSplit cA, cB;   // beside the dX GEMM
+  int side_sms;
   size_t cntA, cntB;
   size_t partA, partB;
 };
 size_t grad_counter_words(const ft_linear_t* L) { return cdiv(L->K, 128) + cdiv(L->N, 128); }
-// dA reads X from HBM; dB reads G, which the G pass has just streamed through L2,
-// so dA gets two thirds of the SMs
+// SMs given to dA/dB when they run beside the dX GEMM, which then gets the
+// rest: split in proportion to the two kernels' work at the per-SM rates
+// measured on this part when they share the GPU (FP4 GEMM ~14 TFLOP/s, dA/dB
+// ~44 GB/s of X and G per SM -- both are paced per SM by TMA latency, not by
+// the GPU-wide L2 or HBM bandwidth); even, 8 .. half of the SMs.
+int grad_side_sms(const ft_linear_t* L, int64_t M, int num_sms) {
+  const double t_gemm = 2.0 * static_cast<double>(M) * L->N * L->K / 14.0e12;
+  const double t_grad = 2.0 * static_cast<double>(M) * static_cast<double>(L->K + L->N) / 44.0e9;
+  int n = static_cast<int>(std::lround(num_sms * t_grad / (t_grad + t_gemm)));
+  n = std::max(8, std::min(num_sms / 2, n));
+  return n & ~1;
+}
+// Serial: dA reads X from HBM; dB reads G, which the G pass has just streamed
+// through L2, so dA gets two thirds of the SMs.  Side: each planned for the
+// side SMs (one split per 128-row output tile when that fills them).
 void plan_grads(GradPair& g, const ft_linear_t* L, int64_t M, int num_sms) {
   g.sA = m_split(M, L->K, std::max(1, 2 * num_sms / 3));
   g.sB = m_split(M, L->N, std::max(1, num_sms / 3));
+  g.side_sms = grad_side_sms(L, M, num_sms);
+  g.cA = m_split(M, L->K, g.side_sms);
+  g.cB = m_split(M, L->N, g.side_sms);
+}
+size_t split_part_bytes(const MSplit& m, int64_t P) {
+  return m.nsplit > 1 ? static_cast<size_t>(m.nsplit) * cdiv(P, 128) * 128 * 64 * 4 : 0;
+}
+// partials of dA (then dB), large enough for both plans
+size_t grad_part_a(const GradPair& g, const ft_linear_t* L) {
+  return std::max(split_part_bytes(g.sA, L->K), split_part_bytes(g.cA, L->K));
 }
 size_t grad_partial_bytes(const GradPair& g, const ft_linear_t* L) {
-  const size_t a = g.sA.nsplit > 1 ? static_cast<size_t>(g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0;
-  const size_t b = g.sB.nsplit > 1 ? static_cast<size_t>(g.sB.nsplit) * cdiv(L->N, 128) * 128 * 64 * 4 : 0;
-  return a + b;
+  return grad_part_a(g, L) + std::max(split_part_bytes(g.sB, L->N), split_part_bytes(g.cB, L->N));
 }
 
 // Each layout starts with a header of `header` bytes (status word, split
@@ -212,7 +236,7 @@ BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   w.qg.carve(c, M, L->N);
   w.P = c.take(static_cast<size_t>(M * rank_all(L) * 2));
   w.g.partA = c.take(grad_partial_bytes(w.g, L));
-  w.g.partB = w.g.partA + (w.g.sA.nsplit > 1 ? static_cast<size_t>(w.g.sA.nsplit) * cdiv(L->K, 128) * 128 * 64 * 4 : 0);
+  w.g.partB = w.g.partA + grad_part_a(w.g, L);
   w.rp_part = c.take(rp_part_bytes(M, L->N, rank_all(L), 0, num_sms));
   w.total = c.o;
   return w;
@@ -265,8 +289,8 @@ MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
   w.P1 = c.take(static_cast<size_t>(M * rank_all(fc1) * 2));
   const size_t part = c.take(std::max(grad_partial_bytes(w.g2, fc2), grad_partial_bytes(w.g1, fc1)));
   w.g2.partA = w.g1.partA = part;
-  w.g2.partB = part + (w.g2.sA.nsplit > 1 ? static_cast<size_t>(w.g2.sA.nsplit) * cdiv(fc2->K, 128) * 128 * 64 * 4 : 0);
-  w.g1.partB = part + (w.g1.sA.nsplit > 1 ? static_cast<size_t>(w.g1.sA.nsplit) * cdiv(fc1->K, 128) * 128 * 64 * 4 : 0);
+  w.g2.partB = part + grad_part_a(w.g2, fc2);
+  w.g1.partB = part + grad_part_a(w.g1, fc1);
   w.rp_part = c.take(std::max(rp_part_bytes(M, fc2->N, rank_all(fc2), 0, num_sms),
                               rp_part_bytes(M, H, rank_all(fc1), 0, num_sms)));
   w.total = c.o;
@@ -286,10 +310,39 @@ struct Events {
   }
 };
 
+// ---------------------------------------------------------------- side stream
+// The backward runs dA/dB beside the dX GEMM (independent; both paced per SM,
+// so splitting the SMs between them beats running them one after the other).
+// One library-owned non-blocking stream per device carries dA/dB: it waits for
+// the caller's stream at the fork and the caller's stream waits for it at the
+// join, so the call keeps single-stream semantics for the caller.  The enqueue
+// of fork .. join is serialised by a lock so that concurrent callers cannot
+// interleave their event records.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+int side_stream(SideStream** out) {
+  static SideStream ss[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FT_ERR_UNSUPPORTED;
+  SideStream& x = ss[dev];
+  if (!x.s) {
+    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
+      return FT_ERR_CUDA;
+  }
+  *out = &x;
+  return FT_OK;
+}
+
 // ---------------------------------------------------------------- launch helpers
 // Fused row pass over X [M, K] bf16: Q(X) -> (codes, scales), L = bf16(X W)
 // with W = D [K, R] (w_mn) or W^T [R, K]; gelu: the input is h and the pass
-// quantizes GELU(h).  Split reduction inside a cluster: needs only the status word.
+// quantizes GELU(h).
 int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
                 float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
                 int* status, int num_sms, cudaStream_t s) {
@@ -364,8 +417,10 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
 
 // dA = T_A^T V_A[:, r_s:] ([K, r]) and dB = (L[:, r_s:]^T G) ([r, N]) of one layer, one launch
 int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, const void* G, const void* Lsaved,
-              float* dA, float* dB, bool accumulate, const GradPair& g, uint8_t* base, int* status,
+              float* dA, float* dB, bool accumulate, const GradPair& g, bool side, uint8_t* base, int* status,
               cudaStream_t s) {
+  const MSplit& sa = side ? g.cA : g.sA;
+  const MSplit& sb = side ? g.cB : g.sB;
   const int64_t R = rank_all(L);
   CUtensorMap tmTa, tmVa, tmTb, tmVb;
   if (!map_bf16(&tmTa, X, L->K, M, 128) || !map_bf16(&tmVa, P, R, M, 128) || !map_bf16(&tmTb, G, L->N, M, 128) ||
@@ -378,16 +433,16 @@ int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, con
   ta.accumulate = tb.accumulate = accumulate ? 1 : 0;
   ta.status = tb.status = status;
   ta.P = static_cast<int>(L->K);
-  ta.mt_per_split = g.sA.mt_per_split;
-  ta.nsplit = g.sA.nsplit;
+  ta.mt_per_split = sa.mt_per_split;
+  ta.nsplit = sa.nsplit;
   ta.out = dA;
   ta.out_sp = L->r;
   ta.out_sj = 1;
   ta.part = reinterpret_cast<float*>(base + g.partA);
   ta.counters = reinterpret_cast<int*>(base + g.cntA);
   tb.P = static_cast<int>(L->N);
-  tb.mt_per_split = g.sB.mt_per_split;
-  tb.nsplit = g.sB.nsplit;
+  tb.mt_per_split = sb.mt_per_split;
+  tb.nsplit = sb.nsplit;
   tb.out = dB;
   tb.out_sp = 1;
   tb.out_sj = L->N;
@@ -403,6 +458,26 @@ int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, con
     if (rc_ != FT_OK) return rc_;                                \
     if (evs.mark((k), 1, s) != cudaSuccess) return FT_ERR_CUDA;  \
   } while (0)
+
+// The dX GEMM on the caller's stream, on all but gp.side_sms SMs, and dA/dB
+// beside it on the side stream (fork before, join after: see SideStream).  The
+// GEMM is launched first so that its persistent CTAs take their SMs as the
+// previous kernel leaves them; dA/dB fill the rest.
+int gemm_and_grads_side(const GemmArgs& g, const ft_linear_t* L, int64_t M, const void* X, const void* P,
+                        const void* G, const void* Lsaved, float* dA, float* dB, bool accumulate, const GradPair& gp,
+                        uint8_t* base, int* status, int num_sms, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  int st = side_stream(&ss);
+  if (st) return st;
+  if (cudaEventRecord(ss->fork, s) != cudaSuccess) return FT_ERR_CUDA;
+  if ((st = run_gemm(g, status, num_sms - gp.side_sms, s))) return st;
+  if (cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess) return FT_ERR_CUDA;
+  if ((st = run_grads(L, M, X, P, G, Lsaved, dA, dB, accumulate, gp, true, base, status, ss->s))) return st;
+  if (cudaEventRecord(ss->join, ss->s) != cudaSuccess || cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+    return FT_ERR_CUDA;
+  return FT_OK;
+}
 
 }  // namespace
 
@@ -602,10 +677,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P,
                         reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                         di.num_sms, s));
-  // dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G -- right after the G pass, while G
-  // (just streamed by it) is still in L2
-  FT_TRY(1, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, s));
-  // dX = deq(Q(G)) deq(Q(R)) + P D^T
+  // dX = deq(Q(G)) deq(Q(R)) + P D^T, and dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G
   GemmArgs g{};
   g.M = M;
   g.N = K;
@@ -620,7 +692,16 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   g.B2 = layer->D;
   g.out = dX;
   g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(2, run_gemm(g, status, di.num_sms, s));
+  if (evs.ev) {
+    // timed: one after the other (dA/dB first, while G is still in L2), so that
+    // every kernel has its own event pair
+    FT_TRY(1, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, false, base, status, s));
+    FT_TRY(2, run_gemm(g, status, di.num_sms, s));
+  } else {
+    st = gemm_and_grads_side(g, layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status,
+                             di.num_sms, s);
+    if (st) return st;
+  }
   return FT_OK;
 }
 
@@ -786,13 +867,12 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g.out2 = abf;
   FT_TRY(1, run_gemm(g, status, di.num_sms, s));
   // FC2 adapter gradients on bf16(GELU(h)) and G
-  FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, base, status, s));
+  FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, false, base, status, s));
   // FC1 backward on d_h: G pass, dX GEMM, adapter gradients
   FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales,
                         base + w.qdh.sf, P1, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
-  // FC1 adapter gradients while d_h (just streamed by the d_h pass) is in L2
-  FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status, s));
+  // FC1 dX GEMM and adapter gradients
   GemmArgs g1{};
   g1.M = M;
   g1.N = K1;
@@ -807,7 +887,14 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g1.B2 = fc1->D;
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
+  if (evs.ev) {
+    FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
+    FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
+  } else {
+    st = gemm_and_grads_side(g1, fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status,
+                             di.num_sms, s);
+    if (st) return st;
+  }
   return FT_OK;
 }
 

@@ -149,7 +149,13 @@ FT_API int fourtune_linear_fwd(const ft_linear_t* layer, const ft_bf16* X, int64
  *   dX [M, K] = deq(Q(G)) deq(Q(R)) + P D^T   (dx_dtype F32 or BF16)
  *   dA [K, r] fp32 = X^T P[:, r_s:]     dB [r, N] fp32 = L[:, r_s:]^T G
  * with P = bf16(G U^T).  accumulate = 1 adds into dA and dB, 0
- * overwrites.  R, S and bias receive no gradient. */
+ * overwrites.  R, S and bias receive no gradient.
+ * Streams: after the G pass, dA and dB run on a library-owned stream (one per
+ * device, created on first use) beside the dX GEMM, which gets the other SMs;
+ * that stream waits for `stream` first and `stream` waits for it before the
+ * call returns, so all work of the call is ordered on `stream` as seen by the
+ * caller.  Calls from several host threads are safe; their dA/dB share the
+ * library stream (so they run one after another there). */
 FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, const ft_bf16* X, const ft_bf16* L_saved,
                         int64_t M, void* dX, int dx_dtype, float* dA, float* dB, int accumulate, void* ws,
                         size_t ws_bytes, void* stream);
@@ -159,7 +165,9 @@ FT_API int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, cons
  * after kernel k (NULL entries and k >= n_events/2 are skipped).  Kernels, in
  * order -- forward: 0 fused X pass (quantize + X D), 1 FP4 GEMM with
  * up-projection; backward: 0 fused G pass (quantize + G U^T), 1 dA and dB (run
- * while G is still in L2), 2 FP4 dX GEMM.  Used for live per-kernel timing. */
+ * while G is still in L2), 2 FP4 dX GEMM.  With events every kernel runs on
+ * `stream` on all SMs, one after another (no library stream).  Used for live
+ * per-kernel timing. */
 FT_API int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
                                      ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
@@ -186,7 +194,8 @@ FT_API int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
  * d_h = bf16(d_a * GELU'(h)) and bf16(GELU(h)) into the workspace; FC2's dA2
  * uses the latter, FC1's backward takes d_h as its incoming gradient (all
  * three branches).  Writes dX [M, K1] and the four adapter gradients (fp32;
- * accumulate = 1 adds). */
+ * accumulate = 1 adds).  FC1's dA1/dB1 run beside FC1's dX GEMM on the library
+ * stream, as in fourtune_linear_bwd. */
 FT_API size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
 FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY, const ft_bf16* X,
                             const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
