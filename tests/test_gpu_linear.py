@@ -203,3 +203,31 @@ def test_config_flux_single_stream_linears(cuda_lib, layer):
     X = synth.layer_input(wl, layer=layer)
     dY = synth.upstream_grad(wl, layer=layer)
     run_sampled(cuda_lib, p, X, dY, _sample_rows(wl.M, seed=layer))
+
+
+def test_timed_and_untimed_backward_agree(cuda_lib):
+    """The plain backward runs dA/dB beside the dX GEMM (other M splits, the GEMM
+    on fewer SMs); the timed one runs them one after the other on all SMs.  dX
+    is the same product tile by tile: bit-identical.  dA and dB are the same fp32
+    sums grouped differently over M: equal to fp32 rounding, and both match the
+    oracle."""
+    import torch
+    M, K, N = 1024, 768, 768
+    p = random_layer(K, N, 32, 32, seed=7, bias=False, M=M)
+    lay = _device_layer(cuda_lib, p)
+    Xd, dYd = to_dev_bf16(p["X"]), to_dev_bf16(p["dY"])
+    Y, L, _ = cuda_lib.linear_fwd(lay, Xd, torch.float32)
+    dX1, dA1, dB1, ws1 = cuda_lib.linear_bwd(lay, dYd, Xd, L, torch.float32)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    dX2, dA2, dB2, ws2 = cuda_lib.linear_bwd(lay, dYd, Xd, L, torch.float32, events=ev)
+    torch.cuda.synchronize()
+    cuda_lib.device_status(ws1)
+    cuda_lib.device_status(ws2)
+    np.testing.assert_array_equal(to_host(dX1), to_host(dX2))
+    for a, b in ((dA1, dA2), (dB1, dB2)):
+        a, b = to_host(a), to_host(b)
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-5 * np.abs(b).max())
+    R_codes, R_scales = block16.quantize(p["R"])
+    ref = olayer.linear_bwd(p["dY"], p["X"], to_host(L), R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"])
+    assert normwise(to_host(dA1), ref["dA"]) <= TOL
+    assert normwise(to_host(dB1), ref["dB"]) <= TOL
