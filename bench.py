@@ -397,7 +397,7 @@ def run_ours(args, rank, world, local_rank):
         "fp4_peak_tflops": fp4_peak,
         "e2e": {"value": job_throughput(fp4 + lr, args.steps, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K + 2 * M * N, "d2h_bytes_per_step": 4 * K * r + 4 * r * N},
-        "gpu_launches": args.steps * (nf + nb),
+        "gpu_launches": args.steps * (nf + nb + 2),   # + each call's workspace-header clear
         "kernel_breakdown": "per-kernel times from K separate steps with an event pair around every kernel; "
                             "those steps run every kernel on all SMs one after another, the timed steps run "
                             "dA/dB on a second stream beside the dX GEMM",

@@ -610,7 +610,7 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(base);
-  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   uint8_t* qc = base + w.qx.codes;
   uint8_t* qs = base + w.qx.scales;
@@ -667,7 +667,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(base);
-  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   uint8_t* gc = base + w.qg.codes;
   uint8_t* gs = base + w.qg.scales;
@@ -765,7 +765,7 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(base);
-  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   // FC1: X pass, then 4-bit GEMM + L1 U1 + b1 -> h (bf16, saved)
   FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
@@ -839,7 +839,7 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(base);
-  if (cudaMemsetAsync(base, 0, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   void* P2 = base + w.P2;
   void* dh = base + w.dh;
@@ -918,7 +918,7 @@ int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(scratch);
   // status word and split counters must start at zero; the array keeps what the last call left
-  if (cudaMemsetAsync(base, 0, header, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_clear_words(base, header, s) != cudaSuccess) return FT_ERR_CUDA;
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128) || !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
   RowpassParams rp{};

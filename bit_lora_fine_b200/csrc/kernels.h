@@ -88,6 +88,9 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
 // compact block16 scales -> MMA-ready layout of the operand [rows, cols]; with
 // `transposed`, the operand is the transpose of the quantized matrix, whose
 // compact scales are [cols/16, rows/16]
+// zero `bytes` (a multiple of 16, 16-aligned) at p after the previous kernel, in a
+// dependent launch (see quant.cu)
+cudaError_t launch_clear_words(void* p, size_t bytes, cudaStream_t stream);
 cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
                           cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,

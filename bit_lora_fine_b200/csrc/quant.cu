@@ -9,6 +9,9 @@
 // every code is +0, else code = E2M1(t / dec(sc)) (fp32 division, round to
 // nearest even, saturate at +-6, sign kept).  Codes: even column in the low
 // nibble of byte [row, col/2]; scales: one byte per block, [rows/16, cols/16].
+// Also: the workspace-header clear that every API call launches first.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -213,6 +216,27 @@ __global__ void sf_mma_kernel(const uint8_t* __restrict__ scales, int rows, int 
     v = transposed ? scales[static_cast<long long>(g) * (rows / 16) + rb] : scales[rb * (cols / 16) + g];
   }
   out[i] = v;
+}
+
+// Zero n16 16-byte words at p (a workspace header: status word, split
+// counters), in stream order: launched with programmatic dependent launch, it
+// releases the next kernel at once (whose prologue then overlaps) and waits for
+// the previous grid before it writes.  A memset in its place would end the
+// chain of dependent launches between the previous kernel and the next.
+__global__ void clear_words_kernel(uint4* __restrict__ p, int n16) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  for (int i = threadIdx.x + blockIdx.x * blockDim.x; i < n16; i += blockDim.x * gridDim.x)
+    p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+cudaError_t launch_clear_words(void* p, size_t bytes, cudaStream_t stream) {
+  if (bytes == 0) return cudaSuccess;
+  if ((bytes % 16) || (reinterpret_cast<uintptr_t>(p) % 16)) return cudaErrorInvalidValue;
+  const long long n16 = static_cast<long long>(bytes / 16);
+  const int blocks = static_cast<int>(std::min<long long>((n16 + 255) / 256, 64));
+  return launch_pdl(clear_words_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<uint4*>(p),
+                    static_cast<int>(n16));
 }
 
 cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
