@@ -171,8 +171,10 @@ size_t grad_counter_words(const ft_linear_t* L) { return cdiv(L->K, 128) + cdiv(
 // rest: split in proportion to the two kernels' work at the per-SM rates
 // measured on this part when they share the GPU (FP4 GEMM ~14 TFLOP/s, dA/dB
 // ~44 GB/s of X and G per SM -- both are paced per SM by TMA latency, not by
-// the GPU-wide L2 or HBM bandwidth); even, 8 .. half of the SMs.
+// the GPU-wide L2 or HBM bandwidth); even, 8 .. half of the SMs.  0 (run them
+// one after the other) on parts with fewer than 16 SMs.
 int grad_side_sms(const ft_linear_t* L, int64_t M, int num_sms) {
+  if (num_sms < 16) return 0;
   const double t_gemm = 2.0 * static_cast<double>(M) * L->N * L->K / 14.0e12;
   const double t_grad = 2.0 * static_cast<double>(M) * static_cast<double>(L->K + L->N) / 44.0e9;
   int n = static_cast<int>(std::lround(num_sms * t_grad / (t_grad + t_gemm)));
@@ -186,8 +188,8 @@ void plan_grads(GradPair& g, const ft_linear_t* L, int64_t M, int num_sms) {
   g.sA = m_split(M, L->K, std::max(1, 2 * num_sms / 3));
   g.sB = m_split(M, L->N, std::max(1, num_sms / 3));
   g.side_sms = grad_side_sms(L, M, num_sms);
-  g.cA = m_split(M, L->K, g.side_sms);
-  g.cB = m_split(M, L->N, g.side_sms);
+  g.cA = m_split(M, L->K, std::max(1, g.side_sms));
+  g.cB = m_split(M, L->N, std::max(1, g.side_sms));
 }
 size_t split_part_bytes(const MSplit& m, int64_t P) {
   return m.nsplit > 1 ? static_cast<size_t>(m.nsplit) * cdiv(P, 128) * 128 * 64 * 4 : 0;
@@ -692,9 +694,9 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   g.B2 = layer->D;
   g.out = dX;
   g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  if (evs.ev) {
-    // timed: one after the other (dA/dB first, while G is still in L2), so that
-    // every kernel has its own event pair
+  if (evs.ev || w.g.side_sms == 0) {
+    // timed (or a small part): one after the other (dA/dB first, while G is
+    // still in L2), so that every kernel has its own event pair
     FT_TRY(1, run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, false, base, status, s));
     FT_TRY(2, run_gemm(g, status, di.num_sms, s));
   } else {
@@ -887,7 +889,7 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g1.B2 = fc1->D;
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
-  if (evs.ev) {
+  if (evs.ev || w.g1.side_sms == 0) {
     FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
     FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
   } else {
