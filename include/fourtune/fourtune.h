@@ -59,7 +59,7 @@ enum {
   FT_ERR_WORKSPACE = -4,   /* ws_bytes smaller than the *_workspace_size() value */
   FT_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed */
   FT_ERR_TIMEOUT = -6,     /* a kernel's bounded wait expired (device status) */
-  FT_ERR_UNSUPPORTED = -7  /* not an sm_100 device, or a size this build does not handle */
+  FT_ERR_UNSUPPORTED = -7  /* not an sm_100 device, or a size the library does not handle */
 };
 
 enum { FT_DTYPE_F32 = 0, FT_DTYPE_BF16 = 1 };
