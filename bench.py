@@ -11,7 +11,8 @@ rank 32, LoRA rank 32, seeded synthetic bf16 data (synth.py).
 Prints one JSON line (rank 0).  `value` is device time from CUDA events summed
 over exactly K steps (L2 flushed before each step, outside the events, by a
 256 MB write followed by a 256 MB read of another buffer), max over ranks, with
-no event between the kernels of a step; K further steps with an event pair
+no event between the kernels of a step; that block of K steps is repeated back
+to back for ~0.4 s (the clock sampler's window) and the median block counts; K further steps with an event pair
 around every kernel give the per-kernel times (`kernels`, `roofline`);
 `e2e` runs K steps through the same C ABI with
 inputs in pinned host memory: every step copies its X and dY host -> device and
@@ -41,6 +42,7 @@ METRIC = "W4A4G4 linear fwd+bwd TFLOPS & tokens/s on 1 B200; % of dense FP4 peak
 FALLBACK = dict(hbm_gbs=6650.0, bf16_tflops=1590.0)
 FP4_PER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
 ORACLE_ROWS = 256           # rows of the workload per CPU-oracle sample
+CLOCK_WINDOW_S = 0.4        # repeats of the timed block fill about this long (clock record)
 
 
 def layer_work(M, K, N, r_s, r):
@@ -83,9 +85,10 @@ _REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_
 
 
 class ClockSampler:
-    """Reads SM clock and clock-event reasons through NVML every ~10 ms (read-only)."""
+    """Reads SM clock and clock-event reasons through NVML every ~2 ms (read-only)."""
 
-    def __init__(self, index):
+    def __init__(self, index, period=0.002):
+        self.period = period
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self._stop = threading.Event()
         self._thread = None
@@ -106,7 +109,7 @@ class ClockSampler:
                 self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(self.period)
 
     def start(self):
         if self._nv:
@@ -258,34 +261,43 @@ def run_ours(args, rank, world, local_rank):
         ft.linear_fwd(lay, X, ws=ws_f, Y=Y, L=L, events=evf)
         ft.linear_bwd(lay, dY, X, L, ws=ws_b, dX=dX, dA=dA, dB=dB, events=evb)
 
+    torch.cuda.synchronize()
+    t_w = time.perf_counter()
     for _ in range(max(args.warmup, 1)):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    wall_per_step = (time.perf_counter() - t_w) / max(args.warmup, 1)
     ft.device_status(ws_f)
     ft.device_status(ws_b)
 
     # timed region: K steps with no event between the kernels of a step (the
-    # kernels chain through programmatic dependent launch); then K more steps
-    # with an event pair around every kernel, for the per-kernel breakdown
-    steps = [mk_events(2) for _ in range(args.steps)]
+    # kernels chain through programmatic dependent launch), timed as one block
+    # between a barrier and a synchronize on both sides.  The block is repeated
+    # back to back (the same K steps each time) for ~0.4 s so that the clock
+    # sampler sees the GPU under load; the value is the median block.  Then K
+    # more steps with an event pair around every kernel, for the breakdown.
+    reps = int(min(100, max(3, np.ceil(CLOCK_WINDOW_S / max(args.steps * wall_per_step, 1e-6)))))
+    blocks = [[mk_events(2) for _ in range(args.steps)] for _ in range(reps)]
     ksteps = [(mk_events(2 * nf), mk_events(2 * nb)) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    for se in steps:
-        flush.zero_()
-        se[0].record()
-        step()
-        se[1].record()
+    for steps in blocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for se in steps:
+            flush.zero_()
+            se[0].record()
+            step()
+            se[1].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    block_ms = [sum(se[0].elapsed_time(se[1]) for se in steps) for steps in blocks]
     for evf, evb in ksteps:
         flush.zero_()
         step(evf, evb)
@@ -293,7 +305,7 @@ def run_ours(args, rank, world, local_rank):
     ft.device_status(ws_f)
     ft.device_status(ws_b)
 
-    total_ms = sum(se[0].elapsed_time(se[1]) for se in steps)
+    total_ms = float(statistics.median(block_ms))
     per_kernel = {n: 0.0 for n in names}
     for evf, evb in ksteps:
         for i in range(nf):
@@ -404,6 +416,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "kernels": kern,
         "clocks": clk,
+        "timed_blocks": {"repeats": reps, "steps_each": args.steps, "median_ms": total_ms,
+                         "min_ms": min(block_ms), "max_ms": max(block_ms),
+                         "note": "value = the median of back-to-back timed blocks of exactly K steps"},
     }
     if world == 1 and not args.no_extra:
         line["configs_extra"] = measure_extra(ft, synth, dev, flush, peaks, steps=max(3, min(args.steps, 10)),

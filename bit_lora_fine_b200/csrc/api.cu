@@ -5,8 +5,18 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fourtune/fourtune.h"
 #include "kernels.h"
+
+// One NVTX range around each entry point (visible in timeline profilers; costs
+// nothing when no tool is attached).
+struct FtRange {
+  explicit FtRange(const char* name) { nvtxRangePushA(name); }
+  ~FtRange() { nvtxRangePop(); }
+};
+#define FT_RANGE(name) const FtRange ft_range_(name)
 
 namespace {
 
@@ -369,6 +379,7 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.part = part;
   rp.counters = counters;
   rp.status = status;
+  rp.fault_skip_stage = -1;
   return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
 
@@ -481,6 +492,51 @@ int gemm_and_grads_side(const GemmArgs& g, const ft_linear_t* L, int64_t M, cons
   return FT_OK;
 }
 
+size_t kmajor_rowpass_scratch(int64_t M, int64_t K, int64_t R, int num_sms, size_t* header) {
+  const RowSplit rs = row_split(M, K, R, 0, num_sms, kRowMaxSplit);
+  *header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
+  return *header + (rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * M * R * 4 : 0);
+}
+int check_quant_down(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R, uint8_t* codes,
+                     uint8_t* scales, ft_bf16* L) {
+  if (!X || !W || !codes || !scales || !L) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || M % 16 || K % 32) return FT_ERR_SHAPE;
+  if (R < 16 || R % 16 || R > 128 || M > (1 << 30) || K > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(X) || !al16(W) || !al16(codes) || !al16(L)) return FT_ERR_ALIGN;
+  return FT_OK;
+}
+int launch_kmajor_rowpass(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R, uint8_t* codes,
+                          uint8_t* scales, ft_bf16* L, uint8_t* base, size_t header, int num_sms, int fault_skip_stage,
+                          unsigned long long wait_ns, cudaStream_t s) {
+  const RowSplit rs = row_split(M, K, R, 0, num_sms, kRowMaxSplit);
+  // status word and split counters must start at zero
+  if (ft::launch_clear_words(base, header, s) != cudaSuccess) return FT_ERR_CUDA;
+  CUtensorMap tmX, tmW;
+  if (!map_bf16(&tmX, X, K, M, 128) || !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
+  RowpassParams rp{};
+  rp.M = static_cast<int>(M);
+  rp.K = static_cast<int>(K);
+  rp.R = static_cast<int>(R);
+  rp.w_mn_major = 0;
+  rp.kt_per_split = rs.kt_per_split;
+  rp.nsplit = rs.nsplit;
+  rp.stages = rs.stages;
+  rp.codes = codes;
+  rp.scales = scales;
+  rp.L = L;
+  rp.part = reinterpret_cast<float*>(base + header);
+  rp.counters = reinterpret_cast<int*>(base + 16);
+  rp.status = reinterpret_cast<int*>(base);
+  rp.wait_ns = wait_ns;
+  rp.fault_skip_stage = fault_skip_stage;
+  return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
+}
+int read_status_word(const void* dev_word, cudaStream_t s) {
+  int h = 0;
+  if (cudaMemcpyAsync(&h, dev_word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FT_ERR_CUDA;
+  return h == 0 ? FT_OK : FT_ERR_TIMEOUT;
+}
 }  // namespace
 
 extern "C" {
@@ -501,6 +557,7 @@ const char* fourtune_error_string(int code) {
 
 int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
                               uint8_t* scales, uint8_t* codes_t, void* stream) {
+  FT_RANGE("fourtune_quantize_block16");
   if (!x || !codes || !scales) return FT_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols || ld % 8) return FT_ERR_SHAPE;
   if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
@@ -518,6 +575,7 @@ int fourtune_quantize_block16(const ft_bf16* x, int64_t rows, int64_t cols, int6
 
 int fourtune_quantize_block16_f32(const float* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
                                   uint8_t* scales, void* stream) {
+  FT_RANGE("fourtune_quantize_block16_f32");
   if (!x || !codes || !scales) return FT_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols || ld % 4) return FT_ERR_SHAPE;
   if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
@@ -530,6 +588,7 @@ int fourtune_quantize_block16_f32(const float* x, int64_t rows, int64_t cols, in
 }
 
 int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, uint8_t* codes_t, void* stream) {
+  FT_RANGE("fourtune_transpose_codes");
   if (!codes || !codes_t) return FT_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return FT_ERR_SHAPE;
   if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
@@ -541,12 +600,14 @@ int fourtune_transpose_codes(const uint8_t* codes, int64_t rows, int64_t cols, u
 }
 
 size_t fourtune_mma_scales_size(int64_t rows, int64_t cols) {
+  FT_RANGE("fourtune_mma_scales_size");
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || rows > (1 << 30) || cols > (1 << 30)) return 0;
   return ft::sf_mma_bytes(rows, cols);
 }
 
 int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int transposed, uint8_t* out,
                         void* stream) {
+  FT_RANGE("fourtune_mma_scales");
   if (!scales || !out || (transposed != 0 && transposed != 1)) return FT_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return FT_ERR_SHAPE;
   if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
@@ -560,16 +621,19 @@ int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int t
 
 // ---------------------------------------------------------------- linear
 size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_fwd_workspace_size");
   if (check_layer(layer, false) || M <= 0 || M % 16) return 0;
   return fwd_layout(layer, M, num_sms_or_default()).total;
 }
 
 size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_bwd_workspace_size");
   if (check_layer(layer, true) || M <= 0 || M % 16) return 0;
   return bwd_layout(layer, M, num_sms_or_default()).total;
 }
 
 int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off) {
+  FT_RANGE("fourtune_linear_fwd_ws_offsets");
   int st = check_layer(layer, false);
   if (st) return st;
   const FwdWs w = fwd_layout(layer, M, num_sms_or_default());
@@ -580,6 +644,7 @@ int fourtune_linear_fwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* 
 
 int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* codes_off, size_t* scales_off,
                                    size_t* P_off) {
+  FT_RANGE("fourtune_linear_bwd_ws_offsets");
   int st = check_layer(layer, true);
   if (st) return st;
   const BwdWs w = bwd_layout(layer, M, num_sms_or_default());
@@ -591,12 +656,14 @@ int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, size_t* 
 
 int fourtune_linear_fwd(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
                         ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_fwd");
   return fourtune_linear_fwd_timed(layer, X, M, Y, y_dtype, L_saved, ws, ws_bytes, stream, nullptr, 0);
 }
 
 int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
                               ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream, void* const* events,
                               int n_events) {
+  FT_RANGE("fourtune_linear_fwd_timed");
   const Events evs{events, n_events};
   int st = check_layer(layer, false);
   if (st) return st;
@@ -644,6 +711,7 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
 int fourtune_linear_bwd(const ft_linear_t* layer, const ft_bf16* dY, const ft_bf16* X, const ft_bf16* L_saved,
                         int64_t M, void* dX, int dx_dtype, float* dA, float* dB, int accumulate, void* ws,
                         size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_bwd");
   return fourtune_linear_bwd_timed(layer, dY, X, L_saved, M, dX, dx_dtype, dA, dB, accumulate, ws, ws_bytes, stream,
                                    nullptr, 0);
 }
@@ -652,6 +720,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
                               const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA, float* dB,
                               int accumulate, void* ws, size_t ws_bytes, void* stream, void* const* events,
                               int n_events) {
+  FT_RANGE("fourtune_linear_bwd_timed");
   const Events evs{events, n_events};
   int st = check_layer(layer, true);
   if (st) return st;
@@ -709,17 +778,20 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
 
 // ---------------------------------------------------------------- MLP
 size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
+  FT_RANGE("fourtune_mlp_fwd_workspace_size");
   if (check_mlp(fc1, fc2, false) || M <= 0 || M % 16) return 0;
   return mlp_fwd_layout(fc1, fc2, M, num_sms_or_default()).total;
 }
 
 size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M) {
+  FT_RANGE("fourtune_mlp_bwd_workspace_size");
   if (check_mlp(fc1, fc2, true) || M <= 0 || M % 16) return 0;
   return mlp_bwd_layout(fc1, fc2, M, num_sms_or_default()).total;
 }
 
 int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* qa_codes,
                                 size_t* qa_scales) {
+  FT_RANGE("fourtune_mlp_fwd_ws_offsets");
   int st = check_mlp(fc1, fc2, false);
   if (st) return st;
   const MlpFwdWs w = mlp_fwd_layout(fc1, fc2, M, num_sms_or_default());
@@ -730,6 +802,7 @@ int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, 
 
 int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* dh_off,
                                 size_t* a_off, size_t* qdh_codes, size_t* qdh_scales) {
+  FT_RANGE("fourtune_mlp_bwd_ws_offsets");
   int st = check_mlp(fc1, fc2, true);
   if (st) return st;
   const MlpBwdWs w = mlp_bwd_layout(fc1, fc2, M, num_sms_or_default());
@@ -743,6 +816,7 @@ int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, 
 int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
                      int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a, void* ws,
                      size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_mlp_fwd");
   return fourtune_mlp_fwd_timed(fc1, fc2, X, M, Y, y_dtype, h_saved, L1_saved, L2_saved, dbg_a, ws, ws_bytes, stream,
                                 nullptr, 0);
 }
@@ -750,6 +824,7 @@ int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
 int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
                            int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a,
                            void* ws, size_t ws_bytes, void* stream, void* const* events, int n_events) {
+  FT_RANGE("fourtune_mlp_fwd_timed");
   const Events evs{events, n_events};
   int st = check_mlp(fc1, fc2, false);
   if (st) return st;
@@ -815,6 +890,7 @@ int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf
                      const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M, void* dX,
                      int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate, void* ws,
                      size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_mlp_bwd");
   return fourtune_mlp_bwd_timed(fc1, fc2, dY, X, h_saved, L1_saved, L2_saved, M, dX, dx_dtype, dA1, dB1, dA2, dB2,
                                 accumulate, ws, ws_bytes, stream, nullptr, 0);
 }
@@ -823,6 +899,7 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
                            const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
                            void* dX, int dx_dtype, float* dA1, float* dB1, float* dA2, float* dB2, int accumulate,
                            void* ws, size_t ws_bytes, void* stream, void* const* events, int n_events) {
+  FT_RANGE("fourtune_mlp_bwd_timed");
   const Events evs{events, n_events};
   int st = check_mlp(fc1, fc2, true);
   if (st) return st;
@@ -901,52 +978,54 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
 }
 
 // ---------------------------------------------------------------- static-scratch row pass
+// Row pass over X [M, K] with W^T [R, K] read K-major, its split bookkeeping at
+// `base` (status word, split counters, then partials); `fault_skip_stage` and
+// `wait_ns` are the test hook of fourtune_test_wait_timeout (-1 and 0 otherwise).
+
 int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
                                uint8_t* codes, uint8_t* scales, ft_bf16* L, void* stream) {
-  if (!X || !W || !codes || !scales || !L) return FT_ERR_INVALID_ARG;
-  if (M <= 0 || K <= 0 || M % 16 || K % 32) return FT_ERR_SHAPE;
-  if (R < 16 || R % 16 || R > 128 || M > (1 << 30) || K > (1 << 30)) return FT_ERR_UNSUPPORTED;
-  if (!al16(X) || !al16(W) || !al16(codes) || !al16(L)) return FT_ERR_ALIGN;
-  DevInfo di;
-  int st = device_info(&di);
+  FT_RANGE("fourtune_quant_down_static");
+  int st = check_quant_down(X, M, K, W, R, codes, scales, L);
   if (st) return st;
-  // W^T [R, K] read K-major; split partials in the library's static array
-  const RowSplit rs = row_split(M, K, R, 0, di.num_sms, 1 << 20);
-  const size_t header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128)));
-  const size_t need = header + (rs.nsplit > 1 ? static_cast<size_t>(rs.nsplit) * M * R * 4 : 0);
-  if (need > ft::kRowpassStaticScratchBytes) return FT_ERR_WORKSPACE;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  // split partials in the library's static array
+  size_t header = 0;
+  if (kmajor_rowpass_scratch(M, K, R, di.num_sms, &header) > ft::kRowpassStaticScratchBytes) return FT_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (ft::rowpass_static_scratch(&scratch) != cudaSuccess) return FT_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(scratch);
-  // status word and split counters must start at zero; the array keeps what the last call left
-  if (ft::launch_clear_words(base, header, s) != cudaSuccess) return FT_ERR_CUDA;
-  CUtensorMap tmX, tmW;
-  if (!map_bf16(&tmX, X, K, M, 128) || !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
-  RowpassParams rp{};
-  rp.M = static_cast<int>(M);
-  rp.K = static_cast<int>(K);
-  rp.R = static_cast<int>(R);
-  rp.w_mn_major = 0;
-  rp.kt_per_split = rs.kt_per_split;
-  rp.nsplit = rs.nsplit;
-  rp.stages = rs.stages;
-  rp.codes = codes;
-  rp.scales = scales;
-  rp.L = L;
-  rp.part = reinterpret_cast<float*>(base + header);
-  rp.counters = reinterpret_cast<int*>(base + 16);
-  rp.status = reinterpret_cast<int*>(base);
-  return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
+  return launch_kmajor_rowpass(X, M, K, W, R, codes, scales, L, static_cast<uint8_t*>(scratch), header, di.num_sms, -1,
+                               0, static_cast<cudaStream_t>(stream));
+}
+
+int fourtune_quant_down_static_status(void* stream) {
+  FT_RANGE("fourtune_quant_down_static_status");
+  void* scratch = nullptr;
+  if (ft::rowpass_static_scratch(&scratch) != cudaSuccess) return FT_ERR_CUDA;
+  return read_status_word(scratch, static_cast<cudaStream_t>(stream));
+}
+
+int fourtune_test_wait_timeout(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R, uint8_t* codes,
+                               uint8_t* scales, ft_bf16* L, void* ws, size_t ws_bytes, int64_t wait_ns,
+                               void* stream) {
+  FT_RANGE("fourtune_test_wait_timeout");
+  int st = check_quant_down(X, M, K, W, R, codes, scales, L);
+  if (st) return st;
+  if (!ws) return FT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FT_ERR_ALIGN;
+  if (wait_ns < 1000000 || wait_ns > 1000000000) return FT_ERR_INVALID_ARG;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  size_t header = 0;
+  if (kmajor_rowpass_scratch(M, K, R, di.num_sms, &header) > ws_bytes) return FT_ERR_WORKSPACE;
+  return launch_kmajor_rowpass(X, M, K, W, R, codes, scales, L, static_cast<uint8_t*>(ws), header, di.num_sms, 0,
+                               static_cast<unsigned long long>(wait_ns), static_cast<cudaStream_t>(stream));
 }
 
 int fourtune_device_status(const void* ws, void* stream) {
+  FT_RANGE("fourtune_device_status");
   if (!ws) return FT_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int h = 0;
-  if (cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FT_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return FT_ERR_CUDA;
-  return h == 0 ? FT_OK : FT_ERR_TIMEOUT;
+  return read_status_word(ws, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

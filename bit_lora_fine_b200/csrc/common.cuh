@@ -55,16 +55,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of `bar` with the given parity.  Returns false if
-// the CTA was aborted or the wait expired (then status/abort are set).
+// the CTA was aborted or the wait expired after `limit_ns` (then status/abort
+// are set).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t n = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++n & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) atomicCAS(status, 0, kDevTimeout);
         return false;
@@ -347,10 +348,14 @@ __device__ __forceinline__ float snap19(float q) {
 // N (a multiple of 8) values of one block row and the block maximum -> N/8 words
 // of codes (element i in bits 4(i%8).. of word i/8) and the scale byte.
 // fp32(a / 6) for a bf16 value a (the block maximum of bf16 inputs), correctly
-// rounded without a division: q0 = RN(a * RN(1/6)) is at most one ulp off and one
-// fused correction q0 + RN(a - 6 q0) * RN(1/6) (the residual is exact) lands on the
-// correctly rounded quotient for every finite bf16 a (checked exhaustively against
-// IEEE division on the GPU by the scale tests of every bf16 block maximum).
+// rounded without a division, by the correction step for division by a constant
+// known in advance of Brisebarre, Muller and Raina ("Accelerating correctly
+// rounded floating-point division when the divisor is known in advance", IEEE
+// Trans. Computers 53(8), 2004): q0 = RN(a * RN(1/6)) is at most one ulp off; the
+// residual a - 6 q0 is exact in one fused multiply-add, and q0 + RN(residual) *
+// RN(1/6) lands on the correctly rounded quotient for every finite bf16 a
+// (checked exhaustively against IEEE division on the GPU by the scale tests of
+// every bf16 block maximum).
 __device__ __forceinline__ float div6_bf16(float a) {
   constexpr float kSixth = 1.0f / 6.0f;
   const float q0 = a * kSixth;

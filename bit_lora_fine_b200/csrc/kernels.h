@@ -24,6 +24,8 @@ struct RowpassParams {
   float* part;                           // fp32 [nsplit, M, R] when nsplit > 1
   int* counters;                         // [ceil(M/128)], zero on entry, left zero (nsplit > 1)
   int* status;
+  unsigned long long wait_ns;            // limit of every bounded wait (0: the default, 2 s)
+  int fault_skip_stage;                  // test hook: CTA (0, 0) never loads this stage (-1: none)
 };
 
 // MMA-ready scale layout of a block16 operand with `rows` rows (along M or N)

@@ -84,6 +84,10 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   const int kt0 = split * p.kt_per_split;
   const int kt1 = min(KT, kt0 + p.kt_per_split);
   const int nt = max(0, kt1 - kt0);
+  const uint64_t lim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
+  // test hook: in CTA (0, 0) the producer leaves this stage out, so the waits
+  // for it expire and the bounded-wait abort path runs (never set otherwise)
+  const int skip = (blockIdx.x == 0 && blockIdx.y == 0) ? p.fault_skip_stage : -1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -116,7 +120,9 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       int s = 0;                 // ring slot and its phase parity (no division by the runtime depth)
       uint32_t ph = 0;
       for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
-        if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp)) break;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.status, abortp, lim)) break;
+        issued = i + 1;
+        if (i == skip) continue;
         uint8_t* st = smem + s * stage_bytes;
         const int kc = (kt0 + i) * 64;
         mbar_arrive_expect_tx(&full[s], kRpXBytes + w_bytes);
@@ -127,11 +133,10 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         } else {
           tma_load_2d(st + kRpXBytes, &tmW, &full[s], kc, 0);
         }
-        issued = i + 1;
       }
       if (*abortp) {  // let copies already in flight land before the CTA exits
         for (int i = max(0, issued - NS); i < issued; ++i)  // once, on the abort path only
-          mbar_wait_drain(&full[i % NS], (i / NS) & 1, 100000000ull);
+          if (i != skip) mbar_wait_drain(&full[i % NS], (i / NS) & 1, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -140,8 +145,8 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
-        if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
-        if (GELU && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
+        if (!mbar_wait(&full[s], ph, p.status, abortp, lim)) break;
+        if (GELU && !mbar_wait(&ready[s], ph, p.status, abortp, lim)) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(smem + s * stage_bytes);
         const uint32_t wa = xa + kRpXBytes;
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
-      if (!mbar_wait(&full[s], ph, p.status, abortp)) {
+      if (!mbar_wait(&full[s], ph, p.status, abortp, lim)) {
         ok = false;
         break;
       }
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     // fp32 partials.  All agree on whether to run it, so the named barriers
     // below are always reached by all of them.
     {
-      const bool mine = ok && mbar_wait(acc_full, 0, p.status, abortp);
+      const bool mine = ok && mbar_wait(acc_full, 0, p.status, abortp, lim);
       if (lane == 0) s_ok[w16] = mine ? 1 : 0;
       named_bar_sync(1, 32 * kRpQuantWarps);
       bool go = true;

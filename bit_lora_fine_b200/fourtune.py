@@ -27,7 +27,8 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_quant_down_static", "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_fwd",
             "fourtune_mlp_bwd_workspace_size", "fourtune_mlp_bwd", "fourtune_mlp_fwd_ws_offsets",
             "fourtune_mlp_bwd_ws_offsets", "fourtune_mma_scales_size", "fourtune_mma_scales",
-            "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32")
+            "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32",
+            "fourtune_quant_down_static_status", "fourtune_test_wait_timeout")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
@@ -81,6 +82,8 @@ def load():
     L.fourtune_linear_fwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz)]
     L.fourtune_linear_bwd_ws_offsets.argtypes = [P(ft_linear_t), i64, P(sz), P(sz), P(sz)]
     L.fourtune_quant_down_static.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp, vp]
+    L.fourtune_quant_down_static_status.argtypes = [vp]
+    L.fourtune_test_wait_timeout.argtypes = [vp, i64, i64, vp, i64, vp, vp, vp, vp, sz, i64, vp]
     L.fourtune_device_status.argtypes = [vp, vp]
     L.fourtune_error_string.argtypes = [ctypes.c_int]
     L.fourtune_error_string.restype = ctypes.c_char_p
@@ -124,6 +127,29 @@ def _need(t, dtype, name):
         return
     if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def _shape(t, shape, name):
+    """Raise ValueError unless tensor t (if given) has exactly `shape`."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _out_dtype(t, name):
+    if t is not None and t.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"{name} must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ndim2(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor, got {t.dim()} dimensions")
+
+
+def _same_device(*named):
+    """All given tensors on one device (None entries skipped)."""
+    devs = {(n, t.device) for n, t in named if t is not None}
+    if len({d for _, d in devs}) > 1:
+        raise ValueError("tensors on different devices: " + ", ".join(f"{n}:{d}" for n, d in sorted(devs, key=str)))
 
 
 def quantize_block16(x, transposed=False):
@@ -247,8 +273,14 @@ def _events(events):
 def linear_fwd(layer, X, y_dtype=torch.float32, ws=None, Y=None, L=None, events=None):
     """Y = deq(Q(X) Q(R)^T) + L [S_up ; B] + bias, L = bf16(X [S_dn | A]).  Returns (Y, L, ws).
     `events`: optional 2*len(FWD_KERNELS) torch.cuda.Events recorded around each kernel."""
-    _need(X, torch.bfloat16, "X")
+    _ndim2(X, "X")
     M = X.shape[0]
+    _shape(X, (M, layer.K), "X")
+    _shape(Y, (M, layer.N), "Y")
+    _shape(L, (M, layer.R_all), "L")
+    _same_device(("X", X), ("Y", Y), ("L", L), ("ws", ws))
+    _out_dtype(Y, "Y")
+    _need(X, torch.bfloat16, "X")
     Y = torch.empty((M, layer.N), dtype=y_dtype, device=X.device) if Y is None else Y
     L = torch.empty((M, layer.R_all), dtype=torch.bfloat16, device=X.device) if L is None else L
     ws = layer.fwd_workspace(M) if ws is None else ws
@@ -265,8 +297,19 @@ def linear_fwd(layer, X, y_dtype=torch.float32, ws=None, Y=None, L=None, events=
 def linear_bwd(layer, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumulate=False, ws=None, dX=None,
                events=None):
     """dX = deq(Q(dY)) deq(Q(R)) + P [S_dn | A]^T, dA = X^T P_B, dB = L_B^T dY.  Returns (dX, dA, dB, ws)."""
-    _need(dY, torch.bfloat16, "dY")
+    _ndim2(dY, "dY")
     M = dY.shape[0]
+    _shape(dY, (M, layer.N), "dY")
+    _shape(X, (M, layer.K), "X")
+    _shape(L, (M, layer.R_all), "L")
+    _shape(dX, (M, layer.K), "dX")
+    _shape(dA, (layer.K, layer.r), "dA")
+    _shape(dB, (layer.r, layer.N), "dB")
+    _same_device(("dY", dY), ("X", X), ("L", L), ("dX", dX), ("dA", dA), ("dB", dB), ("ws", ws))
+    _out_dtype(dX, "dX")
+    _need(dY, torch.bfloat16, "dY")
+    _need(X, torch.bfloat16, "X")
+    _need(L, torch.bfloat16, "L")
     dX = torch.empty((M, layer.K), dtype=dx_dtype, device=dY.device) if dX is None else dX
     dA = torch.zeros((layer.K, layer.r), dtype=torch.float32, device=dY.device) if dA is None else dA
     dB = torch.zeros((layer.r, layer.N), dtype=torch.float32, device=dY.device) if dB is None else dB
@@ -319,8 +362,15 @@ class MLP:
 def mlp_fwd(mlp, X, y_dtype=torch.float32, ws=None, dbg_a=False, out=None, events=None):
     """Returns (Y, h, L1, L2, ws, a) -- a is the fp32 activation when dbg_a, else None.
     out: optional preallocated (Y, h, L1, L2); events: 2*len(MLP_FWD_KERNELS) torch.cuda.Events."""
-    _need(X, torch.bfloat16, "X")
+    _ndim2(X, "X")
     M = X.shape[0]
+    _shape(X, (M, mlp.fc1.K), "X")
+    if out is not None:
+        for t, shp, n in zip(out, ((M, mlp.fc2.N), (M, mlp.H), (M, mlp.fc1.R_all), (M, mlp.fc2.R_all)),
+                             ("Y", "h", "L1", "L2")):
+            _shape(t, shp, n)
+    _same_device(("X", X), ("ws", ws), *(() if out is None else zip(("Y", "h", "L1", "L2"), out)))
+    _need(X, torch.bfloat16, "X")
     dev = X.device
     if out is None:
         Y = torch.empty((M, mlp.fc2.N), dtype=y_dtype, device=dev)
@@ -345,8 +395,23 @@ def mlp_fwd(mlp, X, y_dtype=torch.float32, ws=None, dbg_a=False, out=None, event
 def mlp_bwd(mlp, dY, X, h, L1, L2, dx_dtype=torch.float32, accumulate=False, grads=None, ws=None, dX=None,
             events=None):
     """Returns (dX, dA1, dB1, dA2, dB2, ws).  events: 2*len(MLP_BWD_KERNELS) torch.cuda.Events."""
-    _need(dY, torch.bfloat16, "dY")
+    _ndim2(dY, "dY")
     M = dY.shape[0]
+    _shape(dY, (M, mlp.fc2.N), "dY")
+    _shape(X, (M, mlp.fc1.K), "X")
+    _shape(h, (M, mlp.H), "h")
+    _shape(L1, (M, mlp.fc1.R_all), "L1")
+    _shape(L2, (M, mlp.fc2.R_all), "L2")
+    _shape(dX, (M, mlp.fc1.K), "dX")
+    if grads is not None:
+        for t, shp, n in zip(grads, ((mlp.fc1.K, mlp.fc1.r), (mlp.fc1.r, mlp.fc1.N), (mlp.fc2.K, mlp.fc2.r),
+                                     (mlp.fc2.r, mlp.fc2.N)), ("dA1", "dB1", "dA2", "dB2")):
+            _shape(t, shp, n)
+    _same_device(("dY", dY), ("X", X), ("h", h), ("L1", L1), ("L2", L2), ("dX", dX), ("ws", ws),
+                 *(() if grads is None else zip(("dA1", "dB1", "dA2", "dB2"), grads)))
+    _need(dY, torch.bfloat16, "dY")
+    for t, n in ((X, "X"), (h, "h"), (L1, "L1"), (L2, "L2")):
+        _need(t, torch.bfloat16, n)
     dev = dY.device
     dX = torch.empty((M, mlp.fc1.K), dtype=dx_dtype, device=dev) if dX is None else dX
     if grads is None:
@@ -372,15 +437,49 @@ def quant_down_static(X, W, codes=None, scales=None, L=None):
     """Allocation-free fused row pass: block16(X) and L = bf16(X W^T), X [M, K], W [R, K] bf16.
     The library keeps this call's scratch in a fixed device array (no workspace);
     overlapping calls race.  Returns (codes, scales, L)."""
-    _need(X, torch.bfloat16, "X")
-    _need(W, torch.bfloat16, "W")
-    M, K = X.shape
-    R = W.shape[0]
+    M, K, R = _quant_down_shapes(X, W, codes, scales, L)
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device) if codes is None else codes
     scales = torch.empty((M // 16, K // 16), dtype=torch.uint8, device=X.device) if scales is None else scales
     L = torch.empty((M, R), dtype=torch.bfloat16, device=X.device) if L is None else L
     _check(load().fourtune_quant_down_static(_ptr(X), M, K, _ptr(W), R, _ptr(codes), _ptr(scales), _ptr(L),
                                              _stream()), "fourtune_quant_down_static")
+    return codes, scales, L
+
+
+def _quant_down_shapes(X, W, codes, scales, L):
+    """Shape, device and dtype checks of the fused row pass's arguments; returns (M, K, R)."""
+    _ndim2(X, "X")
+    _ndim2(W, "W")
+    M, K = X.shape
+    R = W.shape[0]
+    _shape(W, (R, K), "W")
+    _shape(codes, (M, K // 2), "codes")
+    _shape(scales, (M // 16, K // 16), "scales")
+    _shape(L, (M, R), "L")
+    _same_device(("X", X), ("W", W), ("codes", codes), ("scales", scales), ("L", L))
+    _need(X, torch.bfloat16, "X")
+    _need(W, torch.bfloat16, "W")
+    return M, K, R
+
+
+def quant_down_static_status():
+    """Synchronize and raise FourtuneError(FT_ERR_TIMEOUT) if a kernel wait of the last
+    quant_down_static call on this device expired."""
+    _check(load().fourtune_quant_down_static_status(_stream()), "fourtune_quant_down_static_status")
+
+
+def fault_wait_timeout(X, W, ws, wait_ns=5_000_000):
+    """Failure-path test hook: the fused row pass with one CTA's first stage left
+    unloaded and every wait limited to wait_ns.  Returns (codes, scales, L); the
+    expired wait is then reported by device_status(ws)."""
+    M, K, R = _quant_down_shapes(X, W, None, None, None)
+    _need(ws, torch.uint8, "ws")
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((M // 16, K // 16), dtype=torch.uint8, device=X.device)
+    L = torch.empty((M, R), dtype=torch.bfloat16, device=X.device)
+    _check(load().fourtune_test_wait_timeout(_ptr(X), M, K, _ptr(W), R, _ptr(codes), _ptr(scales), _ptr(L),
+                                             _ptr(ws), ws.numel(), int(wait_ns), _stream()),
+           "fourtune_test_wait_timeout")
     return codes, scales, L
 
 

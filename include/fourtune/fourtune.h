@@ -244,15 +244,40 @@ FT_API int fourtune_linear_bwd_ws_offsets(const ft_linear_t* layer, int64_t M, s
  * FT_STATIC_SCRATCH_BYTES (16 MiB) on every GPU that loads the library, kept
  * until the process exits; no cudaMalloc, cudaFree or other allocation is made.
  * The first call on a device looks up the array's device address on that
- * device, so make that first call before any stream capture begins.  Every
- * call shares the array: calls that overlap on the GPU (other streams, other
- * host threads) race and corrupt each other's results; serialize them.
- * Returns FT_ERR_WORKSPACE when the problem needs more scratch than the array
- * holds (only for M in the millions of tokens), FT_ERR_UNSUPPORTED for R
- * outside 16..128 (multiples of 16), else as the other calls. */
+ * device and keeps it for the life of the process, so make that first call
+ * before any stream capture begins; a cudaDeviceReset (or anything else that
+ * tears down the device's primary context) invalidates the kept address, and
+ * the entry point must not be called on that device afterwards.  Every call
+ * shares the array: calls that overlap on the GPU (other streams, other host
+ * threads) race and corrupt each other's results; serialize them.  The split
+ * rule is the workspace path's, so the outputs are bit-identical to the
+ * forward's.  Returns FT_ERR_WORKSPACE when the problem needs more scratch than
+ * the array holds (only for M in the millions of tokens), FT_ERR_UNSUPPORTED
+ * for R outside 16..128 (multiples of 16), else as the other calls.  An
+ * expired wait is recorded in the array: fourtune_quant_down_static_status
+ * reports it. */
 #define FT_STATIC_SCRATCH_BYTES (16u << 20)
 FT_API int fourtune_quant_down_static(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
                                       uint8_t* codes, uint8_t* scales, ft_bf16* L, void* stream);
+
+/* Status of the last fourtune_quant_down_static call on the current device
+ * (no counterpart in the paper): synchronizes `stream` and returns
+ * FT_ERR_TIMEOUT if one of its kernel waits expired (the outputs are then
+ * incomplete), FT_ERR_CUDA on a CUDA error, else FT_OK.  Allocates nothing. */
+FT_API int fourtune_quant_down_static_status(void* stream);
+
+/* Test hook for the failure path (no counterpart in the paper).  Runs the fused
+ * row pass of fourtune_quant_down_static with its bookkeeping in the caller's
+ * `ws` (256-byte aligned; at least 256 + 4 ceil(M/128) + 64 M R bytes is always
+ * enough) and with every kernel wait limited to `wait_ns` (1e6 .. 1e9 ns), and
+ * makes the first CTA's producer leave its first stage unloaded: the waits for
+ * that stage expire, the CTA records FT_ERR_TIMEOUT in ws, stops waiting,
+ * drains the copies it started and frees its tensor memory.  The outputs of
+ * that CTA's rows are then incomplete; fourtune_device_status(ws) returns
+ * FT_ERR_TIMEOUT.  Nothing faults or traps: the GPU stays usable. */
+FT_API int fourtune_test_wait_timeout(const ft_bf16* X, int64_t M, int64_t K, const ft_bf16* W, int64_t R,
+                                      uint8_t* codes, uint8_t* scales, ft_bf16* L, void* ws, size_t ws_bytes,
+                                      int64_t wait_ns, void* stream);
 
 /* Synchronizes `stream` and returns FT_ERR_TIMEOUT if a kernel of the last call
  * that used `ws` recorded an expired wait, FT_ERR_CUDA on a CUDA error, else FT_OK. */

@@ -43,6 +43,62 @@ def check_bf16_dot(got, ref, absdot, n):
     assert normwise(got, ref) <= 2.0 ** -7
 
 
+# Elementwise bound of an fp32-accumulated sum of n products against its exact
+# value: the tensor cores' products of dequantized FP4 or bf16 operands are
+# exact, each accumulation step rounds with relative error at most 2^-23 (twice
+# the nearest-even unit, for adders that truncate), so the error is at most
+# n * 2^-23 * sum_k |a_k b_k| (absdot), plus the final rounding of the stored fp32.
+GAMMA_FP32 = 2.0 ** -23
+
+
+def fp32_dot_bound(absdot, n):
+    return n * GAMMA_FP32 * np.asarray(absdot, dtype=np.float64)
+
+
+def check_fp32_dot(got, ref, absdot, n, extra=0.0, name="output"):
+    """fp32 output of an fp32-accumulated product vs the exact (float64) value:
+    elementwise |got - ref| <= n 2^-23 absdot + 2^-24 |ref| + extra (extra: a
+    caller-stated bound for inputs that were themselves rounded, e.g. a bf16
+    intermediate one ulp away).  Returns the largest error / bound ratio (the
+    elementwise figure reported next to the normwise one)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    bound = fp32_dot_bound(absdot, n) + 2.0 ** -24 * np.abs(ref) + np.asarray(extra, dtype=np.float64) + 1e-30
+    ratio = np.abs(got - ref) / bound
+    worst = float(ratio.max()) if ratio.size else 0.0
+    assert worst <= 1.0, f"{name}: {int((ratio > 1).sum())} elements beyond the fp32 accumulation bound " \
+                         f"(worst ratio {worst:.3g})"
+    return worst
+
+
+def check_bf16_rounded(got, ref, err_bound, name="output"):
+    """bf16 value that is the rounding of a computed quantity whose exact value is
+    `ref` and whose error before rounding is at most err_bound (elementwise):
+    |got - ref| <= one bf16 ulp at |ref| + err_bound.  Returns the worst ratio."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    mag = np.maximum(np.abs(ref), 2.0 ** -126)
+    bound = 2.0 ** (np.floor(np.log2(mag)) - 7) + np.asarray(err_bound, dtype=np.float64) + 1e-38
+    ratio = np.abs(got - ref) / bound
+    worst = float(ratio.max()) if ratio.size else 0.0
+    assert worst <= 1.0, f"{name}: {int((ratio > 1).sum())} elements beyond one bf16 ulp + bound " \
+                         f"(worst ratio {worst:.3g})"
+    return worst
+
+
+def nan_dev(shape, dtype=None):
+    """Device tensor filled with NaN: an output element a kernel never writes stays NaN."""
+    import torch
+    return torch.full(shape, float("nan"), dtype=dtype or torch.float32, device="cuda")
+
+
+def poisoned_ws(nbytes):
+    """Workspace filled with 0xFF bytes: the call must clear what it needs (status
+    word, counters) and write every intermediate it reads."""
+    import torch
+    return torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")
+
+
 def to_dev_bf16(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda").to(torch.bfloat16)

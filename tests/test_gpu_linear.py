@@ -12,7 +12,8 @@ import pytest
 
 from bit_lora_fine_b200 import synth
 from oracle import block16, formats, layer as olayer
-from tests.helpers import TOL, check_bf16_dot, normwise, random_layer, tie_tensor, to_dev_bf16, to_host
+from tests.helpers import (TOL, check_bf16_dot, check_fp32_dot, nan_dev, normwise, poisoned_ws, random_layer,
+                           tie_tensor, to_dev_bf16, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +27,27 @@ def _device_layer(ft, p):
     return lay
 
 
+def _fwd_ref_on_gpu_L(ref, Lg, U, bias, Xq, Rq):
+    """Exact forward given the GPU's own bf16 L (the GPU's y used it): the oracle's y
+    with its L U replaced by Lg U, and the elementwise |.| sums of the products."""
+    y = ref["y"] + (Lg - ref["L"]) @ U
+    absdot = np.abs(Xq) @ np.abs(Rq).T + np.abs(Lg) @ np.abs(U)
+    if bias is not None:
+        absdot = absdot + np.abs(bias)[None, :]
+    return y, absdot
+
+
+def _bwd_ref_on_gpu_P(b, Pg, D, Gq, Rq):
+    """Exact dX given the GPU's own bf16 P, and its elementwise |.| sums."""
+    dX = b["dX"] + (Pg - b["P"]) @ D.T
+    absdot = np.abs(Gq) @ np.abs(Rq) + np.abs(Pg) @ np.abs(D).T
+    return dX, absdot
+
+
 def run_and_check(ft, p, M, check_bf16=True):
+    """Forward and backward at full size against the oracle, every element.  Outputs
+    and workspaces start poisoned (NaN / 0xFF), so an element that no kernel
+    writes, or a header the call does not clear, fails the comparison."""
     import torch
     X, dY = p["X"], p["dY"]
     lay = _device_layer(ft, p)
@@ -34,44 +55,64 @@ def run_and_check(ft, p, M, check_bf16=True):
     np.testing.assert_array_equal(lay.t["R_codes"].cpu().numpy(), R_codes)
     np.testing.assert_array_equal(lay.t["R_scales"].cpu().numpy(), R_scales)
     np.testing.assert_array_equal(lay.t["R_codes_t"].cpu().numpy(), block16.transpose_pack(R_codes))
+    K, N, R_all, r_s = lay.K, lay.N, lay.R_all, lay.r_s
+    bias = p.get("bias")
+    D = np.concatenate([p["S_dn"], p["A"]], axis=1).astype(np.float64)
+    U = np.concatenate([p["S_up"], p["B"]], axis=0).astype(np.float64)
+    Rq = block16.dequantize(R_codes, R_scales)
 
     Xd, dYd = to_dev_bf16(X), to_dev_bf16(dY)
-    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32)
+    ws = poisoned_ws(lay.fwd_workspace(M).numel())
+    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32, ws=ws, Y=nan_dev((M, N)),
+                             L=nan_dev((M, R_all), torch.bfloat16))
     ft.device_status(ws)
     co, so = lay.fwd_ws_offsets(M)
-    K, N = lay.K, lay.N
     qx_codes = ws[co:co + M * K // 2].view(M, K // 2).cpu().numpy()
     qx_scales = ws[so:so + (M // 16) * (K // 16)].view(M // 16, K // 16).cpu().numpy()
 
-    ref = olayer.linear_fwd(X, R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
+    ref = olayer.linear_fwd(X, R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"], bias)
     np.testing.assert_array_equal(qx_scales, ref["qx_scales"])
     np.testing.assert_array_equal(qx_codes, ref["qx_codes"])
-    D = np.concatenate([p["S_dn"], p["A"]], axis=1).astype(np.float64)
-    check_bf16_dot(to_host(L), ref["L"], np.abs(X) @ np.abs(D), K)
-    assert normwise(to_host(Y), ref["y"]) <= TOL, normwise(to_host(Y), ref["y"])
+    Lg = to_host(L)
+    check_bf16_dot(Lg, ref["L"], np.abs(X) @ np.abs(D), K)
+    Yg = to_host(Y)
+    assert normwise(Yg, ref["y"]) <= TOL, normwise(Yg, ref["y"])
+    y_ex, absdot_y = _fwd_ref_on_gpu_L(ref, Lg, U, bias, block16.dequantize(qx_codes, qx_scales), Rq)
+    check_fp32_dot(Yg, y_ex, absdot_y, K + R_all, name="y")
 
     if check_bf16:
-        Yb, _, _ = ft.linear_fwd(lay, Xd, torch.bfloat16, ws=ws)
+        Yb, _, _ = ft.linear_fwd(lay, Xd, torch.bfloat16, ws=ws, Y=nan_dev((M, N), torch.bfloat16))
         torch.cuda.synchronize()
         np.testing.assert_array_equal(to_host(Yb), to_host(Y.to(torch.bfloat16)))
 
-    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32)
+    wsb = poisoned_ws(lay.bwd_workspace(M).numel())
+    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32, ws=wsb, dX=nan_dev((M, K)),
+                                    dA=nan_dev((K, lay.r)), dB=nan_dev((lay.r, N)))
     ft.device_status(wsb)
     gc, gs, po = lay.bwd_ws_offsets(M)
     qg_codes = wsb[gc:gc + M * N // 2].view(M, N // 2).cpu().numpy()
     qg_scales = wsb[gs:gs + (M // 16) * (N // 16)].view(M // 16, N // 16).cpu().numpy()
-    R_all = lay.R_all
-    P = wsb[po:po + M * R_all * 2].view(torch.bfloat16).view(M, R_all)
+    Pg = to_host(wsb[po:po + M * R_all * 2].view(torch.bfloat16).view(M, R_all))
 
     # backward reference on the GPU's own saved L (the saved tensor is the interface)
-    b = olayer.linear_bwd(dY, X, to_host(L), R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"])
+    b = olayer.linear_bwd(dY, X, Lg, R_codes, R_scales, p["S_dn"], p["S_up"], p["A"], p["B"])
     np.testing.assert_array_equal(qg_scales, b["qg_scales"])
     np.testing.assert_array_equal(qg_codes, b["qg_codes"])
-    U = np.concatenate([p["S_up"], p["B"]], axis=0).astype(np.float64)
-    check_bf16_dot(to_host(P), b["P"], np.abs(dY) @ np.abs(U).T, N)
-    assert normwise(to_host(dX), b["dX"]) <= TOL, normwise(to_host(dX), b["dX"])
-    assert normwise(to_host(dA), b["dA"]) <= TOL, normwise(to_host(dA), b["dA"])
-    assert normwise(to_host(dB), b["dB"]) <= TOL, normwise(to_host(dB), b["dB"])
+    check_bf16_dot(Pg, b["P"], np.abs(dY) @ np.abs(U).T, N)
+    dXg, dAg, dBg = to_host(dX), to_host(dA), to_host(dB)
+    assert normwise(dXg, b["dX"]) <= TOL, normwise(dXg, b["dX"])
+    assert normwise(dAg, b["dA"]) <= TOL, normwise(dAg, b["dA"])
+    assert normwise(dBg, b["dB"]) <= TOL, normwise(dBg, b["dB"])
+    dx_ex, absdot_dx = _bwd_ref_on_gpu_P(b, Pg, D, block16.dequantize(qg_codes, qg_scales), Rq)
+    check_fp32_dot(dXg, dx_ex, absdot_dx, N + R_all, name="dX")
+    Xf = X.astype(np.float64)
+    check_fp32_dot(dAg, Xf.T @ Pg[:, r_s:], np.abs(Xf).T @ np.abs(Pg[:, r_s:]), M, name="dA")
+    check_fp32_dot(dBg, Lg[:, r_s:].T @ dY.astype(np.float64), np.abs(Lg[:, r_s:]).T @ np.abs(dY), M, name="dB")
+
+    if check_bf16:
+        dXb, _, _, _ = ft.linear_bwd(lay, dYd, Xd, L, torch.bfloat16, ws=wsb, dX=nan_dev((M, K), torch.bfloat16))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(to_host(dXb), to_host(dX.to(torch.bfloat16)))
 
     # accumulate = 1 adds into dA, dB
     dX2, dA2, dB2, _ = ft.linear_bwd(lay, dYd, Xd, L, torch.float32, dA=dA.clone(), dB=dB.clone(),
@@ -151,15 +192,20 @@ def test_repeated_calls_are_bit_identical(cuda_lib):
 
 def run_sampled(ft, p, X, dY, rows):
     """Full-size linear fwd+bwd; y, Q(X), Q(G), dX, L, P on sampled 16-row blocks
-    against the oracle; dA and dB in full from the GPU's own L and P."""
+    against the oracle; dA and dB in full from the GPU's own L and P; bf16 y and
+    dX equal to the rounding of the fp32 outputs everywhere."""
     import torch
     M = X.shape[0]
     lay = _device_layer(ft, p)
-    K, N, r_s = lay.K, lay.N, lay.r_s
+    K, N, r_s, R_all = lay.K, lay.N, lay.r_s, lay.R_all
     Rc, Rs = block16.quantize(p["R"])
+    Rq = block16.dequantize(Rc, Rs)
     Xd, dYd = to_dev_bf16(X), to_dev_bf16(dY)
-    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32)
-    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32)
+    ws = poisoned_ws(lay.fwd_workspace(M).numel())
+    wsb = poisoned_ws(lay.bwd_workspace(M).numel())
+    Y, L, ws = ft.linear_fwd(lay, Xd, torch.float32, ws=ws, Y=nan_dev((M, N)), L=nan_dev((M, R_all), torch.bfloat16))
+    dX, dA, dB, wsb = ft.linear_bwd(lay, dYd, Xd, L, torch.float32, ws=wsb, dX=nan_dev((M, K)),
+                                    dA=nan_dev((K, lay.r)), dB=nan_dev((lay.r, N)))
     ft.device_status(ws)
     ft.device_status(wsb)
     co, so = lay.fwd_ws_offsets(M)
@@ -170,25 +216,41 @@ def run_sampled(ft, p, X, dY, rows):
     qg = wsb[gc:gc + M * N // 2].view(M, N // 2).cpu().numpy()[rows]
     qgs = wsb[gs:gs + (M // 16) * (N // 16)].view(M // 16, N // 16).cpu().numpy()[blocks]
     Lh = to_host(L)
-    P = to_host(wsb[po:po + M * lay.R_all * 2].view(torch.bfloat16).view(M, lay.R_all))
+    P = to_host(wsb[po:po + M * R_all * 2].view(torch.bfloat16).view(M, R_all))
+    Yg, dXg = to_host(Y), to_host(dX)
+    assert not np.isnan(Yg).any() and not np.isnan(dXg).any()
 
+    D = np.concatenate([p["S_dn"], p["A"]], axis=1).astype(np.float64)
+    U = np.concatenate([p["S_up"], p["B"]], axis=0).astype(np.float64)
     ref = olayer.linear_fwd(X[rows], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
     np.testing.assert_array_equal(qxs, ref["qx_scales"])
     np.testing.assert_array_equal(qx, ref["qx_codes"])
-    D = np.concatenate([p["S_dn"], p["A"]], axis=1).astype(np.float64)
     check_bf16_dot(Lh[rows], ref["L"], np.abs(X[rows]) @ np.abs(D), K)
-    assert normwise(to_host(Y)[rows], ref["y"]) <= TOL
+    assert normwise(Yg[rows], ref["y"]) <= TOL
+    y_ex, absdot_y = _fwd_ref_on_gpu_L(ref, Lh[rows], U, p.get("bias"), block16.dequantize(qx, qxs), Rq)
+    check_fp32_dot(Yg[rows], y_ex, absdot_y, K + R_all, name="y")
     b = olayer.linear_bwd(dY[rows], X[rows], Lh[rows], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"])
     np.testing.assert_array_equal(qgs, b["qg_scales"])
     np.testing.assert_array_equal(qg, b["qg_codes"])
-    U = np.concatenate([p["S_up"], p["B"]], axis=0).astype(np.float64)
     check_bf16_dot(P[rows], b["P"], np.abs(dY[rows]) @ np.abs(U).T, N)
-    assert normwise(to_host(dX)[rows], b["dX"]) <= TOL
-    assert normwise(to_host(dA), X.astype(np.float64).T @ P[:, r_s:]) <= TOL
-    assert normwise(to_host(dB), Lh[:, r_s:].T @ dY.astype(np.float64)) <= TOL
+    assert normwise(dXg[rows], b["dX"]) <= TOL
+    dx_ex, absdot_dx = _bwd_ref_on_gpu_P(b, P[rows], D, block16.dequantize(qg, qgs), Rq)
+    check_fp32_dot(dXg[rows], dx_ex, absdot_dx, N + R_all, name="dX")
+    Xf, dYf = X.astype(np.float64), dY.astype(np.float64)
+    dA_ex, dB_ex = Xf.T @ P[:, r_s:], Lh[:, r_s:].T @ dYf
+    assert normwise(to_host(dA), dA_ex) <= TOL
+    assert normwise(to_host(dB), dB_ex) <= TOL
+    check_fp32_dot(to_host(dA), dA_ex, np.abs(Xf).T @ np.abs(P[:, r_s:]), M, name="dA")
+    check_fp32_dot(to_host(dB), dB_ex, np.abs(Lh[:, r_s:]).T @ np.abs(dYf), M, name="dB")
+    # the production (bf16) outputs: the rounding of the fp32 outputs, every element
+    Yb, _, _ = ft.linear_fwd(lay, Xd, torch.bfloat16, ws=ws, Y=nan_dev((M, N), torch.bfloat16))
+    dXb, _, _, _ = ft.linear_bwd(lay, dYd, Xd, L, torch.bfloat16, ws=wsb, dX=nan_dev((M, K), torch.bfloat16))
+    torch.cuda.synchronize()
+    assert torch.equal(Yb, Y.to(torch.bfloat16))
+    assert torch.equal(dXb, dX.to(torch.bfloat16))
 
 
-def _sample_rows(M, nblocks=8, seed=0):
+def _sample_rows(M, nblocks=16, seed=0):
     rng = np.random.default_rng(seed)
     blocks = np.sort(rng.choice(M // 16, size=nblocks, replace=False))
     return (blocks[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)

@@ -5,9 +5,10 @@ memory and offer no scratch allocator, runtimes that forbid allocation once
 running), so this entry point keeps its scratch in a fixed device array inside
 the library.  It must compute exactly what the workspace path computes: the
 block16 codes and scales of X and L = bf16(X [S_dn | A]) that
-fourtune_linear_fwd produces, on two calls in a row (the array keeps the
-previous call's contents, so the second call checks that the state is reset).
-This file is collected last on purpose.
+fourtune_linear_fwd produces -- bit for bit, since both choose the same
+split-K -- on two calls in a row (the array keeps the previous call's contents,
+so the second call checks that the state is reset), and report through its own
+status query that no wait expired.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -15,18 +16,27 @@ import numpy as np
 import pytest
 
 from bit_lora_fine_b200 import synth
-from tests.helpers import check_bf16_dot, to_dev_bf16, to_host
+from tests.helpers import check_bf16_dot, random_layer, to_dev_bf16, to_host
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("workload", ["flux-linear-3072", "linear-256x512x512"])
+def _case(name):
+    """(layer params, X) of a named workload, or of the small-M, wide-K case whose
+    row pass splits K sixteen ways (M = 128, K = 4096, ranks 32 + 32)."""
+    if name == "small-m-wide-k":
+        p = random_layer(4096, 256, 32, 32, seed=5, M=128)
+        return p, p["X"]
+    wl = synth.WORKLOADS[name]
+    return synth.layer_params(wl.layers[0]), synth.layer_input(wl)
+
+
+@pytest.mark.parametrize("workload", ["flux-linear-3072", "linear-256x512x512", "small-m-wide-k"])
 def test_static_scratch_row_pass_matches_workspace_path(cuda_lib, workload):
     import torch
     ft = cuda_lib
-    wl = synth.WORKLOADS[workload]
-    p = synth.layer_params(wl.layers[0])
-    X = to_dev_bf16(synth.layer_input(wl))
+    p, Xh = _case(workload)
+    X = to_dev_bf16(Xh)
     dev = {k: to_dev_bf16(p[k]) for k in ("R", "S_dn", "S_up", "A", "B")}
     lay = ft.Linear.from_weights(dev["R"], dev["S_dn"], dev["S_up"], dev["A"], dev["B"])
     M, K, R = X.shape[0], lay.K, lay.R_all
@@ -39,14 +49,14 @@ def test_static_scratch_row_pass_matches_workspace_path(cuda_lib, workload):
     scales_ref = ws[so:so + (M // 16) * (K // 16)].view(M // 16, K // 16).cpu().numpy()
 
     W = torch.cat([dev["S_dn"], dev["A"]], dim=1).t().contiguous()     # [R, K]
-    Xh = synth.layer_input(wl).astype(np.float64)
-    absdot = np.abs(Xh) @ np.abs(to_host(W).T)
+    absdot = np.abs(Xh.astype(np.float64)) @ np.abs(to_host(W).T)
     for _ in range(2):
         codes, scales, L = ft.quant_down_static(X, W)
-        torch.cuda.synchronize()
+        ft.quant_down_static_status()
         np.testing.assert_array_equal(scales.cpu().numpy(), scales_ref)
         np.testing.assert_array_equal(codes.cpu().numpy(), codes_ref)
         check_bf16_dot(to_host(L), to_host(L_ref), absdot, K)
+        assert torch.equal(L, L_ref)                                   # same split-K: same sums
 
 
 def test_static_scratch_rejects_oversize(cuda_lib):
