@@ -261,13 +261,16 @@ def run_ours(args, rank, world, local_rank):
         ft.linear_fwd(lay, X, ws=ws_f, Y=Y, L=L, events=evf)
         ft.linear_bwd(lay, dY, X, L, ws=ws_b, dX=dX, dA=dA, dB=dB, events=evb)
 
-    torch.cuda.synchronize()
-    t_w = time.perf_counter()
     for _ in range(max(args.warmup, 1)):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    wall_per_step = (time.perf_counter() - t_w) / max(args.warmup, 1)
+    t_w = time.perf_counter()                      # wall time of a warm step (flush included)
+    for _ in range(5):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    wall_per_step = (time.perf_counter() - t_w) / 5
     ft.device_status(ws_f)
     ft.device_status(ws_b)
 
@@ -277,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
     # back to back (the same K steps each time) for ~0.4 s so that the clock
     # sampler sees the GPU under load; the value is the median block.  Then K
     # more steps with an event pair around every kernel, for the breakdown.
-    reps = int(min(100, max(3, np.ceil(CLOCK_WINDOW_S / max(args.steps * wall_per_step, 1e-6)))))
+    reps = int(min(200, max(3, np.ceil(CLOCK_WINDOW_S / max(args.steps * wall_per_step, 1e-6)))))
     blocks = [[mk_events(2) for _ in range(args.steps)] for _ in range(reps)]
     ksteps = [(mk_events(2 * nf), mk_events(2 * nb)) for _ in range(args.steps)]
     torch.cuda.synchronize()

@@ -403,11 +403,15 @@ struct GemmArgs {
   void* out2;                   // GELU-backward epilogue: bf16(GELU(h)) [M, N]
 };
 int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
+  // plain epilogues run on CTA pairs (each CTA loads 128 rows of the B tile);
+  // the GELU-backward epilogue on single CTAs (256-row B boxes)
+  const bool pair = a.h == nullptr;
+  const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(ft::kGemmBN);
   CUtensorMap tmA, tmB, tmA2, tmB2;
-  if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, ft::kGemmBN) ||
+  if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, b_rows) ||
       !map_bf16(&tmA2, a.A2, a.R2, a.M, 128))
     return FT_ERR_CUDA;
-  if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, ft::kGemmBN) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
+  if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, b_rows) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
     return FT_ERR_CUDA;
   GemmParams gp{};
   gp.M = static_cast<int>(a.M);
@@ -425,6 +429,7 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   gp.h = a.h;
   gp.out2 = a.out2;
   gp.status = status;
+  if (pair) return cuda_err(ft::launch_gemm_pair(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
   return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
 }
 

@@ -298,6 +298,112 @@ __host__ __device__ constexpr uint32_t idesc_fp4_block16(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// Kernels launched as clusters of two CTAs whose tensor-core work is shared
+// (tcgen05 cta_group::2): rank 0 is the leader that issues the MMAs.  A CTA
+// addresses its peer's shared memory through the cluster window (mapa); the
+// barriers that receive arrivals from the peer are waited on with cluster-scope
+// acquire.  No load here is multicast: each CTA loads its own tiles.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// arrive (release, cluster scope) on a barrier given by its cluster address
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait for barriers that the peer CTA arrives on (cluster-scope acquire)
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status,
+                                                  volatile int* abort_flag, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  uint32_t n = 0;
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if ((++n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        if (status) atomicCAS(status, 0, kDevTimeout);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+// 2-D tiled load into this CTA's shared memory whose completion is counted on
+// the barrier at cluster address `cluster_bar` (the leader's, for pair kernels)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t cluster_bar, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y)
+      : "memory");
+}
+// tensor memory of the CTA pair: the same warp of both CTAs allocates and frees
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// arrive once on the barrier at this shared-memory offset in every CTA of
+// `cta_mask` when all tcgen05 operations issued so far by this thread complete
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+// pair MMAs: M = 256 rows, 128 from each CTA's shared memory (same offsets), B
+// split along N between the two CTAs, each CTA's accumulator rows in its TMEM
+__device__ __forceinline__ void mma_fp4_block16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ conversions
 // E4M3 encode of a non-negative float (round to nearest even, saturate at 448)
 __device__ __forceinline__ uint32_t f32_to_e4m3(float s) {
@@ -434,18 +540,32 @@ __device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, 
 // through 0.5 (1 + tanh(u)) = 1 / (1 + e^{-2u}) =: s (no cancellation for very
 // negative h), so GELU(h) = h s.  Its derivative, with 1 - tanh(u)^2 = 4 s (1 - s)
 // and 1 - s = s e^{-2u}: GELU'(h) = s + 2 h s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 h^2).
-// u is clamped at -40 (e^{-2u} stays finite; s < 2e-35 there either way).  The
-// exponential and the quotient are the fast hardware forms (__expf, __fdividef):
-// over the range where s is not saturated (|2u| <= 20) e^{-2u} is within ~3e-6
-// (relative), which is the relative error of GELU(h) and of s.
+// The exponential and the quotient are the fast hardware forms (__expf,
+// __fdividef): for |u| <= 40 e^{-2u} is within ~5e-6 (relative), the relative
+// error of GELU(h) and of s.  Beyond that s is 0 or 1 to far below fp32
+// resolution of the result: u < -40 gives GELU = -0 and GELU' = 0 (true values
+// below 1e-32 in magnitude), u > 40 gives GELU = h and GELU' = 1 (exact in fp32);
+// both hold for any h, however large (h^3 may overflow to infinity).
 constexpr float kGeluC = 0.7978845608028654f;  // sqrt(2/pi)
 constexpr float kGeluK = 0.044715f;
 __device__ __forceinline__ float gelu_tanh(float h) {
-  const float u = fmaxf(kGeluC * (h + kGeluK * h * h * h), -40.0f);
+  const float u = kGeluC * (h + kGeluK * h * h * h);
+  if (u > 40.0f) return h;
+  if (u < -40.0f) return h * 0.0f;
   return __fdividef(h, 1.0f + __expf(-2.0f * u));
 }
 __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg) {
-  const float u = fmaxf(kGeluC * (h + kGeluK * h * h * h), -40.0f);
+  const float u = kGeluC * (h + kGeluK * h * h * h);
+  if (u > 40.0f) {
+    *g = h;
+    *dg = 1.0f;
+    return;
+  }
+  if (u < -40.0f) {
+    *g = h * 0.0f;
+    *dg = 0.0f;
+    return;
+  }
   const float e = __expf(-2.0f * u);
   const float s = __fdividef(1.0f, 1.0f + e);
   *g = h * s;
@@ -460,6 +580,27 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as
 __device__ __forceinline__ float max16_same_parity(float a, int lane) {
   const unsigned mask = (lane & 1) ? 0xAAAAAAAAu : 0x55555555u;
   return __uint_as_float(__reduce_max_sync(mask, __float_as_uint(a)));
+}
+
+// Launch as clusters of two CTAs along x, with programmatic stream serialization.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                   Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // Launch with programmatic stream serialization (see pdl_wait_prior).

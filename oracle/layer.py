@@ -97,16 +97,27 @@ _GELU_K = 0.044715
 
 
 def gelu_tanh(h):
-    """GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3)))."""
+    """GELU, tanh form: 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))).
+
+    Evaluated through the identity 0.5 (1 + tanh u) = 1 / (1 + e^{-2u}): the same
+    function, without the cancellation of 1 + tanh u for very negative u (which
+    in float64 loses every digit below u ~ -18)."""
     h = _f64(h)
-    return 0.5 * h * (1.0 + np.tanh(_GELU_C * (h + _GELU_K * h ** 3)))
+    u = _GELU_C * (h + _GELU_K * h ** 3)
+    with np.errstate(over="ignore"):
+        return h / (1.0 + np.exp(-2.0 * u))
 
 
 def gelu_tanh_grad(h):
-    """d/dh of gelu_tanh, closed form."""
+    """d/dh of gelu_tanh, closed form: with s = 0.5 (1 + tanh u) = 1 / (1 + e^{-2u}),
+    1 - tanh(u)^2 = 4 s (1 - s) and 1 - s = 1 / (1 + e^{2u}), so
+    GELU'(h) = s + 2 h s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 h^2)."""
     h = _f64(h)
-    t = np.tanh(_GELU_C * (h + _GELU_K * h ** 3))
-    return 0.5 * (1.0 + t) + 0.5 * h * (1.0 - t * t) * _GELU_C * (1.0 + 3.0 * _GELU_K * h * h)
+    u = _GELU_C * (h + _GELU_K * h ** 3)
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-2.0 * u))
+        sc = 1.0 / (1.0 + np.exp(2.0 * u))
+    return s + 2.0 * h * s * sc * _GELU_C * (1.0 + 3.0 * _GELU_K * h * h)
 
 
 def mlp_fwd(X, fc1, fc2, a_f32=None):

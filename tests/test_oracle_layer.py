@@ -177,6 +177,52 @@ def test_gelu_matches_torch():
     np.testing.assert_allclose(layer.gelu_tanh_grad(h), th.grad.numpy(), rtol=1e-12, atol=1e-14)
 
 
+_PI = "3.14159265358979323846264338327950288419716939937510582097494459"
+
+
+def _gelu_exact(x):
+    """The textbook tanh form 0.5 x (1 + tanh u), u = sqrt(2/pi) (x + 0.044715 x^3),
+    in the current decimal context (tanh from exp), with enough digits that
+    1 + tanh u keeps its own significant digits where float64 has none left."""
+    import decimal
+    D = decimal.Decimal
+    u = (D(2) / D(_PI)).sqrt() * (x + D("0.044715") * x ** 3)
+    e2 = (2 * u).exp()
+    return D("0.5") * x * (1 + (e2 - 1) / (e2 + 1))
+
+
+def test_gelu_against_high_precision_textbook_form():
+    """Relative agreement with the 120-digit evaluation of 0.5 h (1 + tanh u) from
+    h = -12 (GELU ~ -1e-61, where float64's 1 + tanh u has lost every digit; 120
+    digits keep ~50 of them there) to 12."""
+    import decimal
+    hs = np.concatenate([np.linspace(-12, 12, 241), [-1e-3, 1e-3, -0.75]])
+    for h in hs[hs != 0]:
+        with decimal.localcontext() as ctx:
+            ctx.prec = 120
+            ref = _gelu_exact(decimal.Decimal(float(h)))
+            got = layer.gelu_tanh(np.float64(h))
+            rel = abs((decimal.Decimal(float(got)) - ref) / ref)
+        assert rel < 1e-13, (h, got, ref)
+    assert layer.gelu_tanh(np.float64(0.0)) == 0.0
+    assert layer.gelu_tanh(np.float64(-1e30)) == 0.0 and layer.gelu_tanh(np.float64(1e30)) == 1e30
+
+
+def test_gelu_grad_against_high_precision_difference_quotient():
+    """The closed-form derivative against a central difference of the 120-digit
+    textbook form (step 1e-25, truncation error ~1e-50), absolute error relative
+    to 1 + |h|^3 (the size of the derivative's terms; it crosses zero near -0.75)."""
+    import decimal
+    for h in np.linspace(-10, 10, 101):
+        with decimal.localcontext() as ctx:
+            ctx.prec = 120
+            d = decimal.Decimal("1e-25")
+            x = decimal.Decimal(float(h))
+            ref = float((_gelu_exact(x + d) - _gelu_exact(x - d)) / (2 * d))
+        got = layer.gelu_tanh_grad(np.float64(h))
+        assert abs(got - ref) <= 1e-13 * (1.0 + abs(h) ** 3), (h, got, ref)
+
+
 def test_mlp_chain_rule_vs_autograd(monkeypatch):
     """With Q and the bf16 roundings replaced by the identity, mlp_fwd/mlp_bwd must be
     the float64 function FC2(GELU(FC1(X))) and its exact gradient."""
