@@ -357,7 +357,7 @@ int side_stream(SideStream** out) {
 // quantizes GELU(h).
 int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
                 float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
-                int* status, int num_sms, cudaStream_t s) {
+                int* status, int num_sms, cudaStream_t s, bool no_quant = false) {
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
   if (w_mn ? !map_bf16(&tmW, W, R, K, 64) : !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
@@ -380,6 +380,7 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.counters = counters;
   rp.status = status;
   rp.fault_skip_stage = -1;
+  rp.no_quant = no_quant ? 1 : 0;
   return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
 
@@ -401,6 +402,7 @@ struct GemmArgs {
   bool out_bf16;
   const void* h;                // GELU-backward epilogue: saved hidden [M, N]
   void* out2;                   // GELU-backward epilogue: bf16(GELU(h)) [M, N]
+  bool main_bf16;               // 16-bit main product: a_codes = A [M, K], b_codes = B [N, K] bf16
 };
 int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   // The CTA-pair kernel (each CTA loads 128 rows of the B tile) computes the
@@ -410,9 +412,10 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   const bool pair = kUsePairGemm && a.h == nullptr;
   const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(ft::kGemmBN);
   CUtensorMap tmA, tmB, tmA2, tmB2;
-  if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, b_rows) ||
-      !map_bf16(&tmA2, a.A2, a.R2, a.M, 128))
-    return FT_ERR_CUDA;
+  const bool maps_ok = a.main_bf16
+                           ? map_bf16(&tmA, a.a_codes, a.K, a.M, 128) && map_bf16(&tmB, a.b_codes, a.K, a.N, b_rows)
+                           : map_codes(&tmA, a.a_codes, a.K, a.M, 128) && map_codes(&tmB, a.b_codes, a.K, a.N, b_rows);
+  if (!maps_ok || !map_bf16(&tmA2, a.A2, a.R2, a.M, 128)) return FT_ERR_CUDA;
   if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, b_rows) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
     return FT_ERR_CUDA;
   GemmParams gp{};
@@ -431,7 +434,8 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   gp.h = a.h;
   gp.out2 = a.out2;
   gp.status = status;
-  if (pair) return cuda_err(ft::launch_gemm_pair(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
+  gp.main_bf16 = a.main_bf16 ? 1 : 0;
+  if (pair && !a.main_bf16) return cuda_err(ft::launch_gemm_pair(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
   return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
 }
 
@@ -781,6 +785,138 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
     if (st) return st;
   }
   return FT_OK;
+}
+
+// ---------------------------------------------------------------- 16-bit precision variants
+namespace {
+// the layer fields the 16-bit variants use (the low-rank factors; no 4-bit weight)
+int check_layer16(const ft_linear_t* L) {
+  if (!L || !L->D || !L->U) return FT_ERR_INVALID_ARG;
+  if (L->K <= 0 || L->N <= 0 || L->K % 32 || L->N % 32) return FT_ERR_SHAPE;
+  if (L->r_s < 0 || L->r < 16 || L->r_s % 16 || L->r % 16 || L->r > 64 || L->r_s + L->r > 128)
+    return FT_ERR_UNSUPPORTED;
+  if (L->K > (1 << 30) || L->N > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(L->D) || !al16(L->U) || (L->bias && !al16(L->bias))) return FT_ERR_ALIGN;
+  return FT_OK;
+}
+}  // namespace
+
+size_t fourtune_linear_fwd_a16_workspace_size(const ft_linear_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_fwd_a16_workspace_size");
+  if (check_layer16(layer) || M <= 0 || M % 16) return 0;
+  return fwd_layout(layer, M, num_sms_or_default()).total;
+}
+
+size_t fourtune_linear_bwd_g16_workspace_size(const ft_linear_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_bwd_g16_workspace_size");
+  if (check_layer16(layer) || M <= 0 || M % 16) return 0;
+  return bwd_layout(layer, M, num_sms_or_default()).total;
+}
+
+int fourtune_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                int transposed, ft_bf16* out, void* stream) {
+  FT_RANGE("fourtune_dequantize_block16");
+  if (!codes || !scales || !out || (transposed != 0 && transposed != 1)) return FT_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return FT_ERR_SHAPE;
+  if (rows > (1 << 30) || cols > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(out) & 3u) return FT_ERR_ALIGN;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  return cuda_err(ft::launch_dequantize_block16(codes, scales, static_cast<int>(rows), static_cast<int>(cols),
+                                                transposed, out, static_cast<cudaStream_t>(stream)));
+}
+
+int fourtune_linear_fwd_a16(const ft_linear_t* layer, const ft_bf16* W16, const ft_bf16* X, int64_t M, void* Y,
+                            int y_dtype, ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_fwd_a16");
+  int st = check_layer16(layer);
+  if (st) return st;
+  if (!W16 || !X || !Y || !L_saved || !ws) return FT_ERR_INVALID_ARG;
+  if (y_dtype != FT_DTYPE_F32 && y_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(W16) || !al16(X) || !al16(Y) || !al16(L_saved) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const FwdWs w = fwd_layout(layer, M, di.num_sms);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
+  // L = bf16(X D) only (the activation is not quantized)
+  st = run_rowpass(X, M, K, layer->D, R, true, false, nullptr, nullptr, nullptr, nullptr, L_saved,
+                   reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                   di.num_sms, s, true);
+  if (st) return st;
+  GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.R2 = R;
+  g.a_codes = reinterpret_cast<const uint8_t*>(X);
+  g.b_codes = reinterpret_cast<const uint8_t*>(W16);
+  g.main_bf16 = true;
+  g.transposed = false;
+  g.A2 = L_saved;
+  g.B2 = layer->U;
+  g.bias = layer->bias;
+  g.out = Y;
+  g.out_bf16 = y_dtype == FT_DTYPE_BF16;
+  return run_gemm(g, status, di.num_sms, s);
+}
+
+int fourtune_linear_bwd_g16(const ft_linear_t* layer, const ft_bf16* W16_t, const ft_bf16* dY, const ft_bf16* X,
+                            const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA, float* dB,
+                            int accumulate, void* ws, size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_bwd_g16");
+  int st = check_layer16(layer);
+  if (st) return st;
+  if (!W16_t || !dY || !X || !L_saved || !dX || !dA || !dB || !ws) return FT_ERR_INVALID_ARG;
+  if (dx_dtype != FT_DTYPE_F32 && dx_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(W16_t) || !al16(dY) || !al16(X) || !al16(L_saved) || !al16(dX) || !al16(dA) || !al16(dB) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const BwdWs w = bwd_layout(layer, M, di.num_sms);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
+  void* P = base + w.P;
+  // P = bf16(G U^T) only (the gradient is not quantized)
+  st = run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, nullptr, nullptr, nullptr, P,
+                   reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                   di.num_sms, s, true);
+  if (st) return st;
+  GemmArgs g{};
+  g.M = M;
+  g.N = K;
+  g.K = N;
+  g.R2 = R;
+  g.a_codes = reinterpret_cast<const uint8_t*>(dY);
+  g.b_codes = reinterpret_cast<const uint8_t*>(W16_t);
+  g.main_bf16 = true;
+  g.transposed = true;
+  g.A2 = P;
+  g.B2 = layer->D;
+  g.out = dX;
+  g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
+  if (w.g.side_sms == 0) {
+    if ((st = run_grads(layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, false, base, status, s)))
+      return st;
+    return run_gemm(g, status, di.num_sms, s);
+  }
+  return gemm_and_grads_side(g, layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, di.num_sms,
+                             s);
 }
 
 // ---------------------------------------------------------------- MLP

@@ -417,6 +417,13 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
+// one E2M1 code (low 4 bits) -> its value, by the hardware conversion
+__device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
+  uint32_t h2;
+  const uint16_t c = static_cast<uint16_t>(code & 0xFu);
+  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u16 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "h"(c));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
 // eight floats -> 32 bits of E2M1 codes, element i in bits 4i..4i+3: the
 // hardware conversion rounds to nearest even, saturates at +-6 and keeps the
 // sign of zero (the parity tests check every E2M1 tie, both signs, against the

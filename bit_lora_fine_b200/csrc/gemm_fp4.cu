@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
   static_assert((3 * kGmStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = (p.K + 255) / 256;       // FP4 K-blocks
+  const bool bf16main = !kCp && p.main_bf16;   // 16-bit main product: 64-wide bf16 K-blocks, no scales
+  const int KB = bf16main ? (p.K + 63) / 64 : (p.K + 255) / 256;   // main-product K-blocks
   const int KS = (p.K + 63) / 64;         // 64-wide k-steps: scale blocks per 128-row chunk
   const int EB = (p.R2 + 63) / 64;        // bf16 low-rank blocks
   const int T = KB + EB;                  // pipeline stages per tile
@@ -208,8 +209,10 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
             } else {
               mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
             }
-            tma_load_2d(st, &tmA, &full[s], i * 128, m0);
-            tma_load_2d(st + Lay::kA, &tmB, &full[s], i * 128, n0);
+            // a K-block is 128 bytes of each row: 256 FP4 codes or 64 bf16 values
+            const int kx = bf16main ? i * 64 : i * 128;
+            tma_load_2d(st, &tmA, &full[s], kx, m0);
+            tma_load_2d(st + Lay::kA, &tmB, &full[s], kx, n0);
           } else {
             const int e = i - KB;
             mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
@@ -234,6 +237,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     if (lane == 0) {
       const uint32_t idesc4 = idesc_fp4_block16(128, BN);
       const uint32_t idesc16 = idesc_bf16(128, BN, false, p.b2_mn_major != 0);
+      const uint32_t idesc16k = idesc_bf16(128, BN, false, false);
       int g = 0, j = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++j) {
@@ -251,7 +255,12 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * Lay::kStage);
           const uint32_t b_addr = a_addr + Lay::kA;
-          if (i < KB) {
+          if (i < KB && bf16main) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              mma_bf16(tmem, desc_kmajor_sw128(a_addr + 32 * t), desc_kmajor_sw128(b_addr + 32 * t), idesc16k,
+                       (i | t) != 0 ? 1u : 0u);
+          } else if (i < KB) {
             const int nks = min(4, KS - 4 * i);
             const uint32_t sfa_addr = b_addr + Lay::kB;
             const uint32_t sfb_addr = sfa_addr + Lay::kSFA;
@@ -364,7 +373,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     auto fetch = [&](int gg, uint32_t (&a)[4], uint32_t (&b)[NB]) {
       const int tile = bx + (gg / T) * gx;
       const int i = gg % T;
-      const int nks = i < KB ? min(4, KS - 4 * i) : 0;
+      const int nks = (i < KB && !bf16main) ? min(4, KS - 4 * i) : 0;
       const int mc = tile / tiles_n, nc = (tile % tiles_n) * Lay::kNC;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -396,7 +405,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       okw = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
       if (!okw) return false;
       tc_fence_after();
-      if (gg % T < KB) {
+      if (gg % T < KB && !bf16main) {
         const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
         uint32_t a16[16];
 #pragma unroll
@@ -517,7 +526,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
-  if (p.epi_gelu_bwd && !p.out_bf16) return cudaErrorInvalidValue;
+  if (p.epi_gelu_bwd && (!p.out_bf16 || p.main_bf16)) return cudaErrorInvalidValue;
   auto kernel = p.epi_gelu_bwd ? gemm_fp4_kernel<BN, true> : gemm_fp4_kernel<BN, false>;
   const uint32_t smem = p.epi_gelu_bwd ? GemmLayout<BN, true>::kSmem : GemmLayout<BN, false>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

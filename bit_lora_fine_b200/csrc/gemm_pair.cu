@@ -21,9 +21,17 @@
 //               and both CTAs' TMA completions (each CTA's loads name the
 //               leader's barrier)
 //   empty[s]    each CTA's: the leader's MMA commit, multicast to both
-//   sf_full[s]  leader's: one arrive per scale warp of both CTAs (8)
+//   sf_full[s]  leader's: one arrive per leader scale warp (4) and one
+//               forwarded from the peer (below)
 //   acc_full    each CTA's: the leader's commit after a tile's last MMA
-//   acc_empty   leader's: one arrive per epilogue warp of both CTAs (16)
+//   acc_empty   leader's: one arrive per leader epilogue warp (8) and one
+//               forwarded from the peer
+// The peer's scale and epilogue warps arrive on barriers of their own CTA
+// (sf_ready[s], acc_done), and one otherwise idle thread of the peer forwards
+// each completed phase to the leader.  An arrive with cluster-scope release
+// waits for every memory operation its thread has in flight -- for a scale
+// warp, the next stage's scale loads -- so the warps that keep loads in flight
+// only ever release at CTA scope.
 // Each CTA's four scale warps write its own tensor memory: A's scales of its
 // 128 rows and B's scales of all 256 columns of the tile (the layout of the
 // single-CTA kernel).  Every wait is bounded (see common.cuh); both CTAs meet
@@ -91,10 +99,12 @@ __global__ void __launch_bounds__(kPrThreads, 1)
   uint64_t* acc_full = sf_full + kPrStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* sf_ready = mma_done + 1;         // [kPrStages] peer only: its scale warps
+  uint64_t* acc_done = sf_ready + kPrStages; // peer only: its epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   volatile int* abortp = abort_flag;
-  static_assert((3 * kPrStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
+  static_assert((4 * kPrStages + 4) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -112,10 +122,12 @@ __global__ void __launch_bounds__(kPrThreads, 1)
     for (int s = 0; s < kPrStages; ++s) {
       mbar_init(&full[s], 1);      // leader's producer (expect_tx of both CTAs' bytes)
       mbar_init(&empty[s], 1);     // leader's MMA commit
-      mbar_init(&sf_full[s], 8);   // the scale warps of both CTAs
+      mbar_init(&sf_full[s], 5);   // the leader's 4 scale warps + the peer's forwarded arrive
+      mbar_init(&sf_ready[s], 4);  // the peer's scale warps
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 16);      // the epilogue warps of both CTAs
+    mbar_init(acc_empty, 9);       // the leader's 8 epilogue warps + the peer's forwarded arrive
+    mbar_init(acc_done, 8);        // the peer's epilogue warps
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -231,7 +243,6 @@ __global__ void __launch_bounds__(kPrThreads, 1)
     const int q = warp & 3;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const int G = (pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0) * T;
-    const uint32_t sf_full0 = cluster_addr(&sf_full[0], 0);
     auto fetch = [&](int gg, uint32_t (&a)[4], uint32_t (&b)[32]) {
       const int tile = pair + (gg / T) * npairs;
       const int i = gg % T;
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kPrThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(sf_full0 + 8u * s);
+      if (lane == 0) mbar_arrive(rank == 0 ? &sf_full[s] : &sf_ready[s]);
       return true;
     };
     // two register sets: stage gg+1's loads are in flight while stage gg is stored
@@ -295,7 +306,7 @@ __global__ void __launch_bounds__(kPrThreads, 1)
     const int q = warp & 3;
     const int c_lo = ((warp - 4) >> 2) * (kPrBN / 2);
     const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c_lo);
-    const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+    uint64_t* acc_free = rank == 0 ? acc_empty : acc_done;   // the peer's are forwarded
     uint8_t* buf = epi + (warp - 4) * 1024;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const long long ldb = p.ldo * (p.out_bf16 ? 2 : 4);   // output row stride in bytes
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(kPrThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty0);
+        if (lane == 0) mbar_arrive(acc_free);
         if (rows_left > 0) {
 #pragma unroll
           for (int c = 0; c < kPrBN / 32; ++c) {
@@ -370,8 +381,25 @@ __global__ void __launch_bounds__(kPrThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty0);
+        if (lane == 0) mbar_arrive(acc_free);
       }
+    }
+  } else if (warp == 2 && lane == 0 && rank == 1) {
+    // the peer's forwarder of its scale warps' phases to the leader's sf_full
+    const int G = (pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0) * T;
+    const uint32_t sf_full0 = cluster_addr(&sf_full[0], 0);
+    for (int gg = 0; gg < G; ++gg) {
+      const int s = gg % kPrStages;
+      if (!mbar_wait(&sf_ready[s], (gg / kPrStages) & 1, p.status, abortp)) break;
+      mbar_arrive_remote(sf_full0 + 8u * s);
+    }
+  } else if (warp == 3 && lane == 0 && rank == 1) {
+    // ... and of its epilogue warps' phases to the leader's acc_empty
+    const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+    int j = 0;
+    for (int tile = pair; tile < tiles; tile += npairs, ++j) {
+      if (!mbar_wait(acc_done, j & 1, p.status, abortp)) break;
+      mbar_arrive_remote(acc_empty0);
     }
   }
 

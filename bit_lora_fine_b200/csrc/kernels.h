@@ -17,6 +17,7 @@ struct RowpassParams {
   int stages;                            // TMA ring depth, 2..rowpass_stages()
   int gelu_input;                        // input is h: quantize a = GELU(h) (fp32) and project bf16(a)
   float* dbg_a;                          // gelu_input: optional fp32 copy of a [M, K] (null = none)
+  int no_quant;                          // only L: no codes or scales (the 16-bit precision variants)
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
   uint8_t* sf_mma;                       // the same scales in the MMA-ready layout (null = not written)
@@ -60,6 +61,9 @@ struct GemmParams {
   const void* h;
   void* out2;
   int* status;
+  // 16-bit main product (the precision variants): A [M, K] and B [N, K] are
+  // bf16 (K contiguous) instead of block16 codes; sfa, sfb unused
+  int main_bf16;
 };
 
 // out[p, j] (+)= sum_m T[m, p] * V[m, v0 + j]   for p < P, j < r (r <= 64)
@@ -78,6 +82,9 @@ cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long
                                     uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_quantize_block16_f32(const float* x, int rows, int cols, long long ld, uint8_t* codes,
                                         uint8_t* scales, cudaStream_t stream);
+// bf16 values of a block16 matrix (or of its transpose), see quant.cu
+cudaError_t launch_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int rows, int cols,
+                                      int transposed, void* out, cudaStream_t stream);
 cudaError_t launch_transpose_codes(const uint8_t* codes, int rows, int cols, uint8_t* codes_t,
                                    cudaStream_t stream);
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,

@@ -249,4 +249,52 @@ cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transpo
   return cudaGetLastError();
 }
 
+// Dequantized values of a block16 matrix [rows, cols] as bf16: value =
+// E2M1(code) * E4M3(scale of its 16x16 block), exact in bf16 (at most 2 + 4
+// significant bits, magnitudes 2^-10 .. 2688).  transposed = 0 writes
+// out[r, c] [rows, cols]; transposed = 1 writes the transpose out[c, r]
+// [cols, rows] (FourTune §3.2: the transposed operand keeps its codes and
+// scales).  One thread per pair of output elements (a byte of codes when not
+// transposed).  The 16-bit precision variants (§4.3) use it to give their GEMMs
+// the 4-bit weight as the tensor cores would see it.
+__global__ void dequantize_block16_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                          int rows, int cols, int transposed, uint32_t* __restrict__ out,
+                                          long long npairs) {
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= npairs) return;
+  float v[2];
+  if (!transposed) {
+    // output pair i = row r, columns 2j, 2j+1 = one code byte
+    const long long r = i / (cols / 2);
+    const int j = static_cast<int>(i % (cols / 2));
+    const float d = e4m3_to_f32(scales[(r / 16) * (cols / 16) + (2 * j) / 16]);
+    const uint32_t byte = codes[i];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) v[e] = e2m1_to_f32((byte >> (4 * e)) & 0xFu) * d;
+  } else {
+    // output pair i = output row c (an input column), output columns 2j, 2j+1
+    // (input rows 2j, 2j+1, one 16-row block)
+    const long long c = i / (rows / 2);
+    const int j = static_cast<int>(i % (rows / 2));
+    const float d = e4m3_to_f32(scales[((2 * j) / 16) * (cols / 16) + c / 16]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const uint32_t byte = codes[static_cast<long long>(2 * j + e) * (cols / 2) + c / 2];
+      v[e] = e2m1_to_f32((byte >> (4 * (c & 1))) & 0xFu) * d;
+    }
+  }
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v[0], v[1]);
+  out[i] = *reinterpret_cast<const uint32_t*>(&b);
+}
+
+cudaError_t launch_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int rows, int cols,
+                                      int transposed, void* out, cudaStream_t stream) {
+  const long long npairs = static_cast<long long>(rows) * cols / 2;
+  if (npairs == 0) return cudaSuccess;
+  const int threads = 256;
+  dequantize_block16_kernel<<<static_cast<unsigned>((npairs + threads - 1) / threads), threads, 0, stream>>>(
+      codes, scales, rows, cols, transposed, static_cast<uint32_t*>(out), npairs);
+  return cudaGetLastError();
+}
+
 }  // namespace ft

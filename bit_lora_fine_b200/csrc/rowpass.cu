@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       const float amax = max16_same_parity(m[0], lane);   // over the block's 16 rows
       const int cstart = (kt0 + i) * 64 + colw;
       const bool inside = block_row_ok && cstart < p.K;
-      if (inside || p.sf_mma) {
+      if (!p.no_quant && (inside || p.sf_mma)) {
         // rows past M and columns past K were zero-filled by the TMA: their scale is 0
         uint32_t packed[2], sc;
         if (GELU)

@@ -28,7 +28,12 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_mlp_bwd_workspace_size", "fourtune_mlp_bwd", "fourtune_mlp_fwd_ws_offsets",
             "fourtune_mlp_bwd_ws_offsets", "fourtune_mma_scales_size", "fourtune_mma_scales",
             "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32",
-            "fourtune_quant_down_static_status", "fourtune_test_wait_timeout")
+            "fourtune_quant_down_static_status", "fourtune_test_wait_timeout", "fourtune_dequantize_block16",
+            "fourtune_linear_fwd_a16", "fourtune_linear_bwd_g16", "fourtune_linear_fwd_a16_workspace_size",
+            "fourtune_linear_bwd_g16_workspace_size")
+SIZE_FUNCS = ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size", "fourtune_mma_scales_size",
+              "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
+              "fourtune_linear_fwd_a16_workspace_size", "fourtune_linear_bwd_g16_workspace_size")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
@@ -99,11 +104,16 @@ def load():
     L.fourtune_mlp_bwd_timed.argtypes = list(L.fourtune_mlp_bwd.argtypes) + [P(vp), ctypes.c_int]
     L.fourtune_mlp_fwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz)]
     L.fourtune_mlp_bwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz), P(sz), P(sz)]
+    L.fourtune_dequantize_block16.argtypes = [vp, vp, i64, i64, ctypes.c_int, vp, vp]
+    L.fourtune_linear_fwd_a16.argtypes = [P(ft_linear_t), vp, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
+    L.fourtune_linear_bwd_g16.argtypes = [P(ft_linear_t), vp, vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, ctypes.c_int,
+                                          vp, sz, vp]
+    L.fourtune_linear_fwd_a16_workspace_size.argtypes = [P(ft_linear_t), i64]
+    L.fourtune_linear_bwd_g16_workspace_size.argtypes = [P(ft_linear_t), i64]
+    for f in SIZE_FUNCS:
+        getattr(L, f).restype = sz
     for f in EXPORTED:
-        if f not in ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size",
-                     "fourtune_mma_scales_size",
-                     "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
-                     "fourtune_error_string"):
+        if f not in SIZE_FUNCS and f != "fourtune_error_string":
             getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L
@@ -444,6 +454,109 @@ def quant_down_static(X, W, codes=None, scales=None, L=None):
     _check(load().fourtune_quant_down_static(_ptr(X), M, K, _ptr(W), R, _ptr(codes), _ptr(scales), _ptr(L),
                                              _stream()), "fourtune_quant_down_static")
     return codes, scales, L
+
+
+def dequantize_block16(codes, scales, rows, cols, transposed=False):
+    """bf16 values of a block16 matrix [rows, cols] (exact), or of its transpose [cols, rows]."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    _shape(codes, (rows, cols // 2), "codes")
+    _shape(scales, (rows // 16, cols // 16), "scales")
+    out = torch.empty((cols, rows) if transposed else (rows, cols), dtype=torch.bfloat16, device=codes.device)
+    _check(load().fourtune_dequantize_block16(_ptr(codes), _ptr(scales), rows, cols, int(transposed), _ptr(out),
+                                              _stream()), "fourtune_dequantize_block16")
+    return out
+
+
+class Linear16:
+    """The 16-bit precision variants' view of a layer (§4.3, Table 4): the low-rank
+    factors D = [S_dn | A], U = [S_up ; B] (bf16), an optional bias, and the weight
+    as bf16 -- W16 [N, K] and its transpose W16_t [K, N].  From a 4-bit Linear,
+    W16 = deq(Q(R)) (from_linear); from a bf16 weight and r_s = 0 it is the
+    standard bf16 LoRA layer (from_bf16_lora)."""
+
+    def __init__(self, W16, W16_t, D, U, r_s, bias=None):
+        self.N, self.K = W16.shape
+        self.r_s, self.r = r_s, D.shape[1] - r_s
+        for t, n in ((W16, "W16"), (W16_t, "W16_t"), (D, "D"), (U, "U"), (bias, "bias")):
+            _need(t, torch.bfloat16, n)
+        _shape(W16_t, (self.K, self.N), "W16_t")
+        _shape(D, (self.K, self.r_s + self.r), "D")
+        _shape(U, (self.r_s + self.r, self.N), "U")
+        self.t = dict(W16=W16, W16_t=W16_t, D=D, U=U, bias=bias)
+        self.c = ft_linear_t(self.K, self.N, self.r_s, self.r, None, None, None, _ptr(D), _ptr(U), _ptr(bias),
+                             None, None)
+
+    @classmethod
+    def from_linear(cls, lay):
+        """W16 = deq(Q(R)) of a 4-bit layer, same low-rank factors and bias."""
+        W = dequantize_block16(lay.t["R_codes"], lay.t["R_scales"], lay.N, lay.K)
+        Wt = dequantize_block16(lay.t["R_codes"], lay.t["R_scales"], lay.N, lay.K, transposed=True)
+        return cls(W, Wt, lay.t["D"], lay.t["U"], lay.r_s, lay.t["bias"])
+
+    @classmethod
+    def from_bf16_lora(cls, W, A, B, bias=None):
+        """Standard LoRA: bf16 weight W [N, K], adapter A [K, r], B [r, N], no stabilizer."""
+        return cls(W.contiguous(), W.t().contiguous(), A.contiguous(), B.contiguous(), 0, bias)
+
+    @property
+    def R_all(self):
+        return self.r_s + self.r
+
+    def _ws(self, fn, M):
+        n = fn(ctypes.byref(self.c), M)
+        if n == 0:
+            raise FourtuneError(-2, "fourtune_linear_*16_workspace_size")
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def fwd_workspace(self, M):
+        return self._ws(load().fourtune_linear_fwd_a16_workspace_size, M)
+
+    def bwd_workspace(self, M):
+        return self._ws(load().fourtune_linear_bwd_g16_workspace_size, M)
+
+
+def linear_fwd_a16(layer16, X, y_dtype=torch.float32, ws=None, Y=None, L=None):
+    """16-bit-activation forward: Y = X W16^T + L U + bias, L = bf16(X D).  Returns (Y, L, ws)."""
+    _ndim2(X, "X")
+    M = X.shape[0]
+    _shape(X, (M, layer16.K), "X")
+    _shape(Y, (M, layer16.N), "Y")
+    _shape(L, (M, layer16.R_all), "L")
+    _out_dtype(Y, "Y")
+    _need(X, torch.bfloat16, "X")
+    Y = torch.empty((M, layer16.N), dtype=y_dtype, device=X.device) if Y is None else Y
+    L = torch.empty((M, layer16.R_all), dtype=torch.bfloat16, device=X.device) if L is None else L
+    ws = layer16.fwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if Y.dtype == torch.float32 else FT_DTYPE_BF16
+    _check(load().fourtune_linear_fwd_a16(ctypes.byref(layer16.c), _ptr(layer16.t["W16"]), _ptr(X), M, _ptr(Y), code,
+                                          _ptr(L), _ptr(ws), ws.numel(), _stream()), "fourtune_linear_fwd_a16")
+    return Y, L, ws
+
+
+def linear_bwd_g16(layer16, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumulate=False, ws=None, dX=None):
+    """16-bit-gradient backward: dX = dY W16 + P D^T, dA = X^T P_B, dB = L_B^T dY.  Returns (dX, dA, dB, ws)."""
+    _ndim2(dY, "dY")
+    M = dY.shape[0]
+    _shape(dY, (M, layer16.N), "dY")
+    _shape(X, (M, layer16.K), "X")
+    _shape(L, (M, layer16.R_all), "L")
+    _shape(dX, (M, layer16.K), "dX")
+    _shape(dA, (layer16.K, layer16.r), "dA")
+    _shape(dB, (layer16.r, layer16.N), "dB")
+    _out_dtype(dX, "dX")
+    for t, n in ((dY, "dY"), (X, "X"), (L, "L")):
+        _need(t, torch.bfloat16, n)
+    dev = dY.device
+    dX = torch.empty((M, layer16.K), dtype=dx_dtype, device=dev) if dX is None else dX
+    dA = torch.zeros((layer16.K, layer16.r), dtype=torch.float32, device=dev) if dA is None else dA
+    dB = torch.zeros((layer16.r, layer16.N), dtype=torch.float32, device=dev) if dB is None else dB
+    ws = layer16.bwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if dX.dtype == torch.float32 else FT_DTYPE_BF16
+    _check(load().fourtune_linear_bwd_g16(ctypes.byref(layer16.c), _ptr(layer16.t["W16_t"]), _ptr(dY), _ptr(X),
+                                          _ptr(L), M, _ptr(dX), code, _ptr(dA), _ptr(dB), int(accumulate), _ptr(ws),
+                                          ws.numel(), _stream()), "fourtune_linear_bwd_g16")
+    return dX, dA, dB, ws
 
 
 def _quant_down_shapes(X, W, codes, scales, L):

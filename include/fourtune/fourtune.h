@@ -176,6 +176,36 @@ FT_API int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY
                                      float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
 
+/* Precision variants (§4.3, Table 4: W4A16G4, W4A4G16, W4A16G16 beside the
+ * paper's W4A4G4).  The weight stays the 4-bit R; a 16-bit activation or
+ * gradient enters its product unquantized, so that product runs on the bf16
+ * tensor cores against R's dequantized values:
+ *   fourtune_dequantize_block16: out = deq(codes, scales) as bf16, exact (an
+ *     E2M1 value times an E4M3 scale has at most 6 significant bits):
+ *     [rows, cols], or with transposed = 1 its transpose [cols, rows].  For the
+ *     layer: W16 = deq(Q(R)) [N, K] (transposed = 0 of R_codes/R_scales),
+ *     W16_t = deq(Q(R))^T [K, N] (transposed = 1).  Frozen: prepared once.
+ *     out 4-byte aligned.
+ *   fourtune_linear_fwd_a16: y = X W16^T + L [S_up ; B] (+ bias),
+ *     L = bf16(X [S_dn | A]) -- fourtune_linear_fwd with a 16-bit activation.
+ *   fourtune_linear_bwd_g16: dX = G W16_t^T + P [S_dn | A]^T (G = dY in bf16),
+ *     dA, dB as in fourtune_linear_bwd -- the backward with a 16-bit gradient.
+ * W4A16G4 = _fwd_a16 + fourtune_linear_bwd; W4A4G16 = fourtune_linear_fwd +
+ * _bwd_g16; W4A16G16 = _fwd_a16 + _bwd_g16.  Given a bf16 weight in place of
+ * W16 (and W16_t = its transpose) and r_s = 0, the same two calls are the
+ * standard bf16 LoRA layer the paper compares against (§4.2).  These calls read
+ * only K, N, r_s, r, D, U and bias of the layer (the codes fields may be NULL);
+ * their workspaces are sized by the two *_workspace_size calls below. */
+FT_API size_t fourtune_linear_fwd_a16_workspace_size(const ft_linear_t* layer, int64_t M);
+FT_API size_t fourtune_linear_bwd_g16_workspace_size(const ft_linear_t* layer, int64_t M);
+FT_API int fourtune_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                       int transposed, ft_bf16* out, void* stream);
+FT_API int fourtune_linear_fwd_a16(const ft_linear_t* layer, const ft_bf16* W16, const ft_bf16* X, int64_t M,
+                                   void* Y, int y_dtype, ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream);
+FT_API int fourtune_linear_bwd_g16(const ft_linear_t* layer, const ft_bf16* W16_t, const ft_bf16* dY,
+                                   const ft_bf16* X, const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype,
+                                   float* dA, float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream);
+
 /* The MLP pair (§3.3 "MLP Fusion"): y = FC2(GELU_tanh(FC1(X))), both layers
  * triple-branch, fc1 [K1 -> H], fc2 [H -> N2] (fc1->N == fc2->K).
  * Forward: the X pass and FC1's 4-bit GEMM (+ bias b1) give the hidden

@@ -91,6 +91,39 @@ def linear_bwd(G, X, L, R_codes, R_scales, S_dn, S_up, A, B, Qg=None):
     return dict(dX=dX, dA=dA, dB=dB, P=P, qg_codes=qg_codes, qg_scales=qg_scales)
 
 
+# -------------------------------------------------------------- precision variants
+# §4.3 (Table 4) ablates which tensors are 4-bit: W4A16G4, W4A4G16, W4A16G16 next
+# to W4A4G4.  A 16-bit activation or gradient enters its GEMM unquantized (bf16);
+# the weight is always the 4-bit one, seen by the GEMM as Rq = deq(Q(R)).  The
+# low-rank branches are the same as in linear_fwd / linear_bwd.  With a bf16
+# weight in place of Rq and no stabilizer (r_s = 0), the 16-bit forward and
+# backward are the standard bf16 LoRA layer the pages compare against (§4.2).
+
+def linear_fwd_a16(X, Rq, S_dn, S_up, A, B, bias=None):
+    """Forward with a 16-bit activation: y = X Rq^T + L [S_up ; B] (+ bias),
+    L = bf16(X [S_dn | A]).  Rq [N, K] in float64 (exact values).
+    Returns dict(y, L)."""
+    X = _f64(X)
+    L = formats.bf16_round(X @ _D(S_dn, A))
+    y = X @ _f64(Rq).T + L @ _U(S_up, B)
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return dict(y=y, L=L)
+
+
+def linear_bwd_g16(G, X, L, Rq, S_dn, S_up, A, B):
+    """Backward with a 16-bit gradient: dX = G Rq + P [S_dn | A]^T with
+    P = bf16(G [S_up ; B]^T); dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G as in
+    linear_bwd.  Returns dict(dX, dA, dB, P)."""
+    G = _f64(G)
+    X = _f64(X)
+    L = _f64(L)
+    r_s = np.asarray(S_dn).shape[1]
+    P = formats.bf16_round(G @ _U(S_up, B).T)
+    dX = G @ _f64(Rq) + P @ _D(S_dn, A).T
+    return dict(dX=dX, dA=X.T @ P[:, r_s:], dB=L[:, r_s:].T @ G, P=P)
+
+
 # ------------------------------------------------------------------------- MLP
 _GELU_C = np.sqrt(2.0 / np.pi)
 _GELU_K = 0.044715

@@ -168,6 +168,74 @@ def test_frozen_parts_get_no_gradient():
     assert not ({"dR", "dS_dn", "dS_up", "dbias"} & set(b))   # §3.2: only the adapter updates
 
 
+def test_16bit_variants_equal_triple_loops():
+    """W4A16 forward and G16 backward (§4.3, Table 4) on unquantized bf16-like
+    operands against triple loops (the activation / gradient is not quantized)."""
+    rng = np.random.default_rng(5)
+    M, K, N, r_s, r = 16, 32, 16, 2, 3
+    f = lambda *s: formats.bf16_round(rng.standard_normal(s))
+    X, G, Rq = f(M, K), f(M, N), f(N, K)
+    S_dn, A, S_up, B = f(K, r_s), f(K, r), f(r_s, N), f(r, N)
+    D, U = np.concatenate([S_dn, A], 1), np.concatenate([S_up, B], 0)
+    o = layer.linear_fwd_a16(X, Rq, S_dn, S_up, A, B)
+    L = np.zeros((M, r_s + r))
+    for m in range(M):
+        for j in range(r_s + r):
+            L[m, j] = sum(X[m, k] * D[k, j] for k in range(K))
+    L = formats.bf16_round(L)
+    np.testing.assert_array_equal(o["L"], L)
+    y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            y[m, n] = sum(X[m, k] * Rq[n, k] for k in range(K)) + sum(L[m, j] * U[j, n] for j in range(r_s + r))
+    np.testing.assert_allclose(o["y"], y, rtol=1e-13, atol=1e-13)
+    b = layer.linear_bwd_g16(G, X, L, Rq, S_dn, S_up, A, B)
+    P = np.zeros((M, r_s + r))
+    for m in range(M):
+        for j in range(r_s + r):
+            P[m, j] = sum(G[m, n] * U[j, n] for n in range(N))
+    P = formats.bf16_round(P)
+    np.testing.assert_array_equal(b["P"], P)
+    dX = np.zeros((M, K))
+    for m in range(M):
+        for k in range(K):
+            dX[m, k] = sum(G[m, n] * Rq[n, k] for n in range(N)) + sum(P[m, j] * D[k, j] for j in range(r_s + r))
+    np.testing.assert_allclose(b["dX"], dX, rtol=1e-13, atol=1e-13)
+    dA = np.array([[sum(X[m, k] * P[m, r_s + j] for m in range(M)) for j in range(r)] for k in range(K)])
+    dB = np.array([[sum(L[m, r_s + j] * G[m, n] for m in range(M)) for n in range(N)] for j in range(r)])
+    np.testing.assert_allclose(b["dA"], dA, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(b["dB"], dB, rtol=1e-13, atol=1e-13)
+
+
+def test_16bit_variants_coincide_with_4bit_on_lossless_operands():
+    """When X and G are exactly representable in block16 FP4 (quantization is the
+    identity), every precision variant is the W4A4G4 layer, exactly."""
+    c = make_case(seed=4)
+    Rq = block16.dequantize(c["Rc"], c["Rs"])
+    o4, o16 = fwd(c), layer.linear_fwd_a16(c["X"], Rq, c["S_dn"], c["S_up"], c["A"], c["B"])
+    np.testing.assert_array_equal(o16["y"], o4["y"])
+    np.testing.assert_array_equal(o16["L"], o4["L"])
+    b4 = bwd(c, o4["L"])
+    b16 = layer.linear_bwd_g16(c["G"], c["X"], o4["L"], Rq, c["S_dn"], c["S_up"], c["A"], c["B"])
+    for k in ("dX", "dA", "dB", "P"):
+        np.testing.assert_array_equal(b16[k], b4[k])
+
+
+def test_16bit_variants_differ_from_4bit_on_generic_operands():
+    """On operands that are not on the FP4 grid, the 16-bit activation path does not
+    see the quantization error: its difference from W4A4 is the 4-bit branch's
+    (Q(X) - X) R^T, exactly."""
+    rng = np.random.default_rng(6)
+    c = make_case(seed=6)
+    X = formats.bf16_round(rng.standard_normal(c["X"].shape))
+    Rq = block16.dequantize(c["Rc"], c["Rs"])
+    o4 = layer.linear_fwd(X, c["Rc"], c["Rs"], c["S_dn"], c["S_up"], c["A"], c["B"])
+    o16 = layer.linear_fwd_a16(X, Rq, c["S_dn"], c["S_up"], c["A"], c["B"])
+    Xq = block16.dequantize(o4["qx_codes"], o4["qx_scales"])
+    assert np.abs(Xq - X).max() > 0
+    np.testing.assert_allclose(o4["y"] - o16["y"], (Xq - X) @ Rq.T, rtol=1e-12, atol=1e-12)
+
+
 def test_gelu_matches_torch():
     h = np.linspace(-9, 9, 20001)
     th = torch.tensor(h, requires_grad=True)
