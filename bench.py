@@ -426,6 +426,13 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extra:
         line["configs_extra"] = measure_extra(ft, synth, dev, flush, peaks, steps=max(3, min(args.steps, 10)),
                                               warmup=max(1, min(args.warmup, 3)))
+        v = measure_variants(ft, synth, dev, flush, steps=max(3, min(args.steps, 10)), warmup=max(1, min(args.warmup, 3)))
+        ours_ms = total_ms / args.steps
+        for rec in v["variants"].values():
+            rec["fourtune_speedup"] = rec["ms_per_step"] / ours_ms
+        v["note"] = ("fourtune_speedup = variant step time / the fused W4A4G4 step time of this line "
+                     "(ms_per_step); the bf16 LoRA layer has no stabilizer (rank-32 adapter only)")
+        line["variants"] = v
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, flop_s = time_oracle(M, repeats=1)
         t = min(times)
@@ -533,6 +540,106 @@ def measure_extra(ft, synth, dev, flush, peaks, steps, warmup):
         }
         del layers, step
         torch.cuda.empty_cache()
+    return out
+
+
+def measure_variants(ft, synth, dev, flush, steps, warmup):
+    """FLUX-width layer (M = 4608, K = N = 3072, ranks 32/32) under the precision
+    variants of the paper's ablation (W4A16G4, W4A4G16, W4A16G16), the standard
+    bf16 LoRA layer (bf16 weight, rank-32 adapter, no stabilizer) on this
+    library's bf16 tensor-core path and through cuBLAS (torch.matmul), and the
+    unfused 4-bit layer (separate quantizer, 4-bit GEMM and cuBLAS low-rank
+    products: the form the paper's LoRA fusion replaces).  Device time of fwd+bwd
+    steps, L2 flushed before each."""
+    import torch
+    wl = synth.WORKLOADS[WORKLOAD]
+    spec = wl.layers[0]
+    M, K, N, r_s, r = wl.M, spec.K, spec.N, spec.r_s, spec.r
+    p = synth.layer_params(spec)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16)
+    bf = torch.bfloat16
+    lay = ft.Linear.from_weights(up(p["R"]), up(p["S_dn"]), up(p["S_up"]), up(p["A"]), up(p["B"]))
+    l16 = ft.Linear16.from_linear(lay)
+    W, A, B = up(p["R"]), up(p["A"]), up(p["B"])
+    lora16 = ft.Linear16.from_bf16_lora(W, A, B)
+    X, dY = up(synth.layer_input(wl)), up(synth.upstream_grad(wl))
+    R = r_s + r
+    Y, L, dX = (torch.empty((M, N), dtype=bf, device=dev), torch.empty((M, R), dtype=bf, device=dev),
+                torch.empty((M, K), dtype=bf, device=dev))
+    dA, dB = torch.zeros((K, r), device=dev), torch.zeros((r, N), device=dev)
+    L0 = torch.empty((M, r), dtype=bf, device=dev)
+    wsf, wsb = lay.fwd_workspace(M), lay.bwd_workspace(M)
+    wsf16, wsb16 = l16.fwd_workspace(M), l16.bwd_workspace(M)
+    wsl_f, wsl_b = lora16.fwd_workspace(M), lora16.bwd_workspace(M)
+    D, U = lay.t["D"], lay.t["U"]
+
+    def w4a16g4():
+        ft.linear_fwd_a16(l16, X, ws=wsf16, Y=Y, L=L)
+        ft.linear_bwd(lay, dY, X, L, ws=wsb, dX=dX, dA=dA, dB=dB)
+
+    def w4a4g16():
+        ft.linear_fwd(lay, X, ws=wsf, Y=Y, L=L)
+        ft.linear_bwd_g16(l16, dY, X, L, ws=wsb16, dX=dX, dA=dA, dB=dB)
+
+    def w4a16g16():
+        ft.linear_fwd_a16(l16, X, ws=wsf16, Y=Y, L=L)
+        ft.linear_bwd_g16(l16, dY, X, L, ws=wsb16, dX=dX, dA=dA, dB=dB)
+
+    def lora_bf16_ours():
+        ft.linear_fwd_a16(lora16, X, ws=wsl_f, Y=Y, L=L0)
+        ft.linear_bwd_g16(lora16, dY, X, L0, ws=wsl_b, dX=dX, dA=dA, dB=dB)
+
+    Wt = W.t()
+
+    def lora_bf16_cublas():
+        Lc = X @ A
+        Yc = torch.addmm(Lc @ B, X, Wt)
+        P = dY @ B.t()
+        dXc = torch.addmm(P @ A.t(), dY, W)
+        dAc = X.t() @ P
+        dBc = Lc.t() @ dY
+        return Yc, dXc, dAc, dBc
+
+    R_sf, R_sf_t = lay.t["R_sf"], lay.t["R_sf_t"]
+    ws_g = torch.empty(256, dtype=torch.uint8, device=dev)
+    r_sl = slice(r_s, R)
+
+    def unfused_w4():
+        # forward: quantizer, 4-bit GEMM, then the low-rank branches as separate products
+        xc, xs, _ = ft.quantize_block16(X)
+        Yu, _ = ft.gemm_block16(xc, ft.mma_scales(xs, M, K), lay.t["R_codes"], R_sf, M, N, K, out_dtype=bf, ws=ws_g)
+        Lu = X @ D
+        Yu.add_(Lu @ U)
+        # backward
+        gc, gs, _ = ft.quantize_block16(dY)
+        dXu, _ = ft.gemm_block16(gc, ft.mma_scales(gs, M, N), lay.t["R_codes_t"], R_sf_t, M, K, N, out_dtype=bf,
+                                 ws=ws_g)
+        P = dY @ U.t()
+        dXu.add_(P @ D.t())
+        dAu = X.t() @ P[:, r_sl]
+        dBu = Lu[:, r_sl].t() @ dY
+        return Yu, dXu, dAu, dBu
+
+    fp4, lr = layer_work(M, K, N, r_s, r)
+    out = {"workload": WORKLOAD, "steps": steps, "flop_per_step": fp4 + lr, "variants": {}}
+    for name, fn in (("W4A16G4", w4a16g4), ("W4A4G16", w4a4g16), ("W4A16G16", w4a16g16),
+                     ("bf16-LoRA ours (bf16 tensor cores)", lora_bf16_ours),
+                     ("bf16-LoRA cuBLAS (torch.matmul)", lora_bf16_cublas),
+                     ("W4A4G4 unfused (quantizer + 4-bit GEMM + cuBLAS low-rank)", unfused_w4)):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        out["variants"][name] = {"ms_per_step": ms, "tokens_per_s": M / (ms / 1e3),
+                                 "tflops_equiv": (fp4 + lr) / (ms / 1e3) / 1e12}
     return out
 
 

@@ -415,9 +415,15 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   const bool maps_ok = a.main_bf16
                            ? map_bf16(&tmA, a.a_codes, a.K, a.M, 128) && map_bf16(&tmB, a.b_codes, a.K, a.N, b_rows)
                            : map_codes(&tmA, a.a_codes, a.K, a.M, 128) && map_codes(&tmB, a.b_codes, a.K, a.N, b_rows);
-  if (!maps_ok || !map_bf16(&tmA2, a.A2, a.R2, a.M, 128)) return FT_ERR_CUDA;
-  if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, b_rows) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
-    return FT_ERR_CUDA;
+  if (!maps_ok) return FT_ERR_CUDA;
+  if (a.R2 == 0) {          // no low-rank blocks: the kernel never reads these maps
+    tmA2 = tmA;
+    tmB2 = tmB;
+  } else {
+    if (!map_bf16(&tmA2, a.A2, a.R2, a.M, 128)) return FT_ERR_CUDA;
+    if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, b_rows) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
+      return FT_ERR_CUDA;
+  }
   GemmParams gp{};
   gp.M = static_cast<int>(a.M);
   gp.N = static_cast<int>(a.N);
@@ -800,6 +806,51 @@ int check_layer16(const ft_linear_t* L) {
   return FT_OK;
 }
 }  // namespace
+
+int fourtune_stabilizer_residual(const ft_bf16* W, int64_t N, int64_t K, const ft_bf16* S_dn, const ft_bf16* S_up,
+                                 int64_t r_s, ft_bf16* R, void* stream) {
+  FT_RANGE("fourtune_stabilizer_residual");
+  if (!W || !S_dn || !S_up || !R) return FT_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return FT_ERR_SHAPE;
+  if (r_s < 1 || r_s > 128 || N > (1 << 30) || K > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  return cuda_err(ft::launch_stabilizer_residual(W, static_cast<int>(N), static_cast<int>(K), S_dn, S_up,
+                                                 static_cast<int>(r_s), R, static_cast<cudaStream_t>(stream)));
+}
+
+int fourtune_gemm_block16(const uint8_t* A_codes, const uint8_t* A_sf, const uint8_t* B_codes, const uint8_t* B_sf,
+                          int64_t M, int64_t N, int64_t K, const ft_bf16* bias, void* out, int out_dtype, void* ws,
+                          size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_gemm_block16");
+  if (!A_codes || !A_sf || !B_codes || !B_sf || !out || !ws) return FT_ERR_INVALID_ARG;
+  if (out_dtype != FT_DTYPE_F32 && out_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 32 || K % 32) return FT_ERR_SHAPE;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(A_codes) || !al16(A_sf) || !al16(B_codes) || !al16(B_sf) || !al16(out) || (bias && !al16(bias)) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  if (ws_bytes < 256) return FT_ERR_WORKSPACE;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ft::launch_clear_words(ws, 256, s) != cudaSuccess) return FT_ERR_CUDA;
+  GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.R2 = 0;
+  g.a_codes = A_codes;
+  g.a_sf = A_sf;
+  g.b_codes = B_codes;
+  g.b_sf = B_sf;
+  g.bias = bias;
+  g.out = out;
+  g.out_bf16 = out_dtype == FT_DTYPE_BF16;
+  return run_gemm(g, static_cast<int*>(ws), di.num_sms, s);
+}
 
 size_t fourtune_linear_fwd_a16_workspace_size(const ft_linear_t* layer, int64_t M) {
   FT_RANGE("fourtune_linear_fwd_a16_workspace_size");

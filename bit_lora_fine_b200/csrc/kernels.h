@@ -82,6 +82,9 @@ cudaError_t launch_quantize_block16(const void* x, int rows, int cols, long long
                                     uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_quantize_block16_f32(const float* x, int rows, int cols, long long ld, uint8_t* codes,
                                         uint8_t* scales, cudaStream_t stream);
+// R = bf16(W - (S_dn S_up)^T) [N, K] (the stabilizer split's residual), see quant.cu
+cudaError_t launch_stabilizer_residual(const void* W, int N, int K, const void* S_dn, const void* S_up, int r_s,
+                                       void* R, cudaStream_t stream);
 // bf16 values of a block16 matrix (or of its transpose), see quant.cu
 cudaError_t launch_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int rows, int cols,
                                       int transposed, void* out, cudaStream_t stream);

@@ -287,6 +287,52 @@ __global__ void dequantize_block16_kernel(const uint8_t* __restrict__ codes, con
   out[i] = *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// Residual weight of the stabilizer split (FourTune §3.1): R[n, k] =
+// bf16(W[n, k] - sum_j S_dn[k, j] S_up[j, n]), the rank-r_s product summed in
+// fp32 and the difference rounded once.  A block of 256 threads covers 16 rows
+// n x 64 columns k; it stages S_up[:, n0:n0+16] and S_dn[k0:k0+64, :] in shared
+// memory (fp32) and each thread computes four outputs of one row.
+constexpr int kResRows = 16, kResCols = 64, kResMaxRank = 128;
+__global__ void __launch_bounds__(256) stabilizer_residual_kernel(const __nv_bfloat16* __restrict__ W, int N, int K,
+                                                                  const __nv_bfloat16* __restrict__ S_dn,
+                                                                  const __nv_bfloat16* __restrict__ S_up, int r_s,
+                                                                  __nv_bfloat16* __restrict__ R) {
+  __shared__ float sup[kResMaxRank][kResRows];
+  __shared__ float sdn[kResCols][kResMaxRank + 1];
+  const int n0 = blockIdx.y * kResRows, k0 = blockIdx.x * kResCols;
+  for (int i = threadIdx.x; i < r_s * kResRows; i += blockDim.x) {
+    const int j = i / kResRows, nn = i % kResRows;
+    sup[j][nn] = n0 + nn < N ? __bfloat162float(S_up[static_cast<long long>(j) * N + n0 + nn]) : 0.0f;
+  }
+  for (int i = threadIdx.x; i < r_s * kResCols; i += blockDim.x) {
+    const int kk = i / r_s, j = i % r_s;
+    sdn[kk][j] = k0 + kk < K ? __bfloat162float(S_dn[static_cast<long long>(k0 + kk) * r_s + j]) : 0.0f;
+  }
+  __syncthreads();
+  const int nn = threadIdx.x / 16, kq = (threadIdx.x % 16) * 4;
+  const int n = n0 + nn;
+  if (n >= N) return;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int k = k0 + kq + e;
+    if (k >= K) break;
+    float acc = 0.0f;
+    for (int j = 0; j < r_s; ++j) acc = fmaf(sdn[kq + e][j], sup[j][nn], acc);
+    const long long o = static_cast<long long>(n) * K + k;
+    R[o] = __float2bfloat16_rn(__bfloat162float(W[o]) - acc);
+  }
+}
+
+cudaError_t launch_stabilizer_residual(const void* W, int N, int K, const void* S_dn, const void* S_up, int r_s,
+                                       void* R, cudaStream_t stream) {
+  if (r_s < 1 || r_s > kResMaxRank) return cudaErrorInvalidValue;
+  const dim3 grid((K + kResCols - 1) / kResCols, (N + kResRows - 1) / kResRows);
+  stabilizer_residual_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(W), N, K, static_cast<const __nv_bfloat16*>(S_dn),
+      static_cast<const __nv_bfloat16*>(S_up), r_s, static_cast<__nv_bfloat16*>(R));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequantize_block16(const uint8_t* codes, const uint8_t* scales, int rows, int cols,
                                       int transposed, void* out, cudaStream_t stream) {
   const long long npairs = static_cast<long long>(rows) * cols / 2;

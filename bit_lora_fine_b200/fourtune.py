@@ -30,7 +30,7 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32",
             "fourtune_quant_down_static_status", "fourtune_test_wait_timeout", "fourtune_dequantize_block16",
             "fourtune_linear_fwd_a16", "fourtune_linear_bwd_g16", "fourtune_linear_fwd_a16_workspace_size",
-            "fourtune_linear_bwd_g16_workspace_size")
+            "fourtune_linear_bwd_g16_workspace_size", "fourtune_stabilizer_residual", "fourtune_gemm_block16")
 SIZE_FUNCS = ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size", "fourtune_mma_scales_size",
               "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
               "fourtune_linear_fwd_a16_workspace_size", "fourtune_linear_bwd_g16_workspace_size")
@@ -105,6 +105,8 @@ def load():
     L.fourtune_mlp_fwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz)]
     L.fourtune_mlp_bwd_ws_offsets.argtypes = [PL, PL, i64, P(sz), P(sz), P(sz), P(sz)]
     L.fourtune_dequantize_block16.argtypes = [vp, vp, i64, i64, ctypes.c_int, vp, vp]
+    L.fourtune_stabilizer_residual.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
+    L.fourtune_gemm_block16.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, sz, vp]
     L.fourtune_linear_fwd_a16.argtypes = [P(ft_linear_t), vp, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
     L.fourtune_linear_bwd_g16.argtypes = [P(ft_linear_t), vp, vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, ctypes.c_int,
                                           vp, sz, vp]
@@ -454,6 +456,39 @@ def quant_down_static(X, W, codes=None, scales=None, L=None):
     _check(load().fourtune_quant_down_static(_ptr(X), M, K, _ptr(W), R, _ptr(codes), _ptr(scales), _ptr(L),
                                              _stream()), "fourtune_quant_down_static")
     return codes, scales, L
+
+
+def gemm_block16(A_codes, A_sf, B_codes, B_sf, M, N, K, out_dtype=torch.float32, bias=None, out=None, ws=None):
+    """out [M, N] = deq(A) deq(B)^T (+ bias); A, B block16 codes, scales in the MMA-ready
+    layout (mma_scales).  Returns (out, ws)."""
+    for t, n in ((A_codes, "A_codes"), (A_sf, "A_sf"), (B_codes, "B_codes"), (B_sf, "B_sf")):
+        _need(t, torch.uint8, n)
+    _shape(A_codes, (M, K // 2), "A_codes")
+    _shape(B_codes, (N, K // 2), "B_codes")
+    _shape(out, (M, N), "out")
+    _out_dtype(out, "out")
+    out = torch.empty((M, N), dtype=out_dtype, device=A_codes.device) if out is None else out
+    ws = torch.empty(256, dtype=torch.uint8, device=A_codes.device) if ws is None else ws
+    code = FT_DTYPE_F32 if out.dtype == torch.float32 else FT_DTYPE_BF16
+    _check(load().fourtune_gemm_block16(_ptr(A_codes), _ptr(A_sf), _ptr(B_codes), _ptr(B_sf), M, N, K, _ptr(bias),
+                                        _ptr(out), code, _ptr(ws), ws.numel(), _stream()), "fourtune_gemm_block16")
+    return out, ws
+
+
+def stabilizer_residual(W, S_dn, S_up):
+    """R = bf16(W - (S_dn S_up)^T) for W [N, K], S_dn [K, r_s], S_up [r_s, N] (bf16)."""
+    _ndim2(W, "W")
+    N, K = W.shape
+    r_s = S_dn.shape[1] if S_dn.dim() == 2 else -1
+    _shape(S_dn, (K, r_s), "S_dn")
+    _shape(S_up, (r_s, N), "S_up")
+    _same_device(("W", W), ("S_dn", S_dn), ("S_up", S_up))
+    for t, n in ((W, "W"), (S_dn, "S_dn"), (S_up, "S_up")):
+        _need(t, torch.bfloat16, n)
+    R = torch.empty_like(W)
+    _check(load().fourtune_stabilizer_residual(_ptr(W), N, K, _ptr(S_dn), _ptr(S_up), r_s, _ptr(R), _stream()),
+           "fourtune_stabilizer_residual")
+    return R
 
 
 def dequantize_block16(codes, scales, rows, cols, transposed=False):

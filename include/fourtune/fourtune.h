@@ -132,6 +132,31 @@ FT_API size_t fourtune_mma_scales_size(int64_t rows, int64_t cols);
 FT_API int fourtune_mma_scales(const uint8_t* scales, int64_t rows, int64_t cols, int transposed, uint8_t* out,
                                void* stream);
 
+/* Stabilizer split (§3.1: a frozen full-precision low-rank component is
+ * isolated from the backbone weight and only the rest is quantized).  Given the
+ * weight W [N, K] (y = X W^T) and rank-r_s factors S_dn [K, r_s], S_up [r_s, N]
+ * of W^T (bf16; the paper cites SVDQuant, read as the truncated SVD of W^T
+ * with the singular values split evenly between the factors -- a
+ * factorization the caller computes), writes the residual
+ *   R [N, K] = bf16(W - (S_dn S_up)^T)
+ * (the rank-r_s product summed in fp32, the difference rounded once), which
+ * fourtune_quantize_block16 then quantizes.  1 <= r_s <= 128; bf16 arrays
+ * row-major and contiguous.  Run once per frozen weight. */
+FT_API int fourtune_stabilizer_residual(const ft_bf16* W, int64_t N, int64_t K, const ft_bf16* S_dn,
+                                        const ft_bf16* S_up, int64_t r_s, ft_bf16* R, void* stream);
+
+/* The 4-bit product alone, a building block (the unfused form of the layer is
+ * the paper's fusion ablation, §4.3 Fig. 9):
+ *   out [M, N] = deq(A) deq(B)^T (+ bias)
+ * A [M, K] and B [N, K] block16 codes ([rows, K/2] bytes), their scales in the
+ * MMA-ready layout (A_sf = fourtune_mma_scales(A's scales, M, K, 0), B_sf the
+ * same for B; for R^T, R_sf_t).  out fp32 or bf16 row-major (stride N).  ws:
+ * at least 256 bytes, 256-byte aligned (its status word; fourtune_device_status
+ * reads it).  M multiple of 16, N and K of 32. */
+FT_API int fourtune_gemm_block16(const uint8_t* A_codes, const uint8_t* A_sf, const uint8_t* B_codes,
+                                 const uint8_t* B_sf, int64_t M, int64_t N, int64_t K, const ft_bf16* bias, void* out,
+                                 int out_dtype, void* ws, size_t ws_bytes, void* stream);
+
 /* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
 FT_API size_t fourtune_linear_fwd_workspace_size(const ft_linear_t* layer, int64_t M);
 FT_API size_t fourtune_linear_bwd_workspace_size(const ft_linear_t* layer, int64_t M);
