@@ -405,12 +405,7 @@ struct GemmArgs {
   bool main_bf16;               // 16-bit main product: a_codes = A [M, K], b_codes = B [N, K] bf16
 };
 int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
-  // The CTA-pair kernel (each CTA loads 128 rows of the B tile) computes the
-  // same outputs bit for bit but is not yet faster than the single-CTA kernel
-  // (256-row B boxes), which therefore runs every epilogue.
-  constexpr bool kUsePairGemm = false;
-  const bool pair = kUsePairGemm && a.h == nullptr;
-  const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(ft::kGemmBN);
+  const uint32_t b_rows = static_cast<uint32_t>(ft::kGemmBN);
   CUtensorMap tmA, tmB, tmA2, tmB2;
   const bool maps_ok = a.main_bf16
                            ? map_bf16(&tmA, a.a_codes, a.K, a.M, 128) && map_bf16(&tmB, a.b_codes, a.K, a.N, b_rows)
@@ -441,7 +436,6 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   gp.out2 = a.out2;
   gp.status = status;
   gp.main_bf16 = a.main_bf16 ? 1 : 0;
-  if (pair && !a.main_bf16) return cuda_err(ft::launch_gemm_pair(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
   return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
 }
 

@@ -97,11 +97,6 @@ int rowpass_stages(int R, int w_mn_major);
 // persistent: min(tiles, num_sms) CTAs
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream);
-// The same product on CTA pairs (256 x 256 tiles shared by two SMs; plain
-// epilogues only): B's tensor map has boxes of 128 rows (each CTA loads its
-// half of the tile), as has B2's when K-major.  min(tiles, num_sms / 2) pairs.
-cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
-                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream);
 // compact block16 scales -> MMA-ready layout of the operand [rows, cols]; with
 // `transposed`, the operand is the transpose of the quantized matrix, whose
 // compact scales are [cols/16, rows/16]
