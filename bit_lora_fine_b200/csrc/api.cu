@@ -254,30 +254,53 @@ BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
   return w;
 }
 
-// MLP forward: header (status, row-pass counters) | Q(X) | Q(a) | row-pass
-// partials (shared by the two row passes, which run one after the other)
+// Units of the MLP's fused GEMMs (gemm_mlp.cu): a 128-row tile's N tiles split
+// into nsplit runs of `per`; the smallest split whose makespan (tile rounds of
+// the busiest CTA) is within 3 % of the even share of all tiles.
+struct MlpUnits {
+  int nsplit, per;
+};
+MlpUnits plan_units(int64_t M, int64_t N, int num_sms) {
+  const int MT = cdiv(M, 128), NT = cdiv(N, 256);
+  const double ideal = static_cast<double>(MT) * NT / num_sms;
+  for (int ns = 1; ns <= NT; ++ns) {
+    const int per = cdiv(NT, ns);
+    const int nsr = cdiv(NT, per);
+    const double span = static_cast<double>(cdiv(static_cast<int64_t>(MT) * nsr, num_sms)) * per;
+    if (span <= 1.03 * ideal || ns == NT) return {nsr, per};
+  }
+  return {NT, 1};
+}
+size_t proj_part_bytes(int64_t M, int64_t N, int64_t RP, int num_sms) {
+  return static_cast<size_t>(plan_units(M, N, num_sms).nsplit) * static_cast<size_t>(M) * static_cast<size_t>(RP) * 4;
+}
+
+// MLP forward: header (status, row-pass counters, projection counters) | Q(X) |
+// Q(a) | row-pass partials | FC1 projection partials (L2)
 struct MlpFwdWs {
-  size_t header, rp_cnt, rp_part, total;
+  size_t header, rp_cnt, pj_cnt, rp_part, pj_part, total;
   Q16 qx, qa;
 };
 MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, int num_sms) {
   MlpFwdWs w{};
   Carver c;
   w.rp_cnt = 16;
-  c.take(w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128))));
+  w.pj_cnt = w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128));
+  c.take(w.header = up256(w.pj_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qx.carve(c, M, fc1->K);
   w.qa.carve(c, M, fc1->N);
-  w.rp_part = c.take(std::max(rp_part_bytes(M, fc1->K, rank_all(fc1), 1, num_sms),
-                              rp_part_bytes(M, fc1->N, rank_all(fc2), 1, num_sms)));
+  w.rp_part = c.take(rp_part_bytes(M, fc1->K, rank_all(fc1), 1, num_sms));
+  w.pj_part = c.take(proj_part_bytes(M, fc1->N, rank_all(fc2), num_sms));
   w.total = c.o;
   return w;
 }
 
 // MLP backward: header (status, counters of both layers' dA/dB, row-pass
-// counters) | Q(G) | P2 | d_h | bf16(GELU(h)) | Q(d_h) | P1 | dA/dB partials
-// (shared by the two dA/dB launches) | row-pass partials (shared likewise)
+// counters, projection counters) | Q(G) | P2 | d_h | Q(d_h) | P1 | dA/dB
+// partials (shared by the two dA/dB launches) | row-pass partials | FC2-dX
+// projection partials (P1)
 struct MlpBwdWs {
-  size_t header, P2, dh, abf, P1, rp_cnt, rp_part, total;
+  size_t header, P2, dh, P1, rp_cnt, pj_cnt, rp_part, pj_part, total;
   Q16 qg, qdh;
   GradPair g2, g1;
 };
@@ -292,19 +315,19 @@ MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
   w.g1.cntA = w.g2.cntB + 4 * static_cast<size_t>(cdiv(fc2->N, 128));
   w.g1.cntB = w.g1.cntA + 4 * static_cast<size_t>(cdiv(fc1->K, 128));
   w.rp_cnt = 16 + 4 * (grad_counter_words(fc2) + grad_counter_words(fc1));
-  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
+  w.pj_cnt = w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128));
+  c.take(w.header = up256(w.pj_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qg.carve(c, M, fc2->N);
   w.P2 = c.take(static_cast<size_t>(M * rank_all(fc2) * 2));
   w.dh = c.take(static_cast<size_t>(M * H * 2));
-  w.abf = c.take(static_cast<size_t>(M * H * 2));
   w.qdh.carve(c, M, H);
   w.P1 = c.take(static_cast<size_t>(M * rank_all(fc1) * 2));
   const size_t part = c.take(std::max(grad_partial_bytes(w.g2, fc2), grad_partial_bytes(w.g1, fc1)));
   w.g2.partA = w.g1.partA = part;
   w.g2.partB = part + grad_part_a(w.g2, fc2);
   w.g1.partB = part + grad_part_a(w.g1, fc1);
-  w.rp_part = c.take(std::max(rp_part_bytes(M, fc2->N, rank_all(fc2), 0, num_sms),
-                              rp_part_bytes(M, H, rank_all(fc1), 0, num_sms)));
+  w.rp_part = c.take(rp_part_bytes(M, fc2->N, rank_all(fc2), 0, num_sms));
+  w.pj_part = c.take(proj_part_bytes(M, H, rank_all(fc1), num_sms));
   w.total = c.o;
   return w;
 }
@@ -442,7 +465,7 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
 // dA = T_A^T V_A[:, r_s:] ([K, r]) and dB = (L[:, r_s:]^T G) ([r, N]) of one layer, one launch
 int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, const void* G, const void* Lsaved,
               float* dA, float* dB, bool accumulate, const GradPair& g, bool side, uint8_t* base, int* status,
-              cudaStream_t s) {
+              cudaStream_t s, bool x_gelu = false) {
   const MSplit& sa = side ? g.cA : g.sA;
   const MSplit& sb = side ? g.cB : g.sB;
   const int64_t R = rank_all(L);
@@ -457,6 +480,7 @@ int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, con
   ta.accumulate = tb.accumulate = accumulate ? 1 : 0;
   ta.status = tb.status = status;
   ta.P = static_cast<int>(L->K);
+  ta.t_gelu = x_gelu ? 1 : 0;
   ta.mt_per_split = sa.mt_per_split;
   ta.nsplit = sa.nsplit;
   ta.out = dA;
@@ -473,6 +497,62 @@ int run_grads(const ft_linear_t* L, int64_t M, const void* X, const void* P, con
   tb.part = reinterpret_cast<float*>(base + g.partB);
   tb.counters = reinterpret_cast<int*>(base + g.cntB);
   return cuda_err(ft::launch_tgrad2(tmTa, tmVa, ta, tmTb, tmVb, tb, s));
+}
+
+// One of the MLP's fused GEMMs (gemm_mlp.cu): the main product as run_gemm, the
+// epilogue of `epi`, and the projection T Wp -> proj_out (Wp = D2 [N, RP]
+// MN-major for epi 1, U1 [RP, N] K-major for epi 2).
+struct MlpGemmArgs {
+  GemmArgs g;
+  int epi;
+  const void* h;
+  void* out_h;
+  float* dbg;
+  uint8_t *q_codes, *q_scales, *q_sf;
+  const void* Wp;
+  int64_t RP;
+  void* proj_out;
+  float* part;
+  int* counters;
+};
+int run_gemm_mlp(const MlpGemmArgs& m, int* status, int num_sms, cudaStream_t s) {
+  const GemmArgs& a = m.g;
+  CUtensorMap tmA, tmB, tmA2, tmB2, tmW;
+  if (!map_codes(&tmA, a.a_codes, a.K, a.M, 128) || !map_codes(&tmB, a.b_codes, a.K, a.N, ft::kGemmBN) ||
+      !map_bf16(&tmA2, a.A2, a.R2, a.M, 128))
+    return FT_ERR_CUDA;
+  if (a.transposed ? !map_bf16(&tmB2, a.B2, a.R2, a.N, ft::kGemmBN) : !map_bf16(&tmB2, a.B2, a.N, a.R2, 64))
+    return FT_ERR_CUDA;
+  const bool wmn = m.epi == 1;
+  if (wmn ? !map_bf16(&tmW, m.Wp, m.RP, a.N, 64) : !map_bf16(&tmW, m.Wp, a.N, m.RP, static_cast<uint32_t>(m.RP)))
+    return FT_ERR_CUDA;
+  const MlpUnits un = plan_units(a.M, a.N, num_sms);
+  ft::MlpGemmParams mp{};
+  mp.g.M = static_cast<int>(a.M);
+  mp.g.N = static_cast<int>(a.N);
+  mp.g.K = static_cast<int>(a.K);
+  mp.g.R2 = static_cast<int>(a.R2);
+  mp.g.b2_mn_major = a.transposed ? 0 : 1;
+  mp.g.sfa = a.a_sf;
+  mp.g.sfb = a.b_sf;
+  mp.g.bias = a.bias;
+  mp.g.out_bf16 = 1;
+  mp.g.status = status;
+  mp.epi = m.epi;
+  mp.h = m.h;
+  mp.out_h = m.out_h;
+  mp.dbg = m.dbg;
+  mp.q_codes = m.q_codes;
+  mp.q_scales = m.q_scales;
+  mp.q_sf = m.q_sf;
+  mp.RP = static_cast<int>(m.RP);
+  mp.wp_mn_major = wmn ? 1 : 0;
+  mp.nsplit = un.nsplit;
+  mp.per = un.per;
+  mp.part = m.part;
+  mp.counters = m.counters;
+  mp.proj_out = m.proj_out;
+  return cuda_err(ft::launch_gemm_mlp(tmA, tmB, tmA2, tmB2, tmW, mp, num_sms, s));
 }
 
 #define FT_TRY(k, expr)                                          \
@@ -995,7 +1075,7 @@ int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, 
   if (st) return st;
   const MlpBwdWs w = mlp_bwd_layout(fc1, fc2, M, num_sms_or_default());
   if (dh_off) *dh_off = w.dh;
-  if (a_off) *a_off = w.abf;
+  if (a_off) *a_off = SIZE_MAX;   // bf16(GELU(h)) is not stored (recomputed from h where needed)
   if (qdh_codes) *qdh_codes = w.qdh.codes;
   if (qdh_scales) *qdh_scales = w.qdh.scales;
   return FT_OK;
@@ -1032,29 +1112,36 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   int* status = reinterpret_cast<int*>(base);
   if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
-  // FC1: X pass, then 4-bit GEMM + L1 U1 + b1 -> h (bf16, saved)
+  // FC1: X pass (Q(X), L1)
   FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
                         base + w.qx.sf, L1_saved, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
-  GemmArgs g{};
-  g.M = M;
-  g.N = H;
-  g.K = K1;
-  g.R2 = R1;
-  g.a_codes = base + w.qx.codes;
-  g.a_sf = base + w.qx.sf;
-  g.b_codes = fc1->R_codes;
-  g.b_sf = fc1->R_sf;
-  g.A2 = L1_saved;
-  g.B2 = fc1->U;
-  g.bias = fc1->bias;
-  g.out = h_saved;
-  g.out_bf16 = true;
-  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
-  // GELU pass over h: Q(a) of a = GELU(h) and L2 = bf16(bf16(a) D2)
-  FT_TRY(2, run_rowpass(h_saved, M, H, fc2->D, R2, true, true, dbg_a, base + w.qa.codes, base + w.qa.scales,
-                        base + w.qa.sf, L2_saved, reinterpret_cast<float*>(base + w.rp_part),
-                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
+  // FC1's 4-bit GEMM + L1 U1 + b1 with the fused epilogue: h (saved), a =
+  // GELU(h), Q(a) for FC2's 4-bit branch, L2 = bf16(bf16(a) D2) for its low-rank ones
+  MlpGemmArgs m{};
+  m.g.M = M;
+  m.g.N = H;
+  m.g.K = K1;
+  m.g.R2 = R1;
+  m.g.a_codes = base + w.qx.codes;
+  m.g.a_sf = base + w.qx.sf;
+  m.g.b_codes = fc1->R_codes;
+  m.g.b_sf = fc1->R_sf;
+  m.g.A2 = L1_saved;
+  m.g.B2 = fc1->U;
+  m.g.bias = fc1->bias;
+  m.epi = 1;
+  m.out_h = h_saved;
+  m.dbg = dbg_a;
+  m.q_codes = base + w.qa.codes;
+  m.q_scales = base + w.qa.scales;
+  m.q_sf = base + w.qa.sf;
+  m.Wp = fc2->D;
+  m.RP = R2;
+  m.proj_out = L2_saved;
+  m.part = reinterpret_cast<float*>(base + w.pj_part);
+  m.counters = reinterpret_cast<int*>(base + w.pj_cnt);
+  FT_TRY(1, run_gemm_mlp(m, status, di.num_sms, s));
   // FC2: 4-bit GEMM + L2 U2 + b2 -> Y
   GemmArgs g2{};
   g2.M = M;
@@ -1070,7 +1157,7 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g2.bias = fc2->bias;
   g2.out = Y;
   g2.out_bf16 = y_dtype == FT_DTYPE_BF16;
-  FT_TRY(3, run_gemm(g2, status, di.num_sms, s));
+  FT_TRY(2, run_gemm(g2, status, di.num_sms, s));
   return FT_OK;
 }
 
@@ -1110,36 +1197,41 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   void* P2 = base + w.P2;
   void* dh = base + w.dh;
-  void* abf = base + w.abf;
   void* P1 = base + w.P1;
-  // FC2 backward: G pass (Q(G), P2), dX GEMM with the GELU-backward epilogue
+  // FC2 backward: G pass (Q(G), P2)
   FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales,
                         base + w.qg.sf, P2, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
-  GemmArgs g{};
-  g.M = M;
-  g.N = H;
-  g.K = N2;
-  g.R2 = R2;
-  g.a_codes = base + w.qg.codes;
-  g.a_sf = base + w.qg.sf;
-  g.b_codes = fc2->R_codes_t;
-  g.b_sf = fc2->R_sf_t;
-  g.transposed = true;
-  g.A2 = P2;
-  g.B2 = fc2->D;
-  g.out = dh;
-  g.out_bf16 = true;
-  g.h = h_saved;
-  g.out2 = abf;
-  FT_TRY(1, run_gemm(g, status, di.num_sms, s));
-  // FC2 adapter gradients on bf16(GELU(h)) and G
-  FT_TRY(2, run_grads(fc2, M, abf, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, false, base, status, s));
-  // FC1 backward on d_h: G pass, dX GEMM, adapter gradients
-  FT_TRY(3, run_rowpass(dh, M, H, fc1->U, R1, false, false, nullptr, base + w.qdh.codes, base + w.qdh.scales,
-                        base + w.qdh.sf, P1, reinterpret_cast<float*>(base + w.rp_part),
-                        reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
-  // FC1 dX GEMM and adapter gradients
+  // FC2's dX GEMM with the fused epilogue: d_h = bf16(d_a GELU'(h)) (FC1's
+  // incoming gradient), Q(d_h) for FC1's 4-bit branch, P1 = bf16(d_h U1^T)
+  MlpGemmArgs m{};
+  m.g.M = M;
+  m.g.N = H;
+  m.g.K = N2;
+  m.g.R2 = R2;
+  m.g.a_codes = base + w.qg.codes;
+  m.g.a_sf = base + w.qg.sf;
+  m.g.b_codes = fc2->R_codes_t;
+  m.g.b_sf = fc2->R_sf_t;
+  m.g.transposed = true;
+  m.g.A2 = P2;
+  m.g.B2 = fc2->D;
+  m.epi = 2;
+  m.h = h_saved;
+  m.out_h = dh;
+  m.q_codes = base + w.qdh.codes;
+  m.q_scales = base + w.qdh.scales;
+  m.q_sf = base + w.qdh.sf;
+  m.Wp = fc1->U;
+  m.RP = R1;
+  m.proj_out = P1;
+  m.part = reinterpret_cast<float*>(base + w.pj_part);
+  m.counters = reinterpret_cast<int*>(base + w.pj_cnt);
+  FT_TRY(1, run_gemm_mlp(m, status, di.num_sms, s));
+  // FC2 adapter gradients: dA2 on bf16(GELU(h)) (recomputed from h), dB2 on G
+  FT_TRY(2, run_grads(fc2, M, h_saved, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, false, base, status, s,
+                      true));
+  // FC1 dX GEMM and adapter gradients (on d_h)
   GemmArgs g1{};
   g1.M = M;
   g1.N = K1;
@@ -1155,8 +1247,8 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
   if (evs.ev || w.g1.side_sms == 0) {
-    FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
-    FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
+    FT_TRY(3, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
+    FT_TRY(4, run_gemm(g1, status, di.num_sms, s));
   } else {
     st = gemm_and_grads_side(g1, fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status,
                              di.num_sms, s);

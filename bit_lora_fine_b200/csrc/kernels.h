@@ -66,9 +66,41 @@ struct GemmParams {
   int main_bf16;
 };
 
+// The MLP's 4-bit GEMMs with their fused epilogues (FourTune §3.3 "MLP
+// Fusion").  The main product is GemmParams' (A [M, K] and B [N, K] block16
+// codes with MMA-ready scales, + A2 B2^T low-rank blocks); per output tile the
+// epilogue forms a bf16 tensor T [M, N] and
+//   epi == 1 (FC1 forward):  h = bf16(acc + bias) -> out_h;  a = GELU(h) fp32
+//            (-> dbg if set);  Q(a) -> q_*;  T = bf16(a)
+//   epi == 2 (FC2 dX):       d_h = bf16(acc * GELU'(h)) -> out_h;  Q(d_h) -> q_*;
+//            T = d_h
+// and projects it: proj_out [M, RP] = bf16(T Wp), Wp [N, RP] read from D2
+// [N, RP] (wp_mn_major = 1) or from U1 [RP, N] (0), summed over the N tiles of
+// a unit in TMEM and over units through fp32 partials.
+struct MlpGemmParams {
+  GemmParams g;                          // main product (M, N, K, R2, scales, bias, status)
+  int epi;                               // 1 or 2 (above)
+  const void* h;                         // epi 2: bf16 [M, N]
+  void* out_h;                           // bf16 [M, N]: h (epi 1) or d_h (epi 2)
+  float* dbg;                            // epi 1: fp32 a [M, N] or null
+  uint8_t* q_codes;                      // [M, N/2]
+  uint8_t* q_scales;                     // [M/16, N/16]
+  uint8_t* q_sf;                         // MMA-ready scales of Q(T) (rows M, cols N)
+  int RP;                                // projection rank (16..128, multiple of 16)
+  int wp_mn_major;
+  int nsplit, per;                       // units: N tiles [sp*per, +per) of one 128-row tile
+  float* part;                           // fp32 [nsplit, M, RP]
+  int* counters;                         // [ceil(M/128)], zero on entry, left zero
+  void* proj_out;                        // bf16 [M, RP]
+};
+cudaError_t launch_gemm_mlp(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
+                            const CUtensorMap& tmB2, const CUtensorMap& tmW, const MlpGemmParams& p, int num_sms,
+                            cudaStream_t stream);
+
 // out[p, j] (+)= sum_m T[m, p] * V[m, v0 + j]   for p < P, j < r (r <= 64)
 struct TgradParams {
   int M, P, r, v0;
+  int t_gelu;                            // T is h: use bf16(GELU_tanh(T)) (the MLP's FC2 dA)
   int mt_per_split, nsplit;              // 128-row tiles per CTA along M, number of M splits
   float* out;
   long long out_sp, out_sj;

@@ -5,6 +5,10 @@
 // P = G [S_up ; B]^T saved in bf16:
 //   dA = X^T P[:, r_s:]   (T = X,  V = P, out [K, r] row-major)
 //   dB = L[:, r_s:]^T G   (T = G,  V = L, out [r, N] row-major, written as dB^T)
+// For the MLP's FC2, dA = bf16(GELU(h))^T P[:, r_s:] takes T = h (saved by the
+// forward): the epilogue warps, idle during the main loop, replace each staged
+// h tile by bf16(GELU_tanh(h)) in place before its MMAs (t_gelu), so GELU(h) is
+// never stored.
 // Both problems run in one launch (the CTA index selects the problem).  Each is
 // a reduction over the M tokens of a tall bf16 matrix against a thin one:
 // HBM-bound (T is read once).  The tensor cores take both operands MN-major
@@ -22,6 +26,7 @@ constexpr int kTgThreads = 256;
 constexpr uint32_t kTgTBox = 128 * 128;            // 128 m rows x 64 bf16
 constexpr uint32_t kTgStage = 2 * kTgTBox + kTgTBox;  // T (two boxes) + V
 constexpr uint32_t kTgSmem = 1024 + kTgStages * kTgStage + 256;
+static_assert((3 * kTgStages + 1) * 8 + 8 + 16 <= 256, "barriers, TMEM slot and flags fit the tail");
 
 __global__ void __launch_bounds__(kTgThreads, 1)
     tgrad_kernel(const __grid_constant__ CUtensorMap tmT0, const __grid_constant__ CUtensorMap tmV0,
@@ -32,7 +37,8 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTgStages * kTgStage);
   uint64_t* empty = full + kTgStages;
   uint64_t* acc_full = empty + kTgStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* ready = acc_full + 1;           // [kTgStages] t_gelu: the stage's T tile transformed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + kTgStages);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
   volatile int* s_ok = s_last + 1;  // [4]
@@ -60,6 +66,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     for (int s = 0; s < kTgStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 4);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -107,6 +114,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         const int s = i % kTgStages;
         const uint32_t ph = (i / kTgStages) & 1;
         if (!mbar_wait(&full[s], ph, p.status, abortp)) break;
+        if (p.t_gelu && !mbar_wait(&ready[s], ph, p.status, abortp)) break;
         tc_fence_after();
         const uint32_t ta = smem_u32(smem + s * kTgStage);
         const uint32_t va = ta + 2 * kTgTBox;
@@ -120,7 +128,35 @@ __global__ void __launch_bounds__(kTgThreads, 1)
       mbar_wait_drain(acc_full, 0, kWaitLimitNs);
     }
   } else if (warp >= 4) {
-    const bool mine = (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
+    bool ok = true;
+    if (p.t_gelu) {
+      // the T part of every stage (two 16 KB boxes of bf16 h) -> bf16(GELU(h)), in place
+      const int t = static_cast<int>(threadIdx.x) - 128;   // 0..127
+      for (int i = 0; i < nt && ok; ++i) {
+        const int s = i % kTgStages;
+        bool okw = true;
+        if (lane == 0) okw = mbar_wait(&full[s], (i / kTgStages) & 1, p.status, abortp);
+        ok = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        uint4* tile = reinterpret_cast<uint4*>(smem + s * kTgStage);
+#pragma unroll 4
+        for (int k = t; k < static_cast<int>(2 * kTgTBox / 16); k += 128) {
+          uint4 x = tile[k];
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(gelu_tanh(bf16_bits_to_f32(w[e] & 0xFFFFu)),
+                                                           gelu_tanh(bf16_bits_to_f32(w[e] >> 16)));
+            w[e] = *reinterpret_cast<const uint32_t*>(&b);
+          }
+          tile[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ready[s]);
+      }
+    }
+    const bool mine = ok && (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
     if (lane == 0) s_ok[warp - 4] = mine ? 1 : 0;
     named_bar_sync(1, 128);
     const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];

@@ -38,9 +38,9 @@ SIZE_FUNCS = ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspa
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
 BWD_KERNELS = ("gpass_quant_down", "tgrad_dA_dB", "gemm_fp4_dx")
-MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1", "gelu_pass_quant_down", "gemm_fp4_fc2")
-MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_gelu_bwd_fc2", "tgrad_fc2", "dhpass_quant_down_fc1",
-                   "tgrad_fc1", "gemm_fp4_dx_fc1")
+MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1_gelu_quant_proj", "gemm_fp4_fc2")
+MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_fc2_gelu_bwd_quant_proj", "tgrad_fc2", "tgrad_fc1",
+                   "gemm_fp4_dx_fc1")
 
 
 class FourtuneError(RuntimeError):

@@ -233,24 +233,25 @@ FT_API int fourtune_linear_bwd_g16(const ft_linear_t* layer, const ft_bf16* W16_
 
 /* The MLP pair (§3.3 "MLP Fusion"): y = FC2(GELU_tanh(FC1(X))), both layers
  * triple-branch, fc1 [K1 -> H], fc2 [H -> N2] (fc1->N == fc2->K).
- * Forward: the X pass and FC1's 4-bit GEMM (+ bias b1) give the hidden
- * h = bf16(FC1(X)) [M, H] (saved).  One fused pass over h then computes
- * a = GELU_tanh(h) in fp32, quantizes it (Q(a), block16 of the fp32 values)
- * and projects bf16(a) onto FC2's D: L2 = bf16(bf16(a) D2) -- a is never
- * stored.  FC2's 4-bit GEMM adds L2 U2 and b2.  Writes Y [M, N2], h_saved
- * [M, H], L1_saved [M, r_s1 + r1], L2_saved [M, r_s2 + r2]; dbg_a, when not
- * NULL, receives the fp32 a [M, H] that was quantized (for inspection). */
+ * Forward: the X pass, then FC1's 4-bit GEMM (+ L1 U1 + b1) whose epilogue
+ * forms h = bf16(FC1(X)) (saved), a = GELU_tanh(h) in fp32, Q(a) (block16 of
+ * the fp32 values, FC2's 4-bit input) and L2 = bf16(bf16(a) D2) (FC2's
+ * low-rank input) -- the hidden activation a is never stored -- then FC2's
+ * 4-bit GEMM (+ L2 U2 + b2).  Writes Y [M, N2], h_saved [M, H], L1_saved
+ * [M, r_s1 + r1], L2_saved [M, r_s2 + r2]; dbg_a, when not NULL, receives the
+ * fp32 a [M, H] that was quantized (for inspection). */
 FT_API size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
 FT_API int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
                             int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a,
                             void* ws, size_t ws_bytes, void* stream);
 
-/* MLP backward.  FC2's dX GEMM ends in the GELU backward: it reads h and writes
- * d_h = bf16(d_a * GELU'(h)) and bf16(GELU(h)) into the workspace; FC2's dA2
- * uses the latter, FC1's backward takes d_h as its incoming gradient (all
- * three branches).  Writes dX [M, K1] and the four adapter gradients (fp32;
- * accumulate = 1 adds).  FC1's dA1/dB1 run beside FC1's dX GEMM on the library
- * stream, as in fourtune_linear_bwd. */
+/* MLP backward.  FC2's G pass, then FC2's dX GEMM whose epilogue forms
+ * d_h = bf16(d_a GELU'(h)) -- FC1's incoming gradient, taken by all three of
+ * its branches -- with Q(d_h) (FC1's 4-bit gradient) and P1 = bf16(d_h U1^T).
+ * FC2's dA2 = bf16(GELU(h))^T P2[:, r_s2:] recomputes GELU(h) from h (nothing
+ * of the activation is stored).  Writes dX [M, K1] and the four adapter
+ * gradients (fp32; accumulate = 1 adds).  FC1's dA1/dB1 run beside FC1's dX
+ * GEMM on the library stream, as in fourtune_linear_bwd. */
 FT_API size_t fourtune_mlp_bwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
 FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* dY, const ft_bf16* X,
                             const ft_bf16* h_saved, const ft_bf16* L1_saved, const ft_bf16* L2_saved, int64_t M,
@@ -258,9 +259,9 @@ FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
                             void* ws, size_t ws_bytes, void* stream);
 
 /* The MLP calls with per-kernel CUDA events, as fourtune_linear_*_timed.  Kernels,
- * in order -- forward: 0 X pass, 1 FC1 GEMM (h), 2 GELU pass (Q(a), L2), 3 FC2 GEMM;
- * backward: 0 G pass (FC2), 1 FC2 dX GEMM with the GELU backward, 2 FC2 dA/dB,
- * 3 d_h pass (FC1), 4 FC1 dA/dB, 5 FC1 dX GEMM. */
+ * in order -- forward: 0 X pass, 1 FC1 GEMM with the GELU / Q(a) / L2 epilogue,
+ * 2 FC2 GEMM; backward: 0 G pass (FC2), 1 FC2 dX GEMM with the GELU' / Q(d_h) / P1
+ * epilogue, 2 FC2 dA/dB, 3 FC1 dA/dB, 4 FC1 dX GEMM. */
 FT_API int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M,
                                   void* Y, int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved,
                                   float* dbg_a, void* ws, size_t ws_bytes, void* stream, void* const* events,
@@ -272,8 +273,9 @@ FT_API int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2
                                   void* const* events, int n_events);
 
 /* Workspace byte offsets of the MLP's intermediate tensors (inspection, tests):
- * forward: Q(a) codes [M, H/2] and scales [M/16, H/16]; backward: d_h and
- * bf16(GELU(h)) (both bf16 [M, H]) and Q(d_h) codes and scales. */
+ * forward: Q(a) codes [M, H/2] and scales [M/16, H/16]; backward: d_h (bf16
+ * [M, H]) and Q(d_h) codes and scales; a_off is set to SIZE_MAX (bf16(GELU(h))
+ * is not stored). */
 FT_API int fourtune_mlp_fwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* qa_codes,
                                        size_t* qa_scales);
 FT_API int fourtune_mlp_bwd_ws_offsets(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, size_t* dh_off,

@@ -10,8 +10,9 @@ the fp32 accumulation bound.  Backward: d_h = bf16(d_a GELU'(h)) -- the
 gradient FC1's three branches take, rounded to bf16 like any layer's incoming
 gradient -- within one bf16 ulp of the exact value plus the bounds of d_a's
 fp32 sum and GELU's fp32 evaluation; Q(d_h) bit-identical to the oracle's
-quantizer on the GPU's d_h; dX and all four adapter gradients within the
-normwise tolerance and the elementwise fp32 bound.  bf16 y and dX equal the
+quantizer on the GPU's d_h; P1 within the bf16-dot bound (through dX and dA1);
+dX and all four adapter gradients within the normwise tolerance and the
+elementwise fp32 bound; bf16(GELU(h)) is not stored (FC2's dA2 recomputes it).  bf16 y and dX equal the
 rounding of the fp32 outputs.  Outputs and workspaces start poisoned.
 """
 import numpy as np
@@ -77,13 +78,16 @@ def run_mlp(ft, p1, p2, X, dY, rows=None):
     dX, dA1, dB1, dA2, dB2, wsb = ft.mlp_bwd(mlp, dYd, Xd, h, L1, L2, ws=wsb, dX=nan_dev((M, K1)), grads=grads)
     ft.device_status(wsb)
     dho, ao, qdc, qds = mlp.bwd_ws_offsets(M)
+    assert ao == 2 ** 64 - 1                                        # bf16(GELU(h)) is not stored
     dh = wsb[dho:dho + M * H * 2].view(bf).view(M, H)
-    abf = wsb[ao:ao + M * H * 2].view(bf).view(M, H)
     qdh_codes = wsb[qdc:qdc + M * H // 2].view(M, H // 2).cpu().numpy()
     qdh_scales = wsb[qds:qds + (M // 16) * (H // 16)].view(M // 16, H // 16).cpu().numpy()
 
     h_g, L1_g, L2_g, a_g = to_host(h), to_host(L1), to_host(L2), to_host(a).astype(np.float32)
-    dh_g, abf_g = to_host(dh), to_host(abf)
+    dh_g = to_host(dh)
+    # bf16(GELU(h)) as FC2's dA2 uses it (the GPU recomputes it from h in fp32;
+    # one bf16 rounding step apart at most, covered by dA2's bound below)
+    abf_g = formats.bf16_round(olayer.gelu_tanh(h_g).astype(np.float32).astype(np.float64))
     Y_g, dX_g = to_host(Y), to_host(dX)
     assert not np.isnan(Y_g).any() and not np.isnan(dX_g).any()
     rows = np.arange(M) if rows is None else rows
@@ -122,10 +126,8 @@ def run_mlp(ft, p1, p2, X, dY, rows=None):
                 + np.abs(fc2["bias"])[None, :])
     check_fp32_dot(Y_g[rows], y_ex, absdot_y, H + R2, name="y")
 
-    # ---- backward on the sampled rows (oracle fed the GPU's h, L, d_h, bf16(GELU(h)))
-    assert np.all(np.abs(abf_g[rows] - g_ref) <= 2.0 ** -8 * np.abs(g_ref) + GELU_REL * np.abs(g_ref) + GELU_FLOOR)
-    b = olayer.mlp_bwd(dY[rows], Xs, h_g[rows], L1_g[rows], L2_g[rows], fc1, fc2, dh_bf=dh_g[rows],
-                       a_bf=abf_g[rows])
+    # ---- backward on the sampled rows (oracle fed the GPU's h, L, d_h)
+    b = olayer.mlp_bwd(dY[rows], Xs, h_g[rows], L1_g[rows], L2_g[rows], fc1, fc2, dh_bf=dh_g[rows])
     # d_h = bf16(d_a GELU'(h)): d_a is an fp32 sum on the GPU's own P2 (one bf16 ulp,
     # at most 2^-7 relative, from the oracle's), GELU' an fp32 evaluation
     Gq = block16.dequantize(b["qg_codes"], b["qg_scales"])
@@ -153,8 +155,9 @@ def run_mlp(ft, p1, p2, X, dY, rows=None):
             (dB1, L1_g[:, rs1:].T @ dh_g, np.abs(L1_g[:, rs1:]).T @ np.abs(dh_g), False, "dB1")):
         g = to_host(got)
         assert normwise(g, ex) <= TOL, name
-        # P recomputed here may differ from the GPU's P by one bf16 ulp (2^-7 relative)
-        check_fp32_dot(g, ex, absd, M, extra=2.0 ** -7 * absd if extra else 0.0, name=name)
+        # P (and, for dA2, bf16(GELU(h))) recomputed here may differ from the GPU's by
+        # one bf16 ulp each (2^-7 relative)
+        check_fp32_dot(g, ex, absd, M, extra=2.0 ** -6 * absd if extra else 0.0, name=name)
 
     # ---- production outputs: bf16 y and dX are the rounding of the fp32 ones
     outb = (nan_dev((M, N2), bf),) + out[1:]
