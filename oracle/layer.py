@@ -19,12 +19,13 @@ Readings of what the pages leave open (each is also listed in the design notes):
     bf16 (ties-to-even) once, after exact accumulation: they feed bf16 products.
   * dA = X^T P[:, r_s:]   and   dB = L[:, r_s:]^T G   (straight-through: Q has
     no derivative of its own).
-  * MLP: h = bf16(FC1(X) + b1) is the saved hidden; a = GELU_tanh(h);
-    FC2's 4-bit input is Q(a) of float32 a (the quantizer consumes the
-    activation as it is produced, never stored in bf16); its low-rank input is
-    bf16(a).  Backward: d_a from FC2, d_h = bf16(d_a * GELU'(h)) -- the
-    gradient reaching FC1 is a bf16 tensor like any layer's incoming gradient,
-    and all three of FC1's branches take it (Q(d_h) for the 4-bit branch).
+  * MLP: h = bf16(FC1(X) + b1) is the saved hidden; a = GELU_tanh(h) (float32);
+    FC2's three branches share one input, bf16(a) -- Q(bf16(a)) for the 4-bit
+    branch, bf16(a) for the low-rank ones -- as every layer's input is a bf16
+    tensor (§3.3 "LoRA Fusion").  Backward: d_a from FC2, d_h =
+    bf16(d_a * GELU'(h)) -- the gradient reaching FC1 is a bf16 tensor like any
+    layer's incoming gradient, and all three of FC1's branches take it (Q(d_h)
+    for the 4-bit branch).
 
 All GEMMs run in float64 on the exactly dequantized operands; a library matmul
 is the only primitive used.
@@ -157,8 +158,9 @@ def mlp_fwd(X, fc1, fc2, a_f32=None):
     """FC1 -> GELU(tanh) -> FC2, both triple-branch layers.
 
     fc1/fc2: dict(R_codes, R_scales, S_dn, S_up, A, B, bias).
-    `a_f32` optionally overrides the float32 activation that FC2 quantizes (the
-    GPU's own a, so that downstream results compare on identical operands).
+    `a_f32` optionally overrides the float32 activation a (the GPU's own, so
+    that downstream results compare on identical operands); FC2's input is
+    bf16(a) for all three of its branches.
     Returns dict(y, h, a, L1, L2, qa_codes, qa_scales, ...).
     """
     o1 = linear_fwd(X, fc1["R_codes"], fc1["R_scales"], fc1["S_dn"], fc1["S_up"],
@@ -167,7 +169,7 @@ def mlp_fwd(X, fc1, fc2, a_f32=None):
     a = gelu_tanh(h)
     a32 = a.astype(np.float32) if a_f32 is None else np.asarray(a_f32, dtype=np.float32)
     a_bf = formats.bf16_round(a32.astype(np.float64))
-    Qa = block16.quantize(a32)
+    Qa = block16.quantize(a_bf.astype(np.float32))
     o2 = linear_fwd(a_bf, fc2["R_codes"], fc2["R_scales"], fc2["S_dn"], fc2["S_up"],
                     fc2["A"], fc2["B"], fc2.get("bias"), Qx=Qa)
     return dict(y=o2["y"], h=h, a=a, a32=a32, a_bf=a_bf, L1=o1["L"], L2=o2["L"],

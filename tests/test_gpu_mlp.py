@@ -2,11 +2,11 @@
 
 Forward: h = bf16(FC1 output) within one bf16 ulp of the exact value plus the
 fp32 accumulation bound; L1 and L2 within the bf16-dot bound; a = GELU(h) (the
-fp32 values the GPU quantized, from the debug output) within the fp32 GELU
-bound of the float64 GELU of the GPU's h; Q(a) codes and scales bit-identical
-to the oracle's quantizer applied to the GPU's own fp32 a (floating point
-decides the codes, so both sides quantize the same a); y elementwise within
-the fp32 accumulation bound.  Backward: d_h = bf16(d_a GELU'(h)) -- the
+fp32 values from the debug output) within the fp32 GELU bound of the float64
+GELU of the GPU's h; Q(bf16(a)) codes and scales bit-identical to the oracle's
+quantizer applied to the bf16 rounding of the GPU's own a (floating point
+decides the codes, so both sides quantize the same values); y elementwise
+within the fp32 accumulation bound.  Backward: d_h = bf16(d_a GELU'(h)) -- the
 gradient FC1's three branches take, rounded to bf16 like any layer's incoming
 gradient -- within one bf16 ulp of the exact value plus the bounds of d_a's
 fp32 sum and GELU's fp32 evaluation; Q(d_h) bit-identical to the oracle's
@@ -113,10 +113,10 @@ def run_mlp(ft, p1, p2, X, dY, rows=None):
     check_bf16_rounded(h_g[rows], h_ex, fp32_dot_bound(absdot_h, K1 + R1) + 2.0 ** -24 * np.abs(h_ex), name="h")
     g_ref = olayer.gelu_tanh(h_g[rows])
     assert np.all(np.abs(a_s - g_ref) <= GELU_REL * np.abs(g_ref) + GELU_FLOOR), "GELU(h) beyond its fp32 bound"
-    rc, rs_ = block16.quantize(a_s)                                      # oracle quantizer on the GPU's a
+    a_bf = formats.bf16_round(a_s.astype(np.float64))                   # FC2's input, all three branches
+    rc, rs_ = block16.quantize(a_bf.astype(np.float32))                  # oracle quantizer on the GPU's bf16(a)
     np.testing.assert_array_equal(qa_scales[blocks], rs_)
     np.testing.assert_array_equal(qa_codes[rows], rc)
-    a_bf = formats.bf16_round(a_s.astype(np.float64))
     o2 = olayer.linear_fwd(a_bf, fc2["R_codes"], fc2["R_scales"], fc2["S_dn"], fc2["S_up"], fc2["A"], fc2["B"],
                            fc2["bias"], Qx=(rc, rs_))
     check_bf16_dot(L2_g[rows], o2["L"], np.abs(a_bf) @ np.abs(D2), H)
