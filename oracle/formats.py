@@ -120,9 +120,11 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     binade, round the significand with numpy's round-half-to-even, scale back.
     Below 2**-126 the spacing stays 2**-133 (bfloat16 subnormals); values past
     the largest finite bfloat16 are not expected and the assert checks it.
+    Rounding keeps the sign of zero (IEEE 754): -0.0 stays -0.0, and a negative
+    value below half the smallest subnormal rounds to -0.0.
     """
     x = np.asarray(x, dtype=np.float64)
-    out = np.zeros_like(x)
+    out = x.copy()                      # zeros pass through with their sign
     nz = x != 0
     if np.any(nz):
         v = x[nz]

@@ -121,6 +121,17 @@ def test_bf16_round_vs_torch():
     np.testing.assert_array_equal(ours, th)
 
 
+def test_bf16_round_keeps_sign_of_zero():
+    # IEEE rounding: -0 stays -0, a negative value below half the smallest
+    # bfloat16 subnormal (2^-133) rounds to -0; torch's conversion agrees
+    x32 = np.float32([-0.0, 0.0, -1e-45, 1e-45, -3e-41, -2.0 ** -134])
+    ours = formats.bf16_round(x32.astype(np.float64))
+    th = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(ours, th)
+    np.testing.assert_array_equal(np.signbit(ours), np.signbit(th))
+    assert np.signbit(ours[0]) and not np.signbit(ours[1]) and np.signbit(ours[2])
+
+
 def test_bf16_round_ties_even():
     # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties to even -> 1
     assert formats.bf16_round(np.array([1.0 + 2 ** -8]))[0] == 1.0
