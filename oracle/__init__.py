@@ -17,7 +17,11 @@ E2M1 codes, one E4M3 scale per block, round-to-nearest-even.
 Modules
   formats  -- E2M1 / E4M3 code tables and round-to-nearest-even encoders.
   block16  -- the 16x16 block quantizer, its dequantizer, transposed packing.
-  layer    -- triple-branch linear and MLP, forward and backward, float64.
+  group16  -- the 1x16 group-wise quantizer with a power-of-two per-tensor
+              scale (the granularity comparator of §4.3, Table 5).
+  layer    -- triple-branch linear and MLP, forward and backward, float64; the
+              precision variants and the 1x16 variant of the linear layer.
+  stabilizer -- the truncated-SVD split W^T = S_dn S_up + R (§3.1).
 
 Parity status: every function here is pinned by tests under tests/ (tables vs
 ml_dtypes/torch, worked ties, representability, idempotence, transposed-block

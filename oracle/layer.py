@@ -32,7 +32,7 @@ is the only primitive used.
 """
 import numpy as np
 
-from . import block16, formats
+from . import block16, formats, group16
 
 
 def _f64(a):
@@ -123,6 +123,44 @@ def linear_bwd_g16(G, X, L, Rq, S_dn, S_up, A, B):
     P = formats.bf16_round(G @ _U(S_up, B).T)
     dX = G @ _f64(Rq) + P @ _D(S_dn, A).T
     return dict(dX=dX, dA=X.T @ P[:, r_s:], dB=L[:, r_s:].T @ G, P=P)
+
+
+# ------------------------------------------------------- 1x16 group-wise variant
+# §4.3 (Table 5) compares the 16x16 blocks with 1x16 groups (group16.py): the
+# same triple-branch layer with X, G and the weight quantized in 1x16 groups
+# along each GEMM's reduction dimension, plus a per-tensor scale.  The weight
+# has two quantized forms: Q16(R) [N, K] (groups along K) for the forward, and
+# Q16(R^T) [K, N] (groups along N) for dX -- the transposed operand is
+# quantized again, which the block layout avoids (§3.2).
+
+def linear_fwd_1x16(X, Rq, S_dn, S_up, A, B, bias=None, Qx=None):
+    """Forward: y = deq(Q16(X)) Rq^T + L [S_up ; B] (+ bias), L = bf16(X [S_dn | A]).
+    Rq = deq(Q16(R)) [N, K] in float64.  Returns dict(y, L, qx_codes, qx_scales, qx_e)."""
+    X = _f64(X)
+    if Qx is None:
+        Qx = group16.quantize(X.astype(np.float32))
+    codes, scales, e = Qx
+    L = formats.bf16_round(X @ _D(S_dn, A))
+    y = group16.dequantize(codes, scales, e) @ _f64(Rq).T + L @ _U(S_up, B)
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return dict(y=y, L=L, qx_codes=codes, qx_scales=scales, qx_e=e)
+
+
+def linear_bwd_1x16(G, X, L, Rtq, S_dn, S_up, A, B, Qg=None):
+    """Backward: dX = deq(Q16(G)) Rtq^T + P [S_dn | A]^T with Rtq = deq(Q16(R^T))
+    [K, N] and P = bf16(G [S_up ; B]^T); dA, dB as in linear_bwd.
+    Returns dict(dX, dA, dB, P, qg_codes, qg_scales, qg_e)."""
+    G = _f64(G)
+    X = _f64(X)
+    L = _f64(L)
+    r_s = np.asarray(S_dn).shape[1]
+    if Qg is None:
+        Qg = group16.quantize(G.astype(np.float32))
+    codes, scales, e = Qg
+    P = formats.bf16_round(G @ _U(S_up, B).T)
+    dX = group16.dequantize(codes, scales, e) @ _f64(Rtq).T + P @ _D(S_dn, A).T
+    return dict(dX=dX, dA=X.T @ P[:, r_s:], dB=L[:, r_s:].T @ G, P=P, qg_codes=codes, qg_scales=scales, qg_e=e)
 
 
 # ------------------------------------------------------------------------- MLP
