@@ -261,13 +261,20 @@ struct MlpUnits {
   int nsplit, per;
 };
 MlpUnits plan_units(int64_t M, int64_t N, int num_sms) {
+  // units of `per` consecutive N tiles of one 128-row tile: the makespan (tiles
+  // on the busiest CTA) first, then as few splits (fp32 partials) as possible
   const int MT = cdiv(M, 128), NT = cdiv(N, 256);
-  const double ideal = static_cast<double>(MT) * NT / num_sms;
-  for (int ns = 1; ns <= NT; ++ns) {
+  auto span_of = [&](int ns, int* nsr_out) {
     const int per = cdiv(NT, ns);
     const int nsr = cdiv(NT, per);
-    const double span = static_cast<double>(cdiv(static_cast<int64_t>(MT) * nsr, num_sms)) * per;
-    if (span <= 1.03 * ideal || ns == NT) return {nsr, per};
+    if (nsr_out) *nsr_out = nsr;
+    return static_cast<int64_t>(cdiv(static_cast<int64_t>(MT) * nsr, num_sms)) * per;
+  };
+  int64_t best = span_of(NT, nullptr);
+  for (int ns = 1; ns < NT; ++ns) best = std::min(best, span_of(ns, nullptr));
+  for (int ns = 1; ns <= NT; ++ns) {
+    int nsr = 0;
+    if (span_of(ns, &nsr) <= best) return {nsr, cdiv(NT, ns)};
   }
   return {NT, 1};
 }
@@ -376,10 +383,8 @@ int side_stream(SideStream** out) {
 
 // ---------------------------------------------------------------- launch helpers
 // Fused row pass over X [M, K] bf16: Q(X) -> (codes, scales), L = bf16(X W)
-// with W = D [K, R] (w_mn) or W^T [R, K]; gelu: the input is h and the pass
-// quantizes GELU(h).
-int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, bool gelu,
-                float* dbg_a, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
+// with W = D [K, R] (w_mn) or W^T [R, K].
+int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
                 int* status, int num_sms, cudaStream_t s, bool no_quant = false) {
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
@@ -393,8 +398,6 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.kt_per_split = rs.kt_per_split;
   rp.nsplit = rs.nsplit;
   rp.stages = rs.stages;
-  rp.gelu_input = gelu ? 1 : 0;
-  rp.dbg_a = dbg_a;
   rp.codes = codes;
   rp.scales = scales;
   rp.sf_mma = sf_mma;
@@ -423,8 +426,6 @@ struct GemmArgs {
   const void* bias;
   void* out;
   bool out_bf16;
-  const void* h;                // GELU-backward epilogue: saved hidden [M, N]
-  void* out2;                   // GELU-backward epilogue: bf16(GELU(h)) [M, N]
   bool main_bf16;               // 16-bit main product: a_codes = A [M, K], b_codes = B [N, K] bf16
 };
 int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
@@ -454,9 +455,6 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   gp.out = a.out;
   gp.ldo = a.N;
   gp.out_bf16 = a.out_bf16 ? 1 : 0;
-  gp.epi_gelu_bwd = a.h ? 1 : 0;
-  gp.h = a.h;
-  gp.out2 = a.out2;
   gp.status = status;
   gp.main_bf16 = a.main_bf16 ? 1 : 0;
   return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
@@ -776,7 +774,7 @@ int fourtune_linear_fwd_timed(const ft_linear_t* layer, const ft_bf16* X, int64_
   uint8_t* qs = base + w.qx.scales;
   uint8_t* qf = base + w.qx.sf;
   // X pass: Q(X) and L = bf16(X D)
-  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, false, nullptr, qc, qs, qf, L_saved,
+  FT_TRY(0, run_rowpass(X, M, K, layer->D, R, true, qc, qs, qf, L_saved,
                         reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                         di.num_sms, s));
   // 4-bit GEMM + L U + bias
@@ -836,7 +834,7 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   uint8_t* gf = base + w.qg.sf;
   void* P = base + w.P;
   // G pass: Q(G) and P = bf16(G U^T), U [R, N] read K-major
-  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, gc, gs, gf, P,
+  FT_TRY(0, run_rowpass(dY, M, N, layer->U, R, false, gc, gs, gf, P,
                         reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                         di.num_sms, s));
   // dX = deq(Q(G)) deq(Q(R)) + P D^T, and dA = X^T P[:, r_s:], dB = L[:, r_s:]^T G
@@ -973,7 +971,7 @@ int fourtune_linear_fwd_a16(const ft_linear_t* layer, const ft_bf16* W16, const 
   if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   // L = bf16(X D) only (the activation is not quantized)
-  st = run_rowpass(X, M, K, layer->D, R, true, false, nullptr, nullptr, nullptr, nullptr, L_saved,
+  st = run_rowpass(X, M, K, layer->D, R, true, nullptr, nullptr, nullptr, L_saved,
                    reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                    di.num_sms, s, true);
   if (st) return st;
@@ -1018,7 +1016,7 @@ int fourtune_linear_bwd_g16(const ft_linear_t* layer, const ft_bf16* W16_t, cons
   const int64_t K = layer->K, N = layer->N, R = rank_all(layer);
   void* P = base + w.P;
   // P = bf16(G U^T) only (the gradient is not quantized)
-  st = run_rowpass(dY, M, N, layer->U, R, false, false, nullptr, nullptr, nullptr, nullptr, P,
+  st = run_rowpass(dY, M, N, layer->U, R, false, nullptr, nullptr, nullptr, P,
                    reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
                    di.num_sms, s, true);
   if (st) return st;
@@ -1113,7 +1111,7 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
   const int64_t K1 = fc1->K, H = fc1->N, N2 = fc2->N, R1 = rank_all(fc1), R2 = rank_all(fc2);
   // FC1: X pass (Q(X), L1)
-  FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, false, nullptr, base + w.qx.codes, base + w.qx.scales,
+  FT_TRY(0, run_rowpass(X, M, K1, fc1->D, R1, true, base + w.qx.codes, base + w.qx.scales,
                         base + w.qx.sf, L1_saved, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   // FC1's 4-bit GEMM + L1 U1 + b1 with the fused epilogue: h (saved), a =
@@ -1199,7 +1197,7 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   void* dh = base + w.dh;
   void* P1 = base + w.P1;
   // FC2 backward: G pass (Q(G), P2)
-  FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, false, nullptr, base + w.qg.codes, base + w.qg.scales,
+  FT_TRY(0, run_rowpass(dY, M, N2, fc2->U, R2, false, base + w.qg.codes, base + w.qg.scales,
                         base + w.qg.sf, P2, reinterpret_cast<float*>(base + w.rp_part),
                         reinterpret_cast<int*>(base + w.rp_cnt), status, di.num_sms, s));
   // FC2's dX GEMM with the fused epilogue: d_h = bf16(d_a GELU'(h)) (FC1's

@@ -264,6 +264,10 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
+// one word per thread -> the same word in 4 consecutive columns of the warp's lane quadrant
+__device__ __forceinline__ void tmem_st_32x32b_x4_rep(uint32_t taddr, uint32_t w) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%1,%1,%1};" ::"r"(taddr), "r"(w) : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ descriptors
@@ -464,31 +468,31 @@ __device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, 
 // error of GELU(h) and of s.  Beyond that s is 0 or 1 to far below fp32
 // resolution of the result: u < -40 gives GELU = -0 and GELU' = 0 (true values
 // below 1e-32 in magnitude), u > 40 gives GELU = h and GELU' = 1 (exact in fp32);
-// both hold for any h, however large (h^3 may overflow to infinity).
+// both hold for any h, however large (h^3 may overflow to infinity).  The
+// limits are taken as selects, so a warp never branches on its values.
 constexpr float kGeluC = 0.7978845608028654f;  // sqrt(2/pi)
 constexpr float kGeluK = 0.044715f;
+// s = 0.5 (1 + tanh u) with the limits taken as selects (no branches)
+__device__ __forceinline__ float gelu_s(float u, float* e_out) {
+  const float uc = fminf(fmaxf(u, -40.0f), 40.0f);
+  const float e = __expf(-2.0f * uc);
+  float s = __fdividef(1.0f, 1.0f + e);
+  s = u < -40.0f ? 0.0f : s;
+  s = u > 40.0f ? 1.0f : s;
+  *e_out = e;
+  return s;
+}
 __device__ __forceinline__ float gelu_tanh(float h) {
-  const float u = kGeluC * (h + kGeluK * h * h * h);
-  if (u > 40.0f) return h;
-  if (u < -40.0f) return h * 0.0f;
-  return __fdividef(h, 1.0f + __expf(-2.0f * u));
+  float e;
+  return h * gelu_s(kGeluC * (h + kGeluK * h * h * h), &e);
 }
 __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg) {
   const float u = kGeluC * (h + kGeluK * h * h * h);
-  if (u > 40.0f) {
-    *g = h;
-    *dg = 1.0f;
-    return;
-  }
-  if (u < -40.0f) {
-    *g = h * 0.0f;
-    *dg = 0.0f;
-    return;
-  }
-  const float e = __expf(-2.0f * u);
-  const float s = __fdividef(1.0f, 1.0f + e);
+  float e;
+  const float s = gelu_s(u, &e);
   *g = h * s;
-  *dg = s + 2.0f * h * s * (e * s) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
+  const float d = s + 2.0f * h * s * (e * s) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
+  *dg = u > 40.0f ? 1.0f : (u < -40.0f ? 0.0f : d);
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }

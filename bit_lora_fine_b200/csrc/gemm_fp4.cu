@@ -23,19 +23,17 @@
 // more than the 4 MMAs of the K-block take.  Instead four scale warps, one per
 // lane quadrant, load each K-block's scale words from global memory (L2) into
 // registers and write them into their quadrant with tcgen05.st, which runs
-// beside the MMAs.  (The GELU-backward variant, which needs all of its warps'
-// registers for its epilogue, keeps the copy path: the scale blocks come into
-// the stage by bulk copies and the MMA warp moves them with tcgen05.cp.)
+// beside the MMAs.
 // Warp roles:
-//   warp 0 lane 0  producer: TMA code boxes per K-block (+ scale bulk copies in
-//                  the GELU variant); then the bf16 low-rank blocks A2
+//   warp 0 lane 0  producer: TMA code boxes per K-block; then the bf16
+//                  low-rank blocks A2
 //                  [128 x 64] and B2 (K-major [BN x 64] or MN-major [64 x BN]
 //                  in four boxes)
 //   warp 1         TMEM owner; lane 0 issues
 //                  tcgen05.mma kind::mxf4nvf4.block_scale.block16 (M=128,
 //                  N=BN, K=64) once a stage's codes and scales are in, then
 //                  kind::f16 for the low-rank blocks
-//   warps 12..15   scale warps (all but the GELU variant): warp 12+q fills
+//   warps 12..15   scale warps: warp 12+q fills
 //                  quadrant q's scale columns of each stage, one stage ahead
 //                  in registers; a stage's columns are rewritten only after
 //                  the MMAs that read them have completed (the stage's
@@ -44,10 +42,8 @@
 //                  columns.  bf16 output: the warp's accumulator slice goes to
 //                  registers (+ bias, packed to bf16), the accumulator is
 //                  handed back to the MMA warp at once, and the rows are
-//                  written while the next tile's MMAs run.  fp32 output and
-//                  the MLP's GELU-backward variant (d_h = bf16(acc * GELU'(h))
-//                  and bf16(GELU(h)), FourTune §3.3 MLP) hand it back after
-//                  their last TMEM read.  Rows go out through a 1 KB per-warp
+//                  written while the next tile's MMAs run.  fp32 output hands
+//                  it back after its last TMEM read.  Rows go out through a 1 KB per-warp
 //                  smem transpose as 16-row x 32-byte (whole-sector) stores.
 #include "common.cuh"
 #include "kernels.h"
@@ -56,17 +52,13 @@ namespace ft {
 
 constexpr int kGmStages = 4;
 constexpr int kGmThreads = 512;      // warps 0-3 roles, 4-11 epilogue, 12-15 scale warps
-constexpr int kGmThreadsGelu = 640;  // GELU-backward variant: 16 epilogue warps, copy path for scales
 
-template <int BN, bool kSmemScales>
+template <int BN>
 struct GemmLayout {
   static constexpr int kNC = BN / 128;                       // 128-row scale chunks of the B tile
   static constexpr uint32_t kA = 128 * 128;                  // A codes / A2 bf16 tile
   static constexpr uint32_t kB = BN * 128;                   // B codes / B2 bf16 tile
-  // scale blocks in the stage (copy path only): A 4 k-steps x 512 B, B [chunk][k-step][512 B]
-  static constexpr uint32_t kSFA = kSmemScales ? 4 * 512 : 0;
-  static constexpr uint32_t kSFB = kSmemScales ? kNC * 4 * 512 : 0;
-  static constexpr uint32_t kStage = kA + kB + kSFA + kSFB;  // multiple of 1024
+  static constexpr uint32_t kStage = kA + kB;                // multiple of 1024
   static constexpr uint32_t kEpi = 8 * 1024;                 // one transpose buffer per epilogue warp
   static constexpr uint32_t kSmem = 1024 + kGmStages * kStage + kEpi + 256;
   // TMEM columns: accumulator, then per stage 16 (SFA) + 16*kNC (SFB)
@@ -101,16 +93,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// GELU: the MLP's GELU-backward epilogue (its own instantiation, so that the
-// other epilogues do not carry its registers)
-template <int BN, bool GELU>
-__global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
+template <int BN>
+__global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmParams p) {
-  constexpr bool kCp = GELU;   // scales through the stage and tcgen05.cp (else scale warps)
-  using Lay = GemmLayout<BN, kCp>;
-  static_assert(kCp || Lay::kNC == 2, "scale warps store the B scales of two 128-row chunks (32 columns)");
+  using Lay = GemmLayout<BN>;
+  static_assert(Lay::kNC == 2, "scale warps store the B scales of two 128-row chunks (32 columns)");
   static_assert(Lay::kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(Lay::kTmemUsed <= 512, "TMEM budget");
   static_assert(Lay::kSmem <= 232448, "shared memory budget");
@@ -129,7 +118,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
   static_assert((3 * kGmStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and flag fit the tail");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool bf16main = !kCp && p.main_bf16;   // 16-bit main product: 64-wide bf16 K-blocks, no scales
+  const bool bf16main = p.main_bf16 != 0;   // 16-bit main product: 64-wide bf16 K-blocks, no scales
   const int KB = bf16main ? (p.K + 63) / 64 : (p.K + 255) / 256;   // main-product K-blocks
   const int KS = (p.K + 63) / 64;         // 64-wide k-steps: scale blocks per 128-row chunk
   const int EB = (p.R2 + 63) / 64;        // bf16 low-rank blocks
@@ -138,14 +127,6 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
   const int tiles = tiles_n * ((p.M + 127) / 128);
   const int nchunk_b = (p.N + 127) / 128;
 
-  // Scale regions start zeroed: a B tile past N reads scale blocks that no copy
-  // fills, and their E4M3 bytes must not be NaN (they multiply zero codes).
-  for (int s = 0; s < kGmStages; ++s) {
-    uint4* z = reinterpret_cast<uint4*>(smem + s * Lay::kStage + Lay::kA + Lay::kB);
-    for (int k = threadIdx.x; k < static_cast<int>((Lay::kSFA + Lay::kSFB) / 16); k += blockDim.x)
-      z[k] = make_uint4(0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGmStages; ++s) {
       mbar_init(&full[s], 1);      // producer (expect_tx)
@@ -153,7 +134,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       mbar_init(&sf_full[s], 4);   // one arrive per scale warp
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, GELU ? 16 : 8);   // one arrive per epilogue warp
+    mbar_init(acc_empty, 8);   // one arrive per epilogue warp
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -183,7 +164,6 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int m0 = (tile / tiles_n) * 128, n0 = (tile % tiles_n) * BN;
-        const uint8_t* sfa = p.sfa + static_cast<size_t>(m0 / 128) * KS * 512;
         for (int i = 0; i < T; ++i) {
           const int s = g % kGmStages;
           const uint32_t ph = (g / kGmStages) & 1;
@@ -193,22 +173,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
           }
           uint8_t* st = smem + s * Lay::kStage;
           if (i < KB) {
-            if (kCp) {
-              const int nks = min(4, KS - 4 * i);                 // k-steps of this K-block
-              const uint32_t sfbytes = static_cast<uint32_t>(nks) * 512u;
-              int nb = 0;
-#pragma unroll
-              for (int c = 0; c < Lay::kNC; ++c) nb += (n0 / 128 + c < nchunk_b) ? 1 : 0;
-              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + sfbytes * static_cast<uint32_t>(1 + nb));
-              bulk_load(st + Lay::kA + Lay::kB, sfa + static_cast<size_t>(4 * i) * 512, sfbytes, &full[s]);
-#pragma unroll
-              for (int c = 0; c < Lay::kNC; ++c)
-                if (n0 / 128 + c < nchunk_b)
-                  bulk_load(st + Lay::kA + Lay::kB + Lay::kSFA + c * 2048,
-                            p.sfb + (static_cast<size_t>(n0 / 128 + c) * KS + 4 * i) * 512, sfbytes, &full[s]);
-            } else {
-              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
-            }
+            mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
             // a K-block is 128 bytes of each row: 256 FP4 codes or 64 bf16 values
             const int kx = bf16main ? i * 64 : i * 128;
             tma_load_2d(st, &tmA, &full[s], kx, m0);
@@ -247,8 +212,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
         for (int i = 0; i < T; ++i) {
           const int s = g % kGmStages;
           const uint32_t ph = (g / kGmStages) & 1;
-          if (!mbar_wait(&full[s], ph, p.status, abortp) ||
-              (!kCp && !mbar_wait(&sf_full[s], ph, p.status, abortp))) {
+          if (!mbar_wait(&full[s], ph, p.status, abortp) || !mbar_wait(&sf_full[s], ph, p.status, abortp)) {
             ok = false;
             break;
           }
@@ -262,18 +226,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
                        (i | t) != 0 ? 1u : 0u);
           } else if (i < KB) {
             const int nks = min(4, KS - 4 * i);
-            const uint32_t sfa_addr = b_addr + Lay::kB;
-            const uint32_t sfb_addr = sfa_addr + Lay::kSFA;
             const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
-            if (kCp) {
-              for (int t = 0; t < nks; ++t) {
-                tmem_cp_32x128b_x4(tmem + sf_col + 4 * t, desc_sf_copy(sfa_addr + t * 512));
-#pragma unroll
-                for (int c = 0; c < Lay::kNC; ++c)
-                  tmem_cp_32x128b_x4(tmem + sf_col + 16 + (t * Lay::kNC + c) * 4,
-                                     desc_sf_copy(sfb_addr + (c * 4 + t) * 512));
-              }
-            }
             for (int t = 0; t < nks; ++t)
               mma_fp4_block16(tmem, desc_kmajor_sw128(a_addr + 32 * t), desc_kmajor_sw128(b_addr + 32 * t), idesc4,
                               tmem + sf_col + 4 * t, tmem + sf_col + 16 + t * Lay::kNC * 4,
@@ -294,72 +247,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0, kWaitLimitNs);  // every MMA done before TMEM can be freed
     }
-  } else if (GELU && warp >= 4) {
-    // GELU backward (FourTune §3.3 MLP): d_h = bf16(acc * GELU'(h)) -> out and
-    // bf16(GELU(h)) -> out2.  Four warps per TMEM lane quadrant, 64 columns each.
-    // GELU(h) does not need the accumulator: it is computed and stored while the
-    // tile's MMAs run, so the accumulator is held only for the d_h products.
-    // Rows are stored straight from registers (32 bytes per row and chunk).
-    constexpr int kCols = BN / 4;
-    const int q = warp & 3;
-    const int c_lo = ((warp - 4) >> 2) * kCols;
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c_lo);
-    int j = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
-      const int m0 = (tile / tiles_n) * 128, n0 = (tile % tiles_n) * BN + c_lo;
-      const int row = m0 + 32 * q + lane;
-      const bool row_ok = row < p.M;
-      uint4 hreg[kCols / 8];
-      const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.h) +
-                                                       static_cast<long long>(row) * p.N + n0);
-#pragma unroll
-      for (int k = 0; k < kCols / 8; ++k)
-        hreg[k] = (row_ok && n0 + 8 * k < p.N) ? hp[k] : make_uint4(0u, 0u, 0u, 0u);
-      uint4* g_out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out2) + static_cast<long long>(row) * p.ldo + n0);
-#pragma unroll
-      for (int k = 0; k < kCols / 8; ++k) {
-        const uint32_t hw[4] = {hreg[k].x, hreg[k].y, hreg[k].z, hreg[k].w};
-        uint32_t wg[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          wg[e] = pack_bf16x2(gelu_tanh(bf16_bits_to_f32(hw[e] & 0xFFFFu)), gelu_tanh(bf16_bits_to_f32(hw[e] >> 16)));
-        if (row_ok && n0 + 8 * k < p.N) g_out[k] = make_uint4(wg[0], wg[1], wg[2], wg[3]);
-      }
-      if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
-      __syncwarp();
-      tc_fence_after();
-      uint4* dh_out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(row) * p.ldo + n0);
-#pragma unroll 1
-      for (int c = 0; c < kCols / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(taddr + 16 * c, v);
-        tmem_ld_wait();
-        uint4 h0 = hreg[0], h1 = hreg[1];
-#pragma unroll
-        for (int k = 1; k < kCols / 16; ++k)
-          if (k == c) {
-            h0 = hreg[2 * k];
-            h1 = hreg[2 * k + 1];
-          }
-        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        uint32_t wd[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float g0, d0, g1, d1;
-          gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] & 0xFFFFu), &g0, &d0);
-          gelu_tanh_and_grad(bf16_bits_to_f32(hw[e] >> 16), &g1, &d1);
-          wd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
-        }
-        if (row_ok && n0 + 16 * c < p.N) {
-          dh_out[2 * c] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-          dh_out[2 * c + 1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-    }
-  } else if (!kCp && warp >= 12) {
+  } else if (warp >= 12) {
     // Scale warp of TMEM lane quadrant q.  Stage columns (from sf_col): A's
     // k-step t at 4t..4t+3, of which the MMA reads 4t+q here (the diagonal
     // word of the 512-byte block: rows 32q+lane, byte 16*lane + 4q); B's
@@ -428,7 +316,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
       if (gg + 2 < G) fetch(gg + 2, a0, b0);
       if (!put(gg + 1, a1, b1)) break;
     }
-  } else if (!GELU && warp >= 4) {
+  } else if (warp >= 4) {
     // two warps per TMEM lane quadrant, each owning half of the tile's columns
     const int q = warp & 3;
     const int c_lo = ((warp - 4) >> 2) * (BN / 2);
@@ -436,7 +324,7 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
     uint8_t* buf = epi + (warp - 4) * 1024;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const long long ldb = p.ldo * (p.out_bf16 ? 2 : 4);   // output row stride in bytes
-    const bool fast = !GELU && p.out_bf16;
+    const bool fast = p.out_bf16 != 0;
     int j = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
       if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
@@ -526,15 +414,13 @@ __global__ void __launch_bounds__(GELU ? kGmThreadsGelu : kGmThreads, 1)
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
-  if (p.epi_gelu_bwd && (!p.out_bf16 || p.main_bf16)) return cudaErrorInvalidValue;
-  auto kernel = p.epi_gelu_bwd ? gemm_fp4_kernel<BN, true> : gemm_fp4_kernel<BN, false>;
-  const uint32_t smem = p.epi_gelu_bwd ? GemmLayout<BN, true>::kSmem : GemmLayout<BN, false>::kSmem;
+  auto kernel = gemm_fp4_kernel<BN>;
+  const uint32_t smem = GemmLayout<BN>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = ((p.N + BN - 1) / BN) * ((p.M + 127) / 128);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(kernel, dim3(grid), dim3(p.epi_gelu_bwd ? kGmThreadsGelu : kGmThreads), smem, stream, tmA,
-                    tmB, tmA2, tmB2, p);
+  return launch_pdl(kernel, dim3(grid), dim3(kGmThreads), smem, stream, tmA, tmB, tmA2, tmB2, p);
 }
 
 }  // namespace ft

@@ -3,8 +3,9 @@
 // that the second one needs, so the hidden activation is never materialized).
 //
 //   epi 1, FC1 forward:  acc = Q(X) Q(R1)^T + L1 U1;  h = bf16(acc + b1) (saved
-//                        for the backward);  a = GELU_tanh(h) in fp32;
-//                        Q(a) (FC2's 4-bit input);  L2 = bf16(bf16(a) D2)
+//                        for the backward);  a = GELU_tanh(h) in fp32;  FC2's
+//                        input bf16(a) for all three of its branches:
+//                        Q(bf16(a)) and L2 = bf16(bf16(a) D2)
 //   epi 2, FC2 dX:       acc = Q(G) Q(R2) + P2 D2^T  (= d_a);
 //                        d_h = bf16(acc GELU'(h)) (saved for dB1);  Q(d_h)
 //                        (FC1's 4-bit gradient);  P1 = bf16(d_h U1^T)
@@ -24,13 +25,18 @@
 //   * at the end of a unit its fp32 partial [128, RP] goes to global memory;
 //     the last unit of a 128-row tile (a counter) sums the partials in split
 //     order (deterministic) and rounds once to bf16.
-// Shared memory: three 48 KB stages + the 64 KB T buffer.  TMEM: the 256-column
-// accumulator, two 48-column scale slots (a stage uses slot g % 2, rewritten
-// once the MMAs of stage g - 2 are done) and the projection accumulator.
+// Shared memory: three 48 KB stages, the 64 KB T buffer (which also stages h /
+// d_h for whole-row stores) and 1 KB of code scratch per epilogue warp (code
+// rows leave in 32-byte pieces, not 8).  TMEM: the 256-column accumulator, two
+// 48-column scale slots (a stage uses slot g % 2, rewritten once the MMAs of
+// stage g - 2 are done) and the projection accumulator.
 //
 // Warp roles: warp 0 lane 0 producer; warp 1 TMEM owner, lane 0 issues the
-// MMAs; warps 4..11 epilogue (warp w: TMEM lanes 32 (w % 4).., columns
-// 128 ((w - 4) / 4).. of the tile); warps 12..15 scale warps.
+// MMAs; warps 2..17 epilogue (warp w: TMEM lanes 32 (w % 4).., columns
+// 64 ((w - 2) / 4).. of the tile -- sixteen warps, so that the GELU and
+// quantizer arithmetic of one tile hides its latencies while the next tile's
+// MMAs run); warps 18..21 scale warps.  704 threads leave 80 registers per
+// thread.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,14 +45,23 @@ namespace ft {
 namespace {
 
 constexpr int kMlStages = 3;
-constexpr int kMlThreads = 512;
+constexpr int kMlEpiWarps = 16;
+constexpr int kMlEpiThreads = 32 * kMlEpiWarps;
+constexpr int kMlEpi0 = 2;                            // first epilogue warp
+constexpr int kMlScale0 = kMlEpi0 + kMlEpiWarps;      // first scale warp
+constexpr int kMlThreads = 32 * (kMlScale0 + 4);      // 704
+// Registers are allocated per warp from the register file quarter of the SM
+// sub-partition the warp runs on (16384 each): 22 warps put 6 on a quarter.
+constexpr int kMlMaxReg = 80;
+static_assert(((kMlThreads / 32 + 3) / 4) * 32 * kMlMaxReg <= 16384, "registers fit each sub-partition");
 constexpr int kMlBN = 256;
 constexpr uint32_t kMlA = 128 * 128;                  // A codes / A2 bf16 tile
 constexpr uint32_t kMlB = kMlBN * 128;                // B codes / B2 bf16 tile / projection weight
 constexpr uint32_t kMlStage = kMlA + kMlB;            // 48 KB
 constexpr uint32_t kMlT = 4 * 128 * 128;              // T: four [128 x 64] bf16 chunks
+constexpr uint32_t kMlCodes = kMlEpiWarps * 1024;     // per epilogue warp: its 32 rows x 32 bytes of Q(T) codes
 constexpr uint32_t kMlTail = 512;
-constexpr uint32_t kMlSmem = 1024 + kMlStages * kMlStage + kMlT + kMlTail;
+constexpr uint32_t kMlSmem = 1024 + kMlStages * kMlStage + kMlT + kMlCodes + kMlTail;
 constexpr int kMlSfSlots = 2;
 constexpr uint32_t kMlSfCols = 16 + 32;               // A's 4 k-steps x 4, B's 4 k-steps x 2 chunks x 4
 constexpr uint32_t kMlProjCol = kMlBN + kMlSfSlots * kMlSfCols;
@@ -68,7 +83,7 @@ __device__ __forceinline__ float max16_half(float a, int lane) {
 }  // namespace
 
 template <int EPI>
-__global__ void __launch_bounds__(kMlThreads, 1)
+__global__ void __maxnreg__(kMlMaxReg)
     gemm_mlp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const __grid_constant__ CUtensorMap tmW, const MlpGemmParams mp) {
@@ -76,7 +91,8 @@ __global__ void __launch_bounds__(kMlThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tbuf = smem + kMlStages * kMlStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tbuf + kMlT);
+  uint8_t* cbuf = tbuf + kMlT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + kMlCodes);
   uint64_t* empty = full + kMlStages;
   uint64_t* sf_full = empty + kMlStages;        // [kMlSfSlots] scale warps -> MMA
   uint64_t* sf_empty = sf_full + kMlSfSlots;    // [kMlSfSlots] MMAs that read the slot are done
@@ -114,8 +130,8 @@ __global__ void __launch_bounds__(kMlThreads, 1)
       mbar_init(&sf_empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
-    mbar_init(t_full, 8);
+    mbar_init(acc_empty, kMlEpiWarps);
+    mbar_init(t_full, kMlEpiWarps);
     mbar_init(t_empty, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -298,7 +314,7 @@ __global__ void __launch_bounds__(kMlThreads, 1)
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0, kWaitLimitNs);  // every MMA done before TMEM can be freed
     }
-  } else if (warp >= 12) {
+  } else if (warp >= kMlScale0) {
     // Scale warp of TMEM lane quadrant q: for an FP4 stage, A's k-step t at
     // columns 4t..4t+3 of the slot (the MMA reads 4t+q here), B's k-step t,
     // chunk c at 16+8t+4c..+3; stages without scales only pass the slot on.
@@ -332,22 +348,18 @@ __global__ void __launch_bounds__(kMlThreads, 1)
       }
     };
     // pass ring stage g: wait for its scale slot, write the scales (if any), hand it to the MMA
-    auto put = [&](const uint32_t* a, const uint32_t* b) -> bool {
+    auto put = [&](bool has, const uint32_t (&a)[4], const uint32_t (&b)[32]) -> bool {
       const int sl = g % kMlSfSlots;
       bool okw = true;
       if (lane == 0) okw = mbar_wait(&sf_empty[sl], ((g / kMlSfSlots) & 1) ^ 1, p.status, abortp);
       okw = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
       if (!okw) return false;
       tc_fence_after();
-      if (a) {
+      if (has) {
         const uint32_t sf_col = kMlBN + sl * kMlSfCols;
-        uint32_t a16[16], b32[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a16[e] = a[e >> 2];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) b32[e] = b[e];
-        tmem_st_32x32b_x16(trow + sf_col, a16);
-        tmem_st_32x32b_x32(trow + sf_col + 16, b32);
+        for (int t = 0; t < 4; ++t) tmem_st_32x32b_x4_rep(trow + sf_col + 4 * t, a[t]);
+        tmem_st_32x32b_x32(trow + sf_col + 16, b);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -361,33 +373,38 @@ __global__ void __launch_bounds__(kMlThreads, 1)
       const int mt = u / mp.nsplit, sp = u % mp.nsplit;
       const int nhi = min(tiles_n, (sp + 1) * mp.per);
       for (int nt = sp * mp.per; nt < nhi && ok; ++nt) {
-        // the tile's FP4 stages, the next one's loads in flight while one is stored
-        uint32_t a0[4], b0[32], a1[4], b1[32];
+        // the tile's FP4 stages: stage i + 1's words are loaded as soon as stage
+        // i's are in TMEM (one stage in registers: 80 registers leave no room
+        // for two without spilling)
+        uint32_t a0[4], b0[32];
         if (KB > 0) fetch(mt, nt, 0, a0, b0);
-        for (int i = 0; i < KB && ok; i += 2) {
-          if (i + 1 < KB) fetch(mt, nt, i + 1, a1, b1);
-          ok = put(a0, b0);
-          if (!ok || i + 1 >= KB) break;
-          if (i + 2 < KB) fetch(mt, nt, i + 2, a0, b0);
-          ok = put(a1, b1);
+        for (int i = 0; i < KB && ok; ++i) {
+          ok = put(true, a0, b0);
+          if (ok && i + 1 < KB) fetch(mt, nt, i + 1, a0, b0);
         }
-        for (int i = 0; i < EB && ok; ++i) ok = put(nullptr, nullptr);
-        for (int i = 0; have_prev && i < kMlProjStages && ok; ++i) ok = put(nullptr, nullptr);
+        for (int i = 0; i < EB && ok; ++i) ok = put(false, a0, b0);
+        for (int i = 0; have_prev && i < kMlProjStages && ok; ++i) ok = put(false, a0, b0);
         have_prev = true;
       }
     }
-    for (int i = 0; have_prev && i < kMlProjStages && ok; ++i) ok = put(nullptr, nullptr);
-  } else if (warp >= 4) {
-    // ---- epilogue: 8 warps; warp w owns rows 32 q.. (q = w % 4) of the tile and
-    // columns c_lo .. c_lo + 127.  The eight warps leave together (named_bar_or).
+    {
+      uint32_t a0[4] = {0u, 0u, 0u, 0u}, b0[32];
+      for (int i = 0; have_prev && i < kMlProjStages && ok; ++i) ok = put(false, a0, b0);
+    }
+  } else if (warp >= kMlEpi0) {
+    // ---- epilogue: 16 warps; warp w owns rows 32 q.. (q = w % 4: the TMEM lane
+    // quadrant a warp may access) of the tile and columns c_lo .. c_lo + 63.  The
+    // sixteen warps leave together (named_bar_or).
+    const int et = static_cast<int>(threadIdx.x) - 32 * kMlEpi0;   // 0 .. 511
     const int q = warp & 3;
-    const int c_lo = ((warp - 4) >> 2) * 128;
+    const int cq = (warp - kMlEpi0) >> 2;
+    const int c_lo = 64 * cq;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c_lo);
     const uint32_t paddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + kMlProjCol;
     const int r_loc = 32 * q + lane;                        // this lane's row of the tile
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
-    const int half = RP / 2;                                // projection columns of this warp's half
-    const int pc0 = ((warp - 4) >> 2) * half;
+    const int quarter = RP / 4;                             // projection columns of this warp (a multiple of 4)
+    const int pc0 = cq * quarter;
     int j = 0;
     int prev_m0 = 0, prev_sp = 0;
     bool have_prev = false, prev_last = false;
@@ -396,15 +413,15 @@ __global__ void __launch_bounds__(kMlThreads, 1)
     // 128-row tile sums all partials in split order and rounds to bf16.
     auto finish_unit = [&](int m0, int sp) {
       const int row = m0 + r_loc;
-      for (int c = 0; c < half; c += 16) {
+      for (int c = 0; c < quarter; c += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(paddr + pc0 + c, v);
         tmem_ld_wait();
         if (row < p.M) {
           float4* dst = reinterpret_cast<float4*>(mp.part + (static_cast<long long>(sp) * p.M + row) * RP + pc0 + c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)   // this warp's columns only (half is a multiple of 8)
-            if (c + 4 * e < half)
+          for (int e = 0; e < 4; ++e)   // this warp's columns only
+            if (c + 4 * e < quarter)
               dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
@@ -412,22 +429,38 @@ __global__ void __launch_bounds__(kMlThreads, 1)
       // one thread publishes this unit's partial (ordered before it by the
       // barrier) with a gpu-scope fence before its counter increment; the last
       // unit's fence after the increment orders its reads after all others
-      named_bar_sync(1, 256);
-      if (threadIdx.x == 128) {
+      named_bar_sync(1, kMlEpiThreads);
+      if (et == 0) {
         __threadfence();
         const int prev = atomicAdd(&mp.counters[m0 / 128], 1);
         __threadfence();
         *s_last = (prev == mp.nsplit - 1);
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kMlEpiThreads);
       if (*s_last) {
         const int c4 = RP / 4;
-        for (int idx = static_cast<int>(threadIdx.x) - 128; idx < 128 * c4; idx += 256) {
+        for (int idx = et; idx < 128 * c4; idx += kMlEpiThreads) {
           const int rr = m0 + idx / c4, cc = 4 * (idx % c4);
           if (rr >= p.M) continue;
+          // split order, four loads in flight at a time
+          const float4* src = reinterpret_cast<const float4*>(mp.part + static_cast<long long>(rr) * RP + cc);
+          const long long stride4 = static_cast<long long>(p.M) * RP / 4;
           float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          for (int s2 = 0; s2 < mp.nsplit; ++s2) {
-            const float4 x = __ldcg(reinterpret_cast<const float4*>(mp.part + (static_cast<long long>(s2) * p.M + rr) * RP + cc));
+          int s2 = 0;
+          for (; s2 + 4 <= mp.nsplit; s2 += 4) {
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = __ldcg(src + (s2 + k) * stride4);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              acc.x += x[k].x;
+              acc.y += x[k].y;
+              acc.z += x[k].z;
+              acc.w += x[k].w;
+            }
+          }
+          for (; s2 < mp.nsplit; ++s2) {
+            const float4 x = __ldcg(src + s2 * stride4);
             acc.x += x.x;
             acc.y += x.y;
             acc.z += x.z;
@@ -436,10 +469,15 @@ __global__ void __launch_bounds__(kMlThreads, 1)
           *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(mp.proj_out) + static_cast<long long>(rr) * RP + cc) =
               make_uint2(ml_pack_bf16x2(acc.x, acc.y), ml_pack_bf16x2(acc.z, acc.w));
         }
-        if (threadIdx.x == 128) mp.counters[m0 / 128] = 0;
+        if (et == 0) mp.counters[m0 / 128] = 0;
       }
     };
 
+    // this lane's row of T: chunk cq (the warp's 64 columns), 128-byte swizzled
+    uint8_t* const t_row = tbuf + cq * 16384 + r_loc * 128;
+    const int sw = r_loc & 7;
+    uint8_t* const cbase = cbuf + (warp - kMlEpi0) * 1024;   // the warp's code scratch
+    uint8_t* const c_row = cbase + lane * 32;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int m0 = (u / mp.nsplit) * 128, sp = u % mp.nsplit;
@@ -448,12 +486,18 @@ __global__ void __launch_bounds__(kMlThreads, 1)
         const int n0 = nt * kMlBN + c_lo;                   // this warp's first column
         const int row = m0 + r_loc;
         const bool row_ok = row < p.M;
-        uint32_t hw[64];                                    // the warp's 128 columns of h / d_h (bf16 pairs)
-        if (EPI == 2) {                                     // h, loaded while the tile's MMAs run
+        // loaded while the tile's MMAs run: EPI 1 the bias of the warp's 64
+        // columns (lane l < 8 holds columns n0 + 8 l .. + 7; shuffled out
+        // below), EPI 2 the lane's row of h
+        uint4 bq = make_uint4(0u, 0u, 0u, 0u);
+        uint32_t hw[32];
+        if (EPI == 1) {
+          if (bias && n0 + 8 * (lane & 7) < p.N) bq = __ldg(reinterpret_cast<const uint4*>(bias + n0) + (lane & 7));
+        } else {
           const uint4* hp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(mp.h) +
                                                            static_cast<long long>(row) * p.N + n0);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             const uint4 x = (row_ok && n0 + 8 * k < p.N) ? hp[k] : make_uint4(0u, 0u, 0u, 0u);
             hw[4 * k] = x.x;
             hw[4 * k + 1] = x.y;
@@ -462,131 +506,135 @@ __global__ void __launch_bounds__(kMlThreads, 1)
           }
         }
         const bool got = mbar_wait(acc_full, j & 1, p.status, abortp);
-        if (named_bar_or(1, 256, !got || *abortp)) {
+        if (named_bar_or(1, kMlEpiThreads, !got || *abortp)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (EPI == 1) {
-          // h = bf16(acc + b1), 32 columns per round
-#pragma unroll
-          for (int rd = 0; rd < 4; ++rd) {
-            uint32_t v[2][16];
-            tmem_ld_32x32b_x16(taddr + 32 * rd, v[0]);
-            tmem_ld_32x32b_x16(taddr + 32 * rd + 16, v[1]);
-            uint4 bw[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              bw[k] = make_uint4(0u, 0u, 0u, 0u);
-              if (bias && n0 + 32 * rd + 8 * k < p.N) bw[k] = __ldg(reinterpret_cast<const uint4*>(bias + n0 + 32 * rd) + k);
-            }
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const uint4 b4 = bw[2 * k + e / 4];
-                const uint32_t bb = (e & 3) == 0 ? b4.x : (e & 3) == 1 ? b4.y : (e & 3) == 2 ? b4.z : b4.w;
-                hw[16 * rd + 8 * k + e] = ml_pack_bf16x2(__uint_as_float(v[k][2 * e]) + bf16_bits_to_f32(bb & 0xFFFFu),
-                                                         __uint_as_float(v[k][2 * e + 1]) + bf16_bits_to_f32(bb >> 16));
-              }
-            }
-          }
-        } else {
-          // d_h = bf16(acc * GELU'(h)), 16 columns per round, in place of h
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(taddr + 16 * c, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float g0, d0, g1, d1;
-              gelu_tanh_and_grad(bf16_bits_to_f32(hw[8 * c + e] & 0xFFFFu), &g0, &d0);
-              gelu_tanh_and_grad(bf16_bits_to_f32(hw[8 * c + e] >> 16), &g1, &d1);
-              hw[8 * c + e] = ml_pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
-        // h (FC1) or d_h (FC2 dX): each lane stores its row, 32-byte pieces
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(mp.out_h) + static_cast<long long>(row) * p.N + n0);
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (n0 + 8 * k < p.N) dst[k] = make_uint4(hw[4 * k], hw[4 * k + 1], hw[4 * k + 2], hw[4 * k + 3]);
-        }
-        // T is free once the previous tile's projection is done; a unit that
-        // ended with the previous tile hands its accumulator on first
+        // T is free once the previous tile's projection is done (it runs right
+        // after this tile's main loop); a unit that ended with the previous
+        // tile hands its projection accumulator on first
         if (have_prev) {
           const bool freed = mbar_wait(t_empty, (j - 1) & 1, p.status, abortp);
-          if (named_bar_or(1, 256, !freed || *abortp)) {
+          if (named_bar_or(1, kMlEpiThreads, !freed || *abortp)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (prev_last) finish_unit(prev_m0, prev_sp);
-        }
-        // per 16-column block: Q(.) codes and scales, T = the projection's input
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int col = n0 + 16 * c;
-          float v[16];
-          uint32_t tw[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            v[2 * e] = bf16_bits_to_f32(hw[8 * c + e] & 0xFFFFu);
-            v[2 * e + 1] = bf16_bits_to_f32(hw[8 * c + e] >> 16);
+          if (prev_last) {
+            tc_fence_after();
+            finish_unit(prev_m0, prev_sp);
           }
+        }
+        tc_fence_after();
+        // ---- phase 1, 16 columns at a time: the accumulator -> h = bf16(acc + b1)
+        // (EPI 1) or d_h = bf16(acc GELU'(h)) (EPI 2), to global memory and to T
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {   // rolled: the epilogue's code stays small
+          const int col = n0 + 16 * c;
+          uint32_t v[16], w[8];
+          tmem_ld_32x32b_x16(taddr + 16 * c, v);
+          tmem_ld_wait();
           if (EPI == 1) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = gelu_tanh(v[e]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) tw[e] = ml_pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t part = (e & 3) == 0 ? bq.x : (e & 3) == 1 ? bq.y : (e & 3) == 2 ? bq.z : bq.w;
+              const uint32_t bb = __shfl_sync(0xFFFFFFFFu, part, 2 * c + (e >> 2));
+              w[e] = ml_pack_bf16x2(__uint_as_float(v[2 * e]) + bf16_bits_to_f32(bb & 0xFFFFu),
+                                    __uint_as_float(v[2 * e + 1]) + bf16_bits_to_f32(bb >> 16));
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) tw[e] = hw[8 * c + e];
+            for (int e = 0; e < 8; ++e) {
+              float g0, d0, g1, d1;
+              const uint32_t hh = hw[e];
+              gelu_tanh_and_grad(bf16_bits_to_f32(hh & 0xFFFFu), &g0, &d0);
+              gelu_tanh_and_grad(bf16_bits_to_f32(hh >> 16), &g1, &d1);
+              w[e] = ml_pack_bf16x2(__uint_as_float(v[2 * e]) * d0, __uint_as_float(v[2 * e + 1]) * d1);
+            }
+#pragma unroll
+            for (int e = 0; e < 24; ++e) hw[e] = hw[e + 8];   // the next 16 columns to the front
           }
+          if (EPI == 2 && !(row_ok && col < p.N)) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = 0u;   // T: zero outside the matrix
+          }
+          *reinterpret_cast<uint4*>(t_row + (((2 * c) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(t_row + (((2 * c + 1) ^ sw) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);   // the next tile's MMAs may start
+        // h / d_h to global memory from T: the warp's 32 rows x 128 bytes, four
+        // whole rows (512 contiguous-by-row bytes) per store
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 32 * q + 4 * i + (lane >> 3), un = lane & 7;
+          const uint4 x = *reinterpret_cast<const uint4*>(tbuf + cq * 16384 + rr * 128 + ((un ^ (rr & 7)) << 4));
+          if (m0 + rr < p.M && n0 + 8 * un < p.N)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(mp.out_h) + static_cast<long long>(m0 + rr) * p.N +
+                                      n0 + 8 * un) = x;
+        }
+        // ---- phase 2, per 16-column block of T: (EPI 1: T = bf16(GELU(h)) in
+        // place) the block's Q(T) codes and scale, T being the shared bf16 input
+        // of the next layer's branches (bf16(a) or d_h)
+        uint32_t sfw = 0u;
+        __syncwarp();   // the previous tile's reads of the code scratch are done
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const int col = n0 + 16 * c;
           const bool inside = row_ok && col < p.N;
-          if (!inside) {
+          uint4* const tp0 = reinterpret_cast<uint4*>(t_row + (((2 * c) ^ sw) << 4));
+          uint4* const tp1 = reinterpret_cast<uint4*>(t_row + (((2 * c + 1) ^ sw) << 4));
+          const uint4 x0 = *tp0, x1 = *tp1;
+          uint32_t tw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          if (EPI == 1) {
+            float2* dbg = (mp.dbg && inside) ? reinterpret_cast<float2*>(mp.dbg + static_cast<long long>(row) * p.N + col)
+                                             : nullptr;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+            for (int e = 0; e < 8; ++e) {
+              const float a0 = gelu_tanh(bf16_bits_to_f32(tw[e] & 0xFFFFu));
+              const float a1 = gelu_tanh(bf16_bits_to_f32(tw[e] >> 16));
+              tw[e] = inside ? ml_pack_bf16x2(a0, a1) : 0u;
+              if (dbg) dbg[e] = make_float2(a0, a1);
+            }
+            *tp0 = make_uint4(tw[0], tw[1], tw[2], tw[3]);
+            *tp1 = make_uint4(tw[4], tw[5], tw[6], tw[7]);
+          }
+          float v[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) tw[e] = 0u;
+          for (int e = 0; e < 8; ++e) {
+            v[2 * e] = bf16_bits_to_f32(tw[e] & 0xFFFFu);
+            v[2 * e + 1] = bf16_bits_to_f32(tw[e] >> 16);
           }
           float m = 0.0f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
           const float amax = max16_half(m, lane);           // the 16x16 block: 16 rows = 16 lanes
           uint32_t packed[2], sc;
-          if (EPI == 1)
-            quantize_block_row_f32<16>(v, amax, packed, &sc);
-          else
-            quantize_block_row<16>(v, amax, packed, &sc);
-          if (inside) {
-            *reinterpret_cast<uint2*>(mp.q_codes + static_cast<long long>(row) * (p.N / 2) + col / 2) =
-                make_uint2(packed[0], packed[1]);
-            if ((lane & 15) == 0)
-              mp.q_scales[static_cast<long long>(row / 16) * (p.N / 16) + col / 16] = static_cast<uint8_t>(sc);
-            if (EPI == 1 && mp.dbg) {
-              float4* dst = reinterpret_cast<float4*>(mp.dbg + static_cast<long long>(row) * p.N + col);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-            }
-          }
-          // MMA-ready copy: every row of the block; groups past N inside the last
-          // 64-column step and rows past M hold 0
-          if (mp.q_sf && col / 16 < 4 * KSo)
-            mp.q_sf[sf_mma_offset(row, col / 16, KSo)] = static_cast<uint8_t>(inside ? sc : 0u);
-          // T chunk (c_lo + 16 c) / 64, 16-byte units u, u + 1 of row r_loc, 128-byte swizzle
-          const int cl = c_lo + 16 * c;
-          uint8_t* trow = tbuf + (cl / 64) * 16384 + r_loc * 128;
-          const int u0 = (cl % 64) / 8;
-          *reinterpret_cast<uint4*>(trow + ((u0 ^ (r_loc & 7)) << 4)) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
-          *reinterpret_cast<uint4*>(trow + (((u0 + 1) ^ (r_loc & 7)) << 4)) = make_uint4(tw[4], tw[5], tw[6], tw[7]);
+          quantize_block_row<16>(v, amax, packed, &sc);      // bf16 values: the exact division-free path
+          if (!inside) sc = 0u;
+          sfw |= sc << (8 * c);
+          // codes into the warp's scratch: row `lane`, 8-byte unit c at
+          // position c ^ ((lane >> 2) & 3) (16 lanes cover the 32 banks)
+          *reinterpret_cast<uint2*>(c_row + 8 * (c ^ ((lane >> 2) & 3))) = make_uint2(packed[0], packed[1]);
+          if (inside && (lane & 15) == 0)
+            mp.q_scales[static_cast<long long>(row / 16) * (p.N / 16) + col / 16] = static_cast<uint8_t>(sc);
         }
+        __syncwarp();
+        // the codes of the warp's 32 rows x 64 columns: 32 bytes a row, two
+        // rows per lane pair, 16 bytes (32 columns) per lane
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int lr = 16 * i + (lane >> 1), hf = lane & 1, x = (lr >> 2) & 3;
+          uint4 v4 = *reinterpret_cast<const uint4*>(cbase + lr * 32 + 16 * (hf ^ (x >> 1)));
+          if (x & 1) v4 = make_uint4(v4.z, v4.w, v4.x, v4.y);   // the pair's two units stored swapped
+          const int rr = m0 + 32 * q + lr;
+          if (rr < p.M && n0 + 32 * hf < p.N)
+            *reinterpret_cast<uint4*>(mp.q_codes + static_cast<long long>(rr) * (p.N / 2) + n0 / 2 + 16 * hf) = v4;
+        }
+        // the MMA-ready copy of the scales: the warp's k-step, four scales of
+        // this row in one word (rows past M and groups past N hold 0)
+        if (mp.q_sf && n0 < 64 * KSo)
+          *reinterpret_cast<uint32_t*>(mp.q_sf + sf_mma_offset(row, n0 / 16, KSo)) = sfw;
         fence_proxy_async_smem();   // T's generic stores -> the tensor cores' reads
         tc_fence_before();          // the projection accumulator was read out before
         __syncwarp();
@@ -599,7 +647,7 @@ __global__ void __launch_bounds__(kMlThreads, 1)
     }
     if (ok && have_prev) {
       const bool freed = mbar_wait(t_empty, (j - 1) & 1, p.status, abortp);
-      if (!named_bar_or(1, 256, !freed || *abortp)) {
+      if (!named_bar_or(1, kMlEpiThreads, !freed || *abortp)) {
         tc_fence_after();
         finish_unit(prev_m0, prev_sp);
       }
@@ -621,7 +669,8 @@ cudaError_t launch_gemm_mlp(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
   if ((p.epi != 1 && p.epi != 2) || p.RP < 16 || p.RP > 128 || p.RP % 16 || p.nsplit < 1 || p.per < 1)
     return cudaErrorInvalidValue;
   auto kernel = p.epi == 1 ? gemm_mlp_kernel<1> : gemm_mlp_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMlSmem));
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMlSmem));
   if (e != cudaSuccess) return e;
   const int units = ((p.g.M + 127) / 128) * p.nsplit;
   const int grid = units < num_sms ? units : num_sms;

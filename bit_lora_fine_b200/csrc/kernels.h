@@ -15,8 +15,6 @@ struct RowpassParams {
   int w_mn_major;                        // 1: D [K, R]; 0: W^T [R, K]
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
   int stages;                            // TMA ring depth, 2..rowpass_stages()
-  int gelu_input;                        // input is h: quantize a = GELU(h) (fp32) and project bf16(a)
-  float* dbg_a;                          // gelu_input: optional fp32 copy of a [M, K] (null = none)
   int no_quant;                          // only L: no codes or scales (the 16-bit precision variants)
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
@@ -55,11 +53,6 @@ struct GemmParams {
   void* out;
   long long ldo;
   int out_bf16;
-  // GELU-backward epilogue: out = bf16(acc * GELU'(h)), out2 = bf16(GELU(h)),
-  // h bf16 [M, N] with row stride N (both outputs bf16, row stride ldo)
-  int epi_gelu_bwd;
-  const void* h;
-  void* out2;
   int* status;
   // 16-bit main product (the precision variants): A [M, K] and B [N, K] are
   // bf16 (K contiguous) instead of block16 codes; sfa, sfb unused

@@ -55,7 +55,7 @@ __host__ __device__ constexpr uint32_t rp_smem_bytes(int R, int mn, int stages) 
   return 1024 + stages * rp_stage_bytes(R, mn) + kRpTail;
 }
 
-template <int RCOLS, bool GELU>
+template <int RCOLS>
 __global__ void __launch_bounds__(kRpThreads, 1)
     rowpass_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const RowpassParams p) {
@@ -70,8 +70,7 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * stage_bytes);
   uint64_t* empty = full + NS;
   uint64_t* acc_full = empty + NS;
-  uint64_t* ready = acc_full + 1;  // [NS] GELU mode: transformed tile written back
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_last = abort_flag + 1;
   volatile int* s_ok = s_last + 1;  // [kRpQuantWarps]
@@ -93,7 +92,6 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + kRpQuantWarps);  // MMA commit + one arrive per quantizer warp
-      mbar_init(&ready[s], kRpQuantWarps);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -146,7 +144,6 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       uint32_t ph = 0;
       for (int i = 0; i < nt; ++i, s = (s + 1 == NS) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
         if (!mbar_wait(&full[s], ph, p.status, abortp, lim)) break;
-        if (GELU && !mbar_wait(&ready[s], ph, p.status, abortp, lim)) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(smem + s * stage_bytes);
         const uint32_t wa = xa + kRpXBytes;
@@ -189,31 +186,8 @@ __global__ void __launch_bounds__(kRpThreads, 1)
           v[q * 8 + 2 * e + 1] = bf16_bits_to_f32(wd[e] >> 16);
         }
       }
-      if (GELU) {
-        // a = GELU(h) in fp32; bf16(a) goes back into the tile for the down-projection
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = gelu_tanh(v[e]);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t wd[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
-            wd[e] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          const int phys = (colw / 8 + q) ^ (r & 7);
-          *reinterpret_cast<uint4*>(tile + r * 128 + phys * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&ready[s]);
-          mbar_arrive(&empty[s]);
-        }
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // the tile is in registers: release the stage early
       float m[8];                               // this lane's 16 magnitudes, tree-reduced
 #pragma unroll
       for (int e = 0; e < 8; ++e) m[e] = fmaxf(fabsf(v[e]), fabsf(v[e + 8]));
@@ -227,20 +201,12 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       if (!p.no_quant && (inside || p.sf_mma)) {
         // rows past M and columns past K were zero-filled by the TMA: their scale is 0
         uint32_t packed[2], sc;
-        if (GELU)
-          quantize_1block_f32(v, amax, packed, &sc);
-        else
-          quantize_1block(v, amax, packed, &sc);
+        quantize_1block(v, amax, packed, &sc);
         if (inside) {
           *reinterpret_cast<uint2*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
               make_uint2(packed[0], packed[1]);
           if ((lane >> 1) == 0)
             p.scales[(m0 / 16 + blk) * static_cast<long long>(kblocks) + cstart / 16] = static_cast<uint8_t>(sc);
-          if (GELU && p.dbg_a) {
-            float4* dst = reinterpret_cast<float4*>(p.dbg_a + static_cast<long long>(m0 + r) * p.K + cstart);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          }
         }
         if (p.sf_mma) {
           // MMA-ready copy: group colw/16 of k-step kt0+i for row r of chunk blockIdx.x
@@ -369,15 +335,15 @@ __global__ void __launch_bounds__(kRpThreads, 1)
   }
 }
 
-template <int RCOLS, bool GELU>
+template <int RCOLS>
 static cudaError_t launch_rowpass_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
                                     cudaStream_t stream) {
   const uint32_t smem = rp_smem_bytes(p.R, p.w_mn_major, p.stages);
-  cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS, GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(rowpass_kernel<RCOLS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(rowpass_kernel<RCOLS, GELU>, dim3((p.M + 127) / 128, p.nsplit), dim3(kRpThreads), smem, stream,
-                    tmX, tmW, p);
+  return launch_pdl(rowpass_kernel<RCOLS>, dim3((p.M + 127) / 128, p.nsplit), dim3(kRpThreads), smem, stream, tmX,
+                    tmW, p);
 }
 
 cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const RowpassParams& p,
@@ -385,14 +351,9 @@ cudaError_t launch_rowpass(const CUtensorMap& tmX, const CUtensorMap& tmW, const
   if (p.stages < 2 || p.stages > kRpStages || rp_smem_bytes(p.R, p.w_mn_major, p.stages) > 232448u)
     return cudaErrorInvalidValue;
   const int n = rp_n_mma(p.R, p.w_mn_major);
-  if (p.gelu_input) {
-    if (n <= 32) return launch_rowpass_t<32, true>(tmX, tmW, p, stream);
-    if (n <= 64) return launch_rowpass_t<64, true>(tmX, tmW, p, stream);
-    return launch_rowpass_t<128, true>(tmX, tmW, p, stream);
-  }
-  if (n <= 32) return launch_rowpass_t<32, false>(tmX, tmW, p, stream);
-  if (n <= 64) return launch_rowpass_t<64, false>(tmX, tmW, p, stream);
-  return launch_rowpass_t<128, false>(tmX, tmW, p, stream);
+  if (n <= 32) return launch_rowpass_t<32>(tmX, tmW, p, stream);
+  if (n <= 64) return launch_rowpass_t<64>(tmX, tmW, p, stream);
+  return launch_rowpass_t<128>(tmX, tmW, p, stream);
 }
 
 int rowpass_stages(int R, int w_mn_major) {

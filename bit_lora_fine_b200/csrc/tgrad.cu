@@ -22,7 +22,8 @@
 namespace ft {
 
 constexpr int kTgStages = 4;
-constexpr int kTgThreads = 256;
+constexpr int kTgThreads = 384;        // warps 4..11 transform T when t_gelu; 4..7 also drain the accumulator
+constexpr int kTgXWarps = 8;
 constexpr uint32_t kTgTBox = 128 * 128;            // 128 m rows x 64 bf16
 constexpr uint32_t kTgStage = 2 * kTgTBox + kTgTBox;  // T (two boxes) + V
 constexpr uint32_t kTgSmem = 1024 + kTgStages * kTgStage + 256;
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     for (int s = 0; s < kTgStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&ready[s], 4);
+      mbar_init(&ready[s], kTgXWarps);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -130,8 +131,9 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   } else if (warp >= 4) {
     bool ok = true;
     if (p.t_gelu) {
-      // the T part of every stage (two 16 KB boxes of bf16 h) -> bf16(GELU(h)), in place
-      const int t = static_cast<int>(threadIdx.x) - 128;   // 0..127
+      // the T part of every stage (two 16 KB boxes of bf16 h) -> bf16(GELU(h)), in
+      // place, by eight warps (enough in flight to hide the exponential's latency)
+      const int t = static_cast<int>(threadIdx.x) - 128;   // 0..255
       for (int i = 0; i < nt && ok; ++i) {
         const int s = i % kTgStages;
         bool okw = true;
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         if (!ok) break;
         uint4* tile = reinterpret_cast<uint4*>(smem + s * kTgStage);
 #pragma unroll 4
-        for (int k = t; k < static_cast<int>(2 * kTgTBox / 16); k += 128) {
+        for (int k = t; k < static_cast<int>(2 * kTgTBox / 16); k += 32 * kTgXWarps) {
           uint4 x = tile[k];
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -156,94 +158,96 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         if (lane == 0) mbar_arrive(&ready[s]);
       }
     }
-    const bool mine = ok && (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
-    if (lane == 0) s_ok[warp - 4] = mine ? 1 : 0;
-    named_bar_sync(1, 128);
-    const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
-    if (go) {
-      __syncwarp();
-      tc_fence_after();
-      const int q = warp & 3;
-      const int prow = pbase + 32 * q + lane;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      float acc[64];
-      {
-        uint32_t a[32], b[32];
-        tmem_ld_32x32b_x32(taddr, a);
-        tmem_ld_32x32b_x32(taddr + 32, b);
-        tmem_ld_wait();
+    if (warp < 8) {   // warps 8..11 only transform
+      const bool mine = ok && (nt > 0) && mbar_wait(acc_full, 0, p.status, abortp);
+      if (lane == 0) s_ok[warp - 4] = mine ? 1 : 0;
+      named_bar_sync(1, 128);
+      const bool go = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
+      if (go) {
+        __syncwarp();
+        tc_fence_after();
+        const int q = warp & 3;
+        const int prow = pbase + 32 * q + lane;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        float acc[64];
+        {
+          uint32_t a[32], b[32];
+          tmem_ld_32x32b_x32(taddr, a);
+          tmem_ld_32x32b_x32(taddr + 32, b);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          acc[e] = __uint_as_float(a[e]);
-          acc[32 + e] = __uint_as_float(b[e]);
+          for (int e = 0; e < 32; ++e) {
+            acc[e] = __uint_as_float(a[e]);
+            acc[32 + e] = __uint_as_float(b[e]);
+          }
         }
-      }
-      bool write = true;
-      if (p.nsplit > 1) {
-        // only the r columns that are output travel through the partials
-        const int nq = (p.r + 3) / 4;
-        float4* dst = reinterpret_cast<float4*>(p.part + (static_cast<long long>(split) * Ppad + prow) * 64);
+        bool write = true;
+        if (p.nsplit > 1) {
+          // only the r columns that are output travel through the partials
+          const int nq = (p.r + 3) / 4;
+          float4* dst = reinterpret_cast<float4*>(p.part + (static_cast<long long>(split) * Ppad + prow) * 64);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (e < nq) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-        // one thread publishes the CTA's partial (ordered before it by the
-        // barrier) with a gpu-scope fence before the counter increment; the last
-        // CTA's fence after the increment orders its partial reads after all others
-        named_bar_sync(1, 128);
-        if (threadIdx.x == 128) {
-          __threadfence();
-          const int prev = atomicAdd(&p.counters[ptile], 1);
-          __threadfence();
-          *s_last = (prev == p.nsplit - 1);
-        }
-        named_bar_sync(1, 128);
-        write = *s_last != 0;
-        if (write) {
-          // sum every split's partial row in split order (vector loads, registers
-          // only), two splits' loads in flight at a time
+          for (int e = 0; e < 16; ++e)
+            if (e < nq) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+          // one thread publishes the CTA's partial (ordered before it by the
+          // barrier) with a gpu-scope fence before the counter increment; the last
+          // CTA's fence after the increment orders its partial reads after all others
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 128) {
+            __threadfence();
+            const int prev = atomicAdd(&p.counters[ptile], 1);
+            __threadfence();
+            *s_last = (prev == p.nsplit - 1);
+          }
+          named_bar_sync(1, 128);
+          write = *s_last != 0;
+          if (write) {
+            // sum every split's partial row in split order (vector loads, registers
+            // only), two splits' loads in flight at a time
 #pragma unroll
-          for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-          for (int sp = 0; sp < p.nsplit; sp += 2) {
-            const float4* src0 = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
-            const float4* src1 = src0 + static_cast<long long>(Ppad) * 16;
-            const bool two = sp + 1 < p.nsplit;
+            for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+            for (int sp = 0; sp < p.nsplit; sp += 2) {
+              const float4* src0 = reinterpret_cast<const float4*>(p.part + (static_cast<long long>(sp) * Ppad + prow) * 64);
+              const float4* src1 = src0 + static_cast<long long>(Ppad) * 16;
+              const bool two = sp + 1 < p.nsplit;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {   // 8 float4 of each split per round (registers)
-              float4 x0[8], x1[8];
+              for (int h = 0; h < 2; ++h) {   // 8 float4 of each split per round (registers)
+                float4 x0[8], x1[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (8 * h + e < nq) {
-                  x0[e] = __ldcg(src0 + 8 * h + e);
-                  if (two) x1[e] = __ldcg(src1 + 8 * h + e);
+                for (int e = 0; e < 8; ++e) {
+                  if (8 * h + e < nq) {
+                    x0[e] = __ldcg(src0 + 8 * h + e);
+                    if (two) x1[e] = __ldcg(src1 + 8 * h + e);
+                  }
                 }
-              }
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (8 * h + e < nq) {
-                  const int c = 4 * (8 * h + e);
-                  acc[c] += x0[e].x;
-                  acc[c + 1] += x0[e].y;
-                  acc[c + 2] += x0[e].z;
-                  acc[c + 3] += x0[e].w;
-                  if (two) {
-                    acc[c] += x1[e].x;
-                    acc[c + 1] += x1[e].y;
-                    acc[c + 2] += x1[e].z;
-                    acc[c + 3] += x1[e].w;
+                for (int e = 0; e < 8; ++e) {
+                  if (8 * h + e < nq) {
+                    const int c = 4 * (8 * h + e);
+                    acc[c] += x0[e].x;
+                    acc[c + 1] += x0[e].y;
+                    acc[c + 2] += x0[e].z;
+                    acc[c + 3] += x0[e].w;
+                    if (two) {
+                      acc[c] += x1[e].x;
+                      acc[c + 1] += x1[e].y;
+                      acc[c + 2] += x1[e].z;
+                      acc[c + 3] += x1[e].w;
+                    }
                   }
                 }
               }
             }
+            if (threadIdx.x == 128) p.counters[ptile] = 0;
           }
-          if (threadIdx.x == 128) p.counters[ptile] = 0;
         }
-      }
-      if (write && prow < p.P) {
+        if (write && prow < p.P) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          if (j < p.r) {
-            float* o = p.out + prow * p.out_sp + j * p.out_sj;
-            *o = p.accumulate ? *o + acc[j] : acc[j];
+          for (int j = 0; j < 64; ++j) {
+            if (j < p.r) {
+              float* o = p.out + prow * p.out_sp + j * p.out_sj;
+              *o = p.accumulate ? *o + acc[j] : acc[j];
+            }
           }
         }
       }
