@@ -13,7 +13,9 @@ quantized on its own (§3.2's contrast with the block layout).
 Readings (the pages fix neither):
   * per-tensor scale s_t = 2^e, the smallest power of two with
     amax(T) / (6 * 2^e) <= 448 (the E4M3 maximum), i.e. the power of two at or
-    above amax / 2688; amax = 0 gives e = 0.  A power of two keeps every step
+    above amax / 2688; amax = 0 gives e = 0, and e is at least -126 (so that
+    2^-e is a float32 number; only a tensor whose largest magnitude is below
+    2688 * 2^-127 ~ 1e-35 meets the bound).  A power of two keeps every step
     below exact: T' = T * 2^-e changes no significand (float32 rounding only
     if an element lands below 2^-126), and the GEMM's output scale
     s_tA * s_tB is an exact multiply.
@@ -38,10 +40,12 @@ E2M1_MAX = 6.0
 
 def tensor_exponent(amax: float) -> int:
     """The exponent e of the per-tensor scale 2^e: the least integer with
-    amax <= 2688 * 2^e (2688 = 6 * 448); 0 for amax = 0."""
+    amax <= 2688 * 2^e (2688 = 6 * 448), and at least -126; 0 for amax = 0."""
     amax = float(amax)
     if amax == 0.0:
         return 0
+    if amax <= E2M1_MAX * E4M3_MAX * 2.0 ** -127:
+        return -126
     e = int(np.ceil(np.log2(amax / (E2M1_MAX * E4M3_MAX))))
     # guard the log2 rounding on either side of a power of two
     while amax > E2M1_MAX * E4M3_MAX * 2.0 ** e:
