@@ -544,7 +544,8 @@ def measure_extra(ft, synth, dev, flush, peaks, steps, warmup):
 
 
 def measure_variants(ft, synth, dev, flush, steps, warmup):
-    """FLUX-width layer (M = 4608, K = N = 3072, ranks 32/32) under the precision
+    """FLUX-width layer (M = 4608, K = N = 3072, ranks 32/32) under the 1x16
+    group-wise layout (the granularity ablation), the precision
     variants of the paper's ablation (W4A16G4, W4A4G16, W4A16G16), the standard
     bf16 LoRA layer (bf16 weight, rank-32 adapter, no stabilizer) on this
     library's bf16 tensor-core path and through cuBLAS (torch.matmul), and the
@@ -620,9 +621,18 @@ def measure_variants(ft, synth, dev, flush, steps, warmup):
         dBu = Lu[:, r_sl].t() @ dY
         return Yu, dXu, dAu, dBu
 
+    # the 1x16 group-wise layout (§4.3, Table 5's comparator): Q16(R) and Q16(R^T)
+    lay1 = ft.Linear1x16.from_weights(W, up(p["S_dn"]), up(p["S_up"]), A, B)
+    wsf1, wsb1 = lay1.fwd_workspace(M), lay1.bwd_workspace(M)
+
+    def w4a4g4_1x16():
+        ft.linear_fwd_1x16(lay1, X, ws=wsf1, Y=Y, L=L)
+        ft.linear_bwd_1x16(lay1, dY, X, L, ws=wsb1, dX=dX, dA=dA, dB=dB)
+
     fp4, lr = layer_work(M, K, N, r_s, r)
     out = {"workload": WORKLOAD, "steps": steps, "flop_per_step": fp4 + lr, "variants": {}}
-    for name, fn in (("W4A16G4", w4a16g4), ("W4A4G16", w4a4g16), ("W4A16G16", w4a16g16),
+    for name, fn in (("W4A4G4 1x16 groups + per-tensor scale", w4a4g4_1x16),
+                     ("W4A16G4", w4a16g4), ("W4A4G16", w4a4g16), ("W4A16G16", w4a16g16),
                      ("bf16-LoRA ours (bf16 tensor cores)", lora_bf16_ours),
                      ("bf16-LoRA cuBLAS (torch.matmul)", lora_bf16_cublas),
                      ("W4A4G4 unfused (quantizer + 4-bit GEMM + cuBLAS low-rank)", unfused_w4)):

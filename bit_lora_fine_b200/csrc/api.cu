@@ -385,7 +385,7 @@ int side_stream(SideStream** out) {
 // Fused row pass over X [M, K] bf16: Q(X) -> (codes, scales), L = bf16(X W)
 // with W = D [K, R] (w_mn) or W^T [R, K].
 int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, bool w_mn, uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* L, float* part, int* counters,
-                int* status, int num_sms, cudaStream_t s, bool no_quant = false) {
+                int* status, int num_sms, cudaStream_t s, bool no_quant = false, const uint32_t* amax16 = nullptr) {
   CUtensorMap tmX, tmW;
   if (!map_bf16(&tmX, X, K, M, 128)) return FT_ERR_CUDA;
   if (w_mn ? !map_bf16(&tmW, W, R, K, 64) : !map_bf16(&tmW, W, K, R, static_cast<uint32_t>(R))) return FT_ERR_CUDA;
@@ -407,6 +407,8 @@ int run_rowpass(const void* X, int64_t M, int64_t K, const void* W, int64_t R, b
   rp.status = status;
   rp.fault_skip_stage = -1;
   rp.no_quant = no_quant ? 1 : 0;
+  rp.group16 = amax16 ? 1 : 0;   // 1x16 groups below the per-tensor scale of *amax16
+  rp.amax = amax16;
   return cuda_err(ft::launch_rowpass(tmX, tmW, rp, s));
 }
 
@@ -427,6 +429,8 @@ struct GemmArgs {
   void* out;
   bool out_bf16;
   bool main_bf16;               // 16-bit main product: a_codes = A [M, K], b_codes = B [N, K] bf16
+  const uint32_t* amax_a;       // 1x16 groups: the operands' maxima (the product's 2^(eA + eB)), else null
+  const uint32_t* amax_b;
 };
 int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   const uint32_t b_rows = static_cast<uint32_t>(ft::kGemmBN);
@@ -457,6 +461,8 @@ int run_gemm(const GemmArgs& a, int* status, int num_sms, cudaStream_t s) {
   gp.out_bf16 = a.out_bf16 ? 1 : 0;
   gp.status = status;
   gp.main_bf16 = a.main_bf16 ? 1 : 0;
+  gp.amax_a = a.amax_a;
+  gp.amax_b = a.amax_b;
   return cuda_err(ft::launch_gemm_fp4(tmA, tmB, tmA2, tmB2, gp, num_sms, s));
 }
 
@@ -860,6 +866,273 @@ int fourtune_linear_bwd_timed(const ft_linear_t* layer, const ft_bf16* dY, const
   } else {
     st = gemm_and_grads_side(g, layer, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status,
                              di.num_sms, s);
+    if (st) return st;
+  }
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------- 1x16 groups
+namespace {
+int check_layer_1x16(const ft_linear_1x16_t* L) {
+  if (!L || !L->R_codes || !L->R_sf || !L->Rt_codes || !L->Rt_sf || !L->R_amax || !L->D || !L->U)
+    return FT_ERR_INVALID_ARG;
+  if (L->K <= 0 || L->N <= 0 || L->K % 32 || L->N % 32) return FT_ERR_SHAPE;
+  if (L->r_s < 0 || L->r < 16 || L->r_s % 16 || L->r % 16 || L->r > 64 || L->r_s + L->r > 128)
+    return FT_ERR_UNSUPPORTED;
+  if (L->K > (1 << 30) || L->N > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(L->R_codes) || !al16(L->R_sf) || !al16(L->Rt_codes) || !al16(L->Rt_sf) || !al16(L->D) ||
+      !al16(L->U) || (L->bias && !al16(L->bias)) || (reinterpret_cast<uintptr_t>(L->R_amax) & 3u))
+    return FT_ERR_ALIGN;
+  return FT_OK;
+}
+// the shapes and low-rank factors, for the helpers shared with the block layout
+ft_linear_t view_1x16(const ft_linear_1x16_t* L) {
+  ft_linear_t v{};
+  v.K = L->K;
+  v.N = L->N;
+  v.r_s = L->r_s;
+  v.r = L->r;
+  v.D = L->D;
+  v.U = L->U;
+  v.bias = L->bias;
+  return v;
+}
+// 1x16 activations of a [M, C] matrix: codes, compact scales [M, C/16], MMA-ready scales
+struct Q1x16 {
+  size_t codes, scales, sf;
+  void carve(Carver& c, int64_t M, int64_t C) {
+    codes = c.take(static_cast<size_t>(M * C / 2));
+    scales = c.take(static_cast<size_t>(M * (C / 16)));
+    sf = c.take(ft::sf_mma_bytes(M, C));
+  }
+};
+// header: status (byte 0), the tensor's maximum word (byte 8), split counters from 16
+constexpr size_t kAmaxWord = 8;
+// forward: header | Q16(X) | row-pass partials | U rescaled
+struct Fwd1x16Ws {
+  size_t header, rp_cnt, rp_part, Us, total;
+  Q1x16 qx;
+};
+Fwd1x16Ws fwd_1x16_layout(const ft_linear_t* L, int64_t M, int num_sms) {
+  Fwd1x16Ws w{};
+  Carver c;
+  w.rp_cnt = 16;
+  c.take(w.header = up256(16 + 4 * static_cast<size_t>(cdiv(M, 128))));
+  w.qx.carve(c, M, L->K);
+  w.rp_part = c.take(rp_part_bytes(M, L->K, rank_all(L), 1, num_sms));
+  w.Us = c.take(static_cast<size_t>(rank_all(L) * L->N * 2));
+  w.total = c.o;
+  return w;
+}
+// backward: header (status, maximum, dA/dB and row-pass counters) | Q16(G) | P |
+// dA/dB partials | row-pass partials | D rescaled
+struct Bwd1x16Ws {
+  size_t header, P, rp_cnt, rp_part, Ds, total;
+  Q1x16 qg;
+  GradPair g;
+};
+Bwd1x16Ws bwd_1x16_layout(const ft_linear_t* L, int64_t M, int num_sms) {
+  Bwd1x16Ws w{};
+  plan_grads(w.g, L, M, num_sms);
+  Carver c;
+  w.g.cntA = 16;
+  w.g.cntB = w.g.cntA + 4 * static_cast<size_t>(cdiv(L->K, 128));
+  w.rp_cnt = 16 + 4 * grad_counter_words(L);
+  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
+  w.qg.carve(c, M, L->N);
+  w.P = c.take(static_cast<size_t>(M * rank_all(L) * 2));
+  w.g.partA = c.take(grad_partial_bytes(w.g, L));
+  w.g.partB = w.g.partA + grad_part_a(w.g, L);
+  w.rp_part = c.take(rp_part_bytes(M, L->N, rank_all(L), 0, num_sms));
+  w.Ds = c.take(static_cast<size_t>(L->K * rank_all(L) * 2));
+  w.total = c.o;
+  return w;
+}
+}  // namespace
+
+int fourtune_quantize_1x16(const ft_bf16* W, int64_t rows, int64_t cols, int transposed, uint32_t* amax_word,
+                           uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* stream) {
+  FT_RANGE("fourtune_quantize_1x16");
+  if (!W || !amax_word || !codes || !scales || (transposed != 0 && transposed != 1)) return FT_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows % 32 || cols % 32) return FT_ERR_SHAPE;
+  if (rows > (1 << 30) || cols > (1 << 30) || rows * cols > (1LL << 40)) return FT_ERR_UNSUPPORTED;
+  if (!al16(W) || !al16(codes) || !al16(amax_word) || (sf_mma && !al16(sf_mma))) return FT_ERR_ALIGN;
+  DevInfo di;
+  int st = device_info(&di);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t orows = transposed ? cols : rows, ocols = transposed ? rows : cols;
+  // the maximum word (16 bytes cleared) and the MMA-ready padding start at zero
+  if (ft::launch_clear_words(amax_word, 16, s) != cudaSuccess) return FT_ERR_CUDA;
+  if (sf_mma && ft::launch_clear_words(sf_mma, ft::sf_mma_bytes(orows, ocols), s) != cudaSuccess) return FT_ERR_CUDA;
+  if (ft::launch_tensor_amax(W, rows * cols, amax_word, di.num_sms, s) != cudaSuccess) return FT_ERR_CUDA;
+  return cuda_err(ft::launch_quantize_group16(W, static_cast<int>(rows), static_cast<int>(cols), transposed, amax_word,
+                                             codes, scales, sf_mma, s));
+}
+
+size_t fourtune_linear_fwd_1x16_workspace_size(const ft_linear_1x16_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_fwd_1x16_workspace_size");
+  if (check_layer_1x16(layer) || M <= 0 || M % 16) return 0;
+  const ft_linear_t v = view_1x16(layer);
+  return fwd_1x16_layout(&v, M, num_sms_or_default()).total;
+}
+
+size_t fourtune_linear_bwd_1x16_workspace_size(const ft_linear_1x16_t* layer, int64_t M) {
+  FT_RANGE("fourtune_linear_bwd_1x16_workspace_size");
+  if (check_layer_1x16(layer) || M <= 0 || M % 16) return 0;
+  const ft_linear_t v = view_1x16(layer);
+  return bwd_1x16_layout(&v, M, num_sms_or_default()).total;
+}
+
+int fourtune_linear_1x16_ws_offsets(const ft_linear_1x16_t* layer, int64_t M, int backward, size_t* codes_off,
+                                    size_t* scales_off, size_t* amax_off, size_t* P_off) {
+  FT_RANGE("fourtune_linear_1x16_ws_offsets");
+  int st = check_layer_1x16(layer);
+  if (st) return st;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  const ft_linear_t v = view_1x16(layer);
+  if (backward) {
+    const Bwd1x16Ws w = bwd_1x16_layout(&v, M, num_sms_or_default());
+    if (codes_off) *codes_off = w.qg.codes;
+    if (scales_off) *scales_off = w.qg.scales;
+    if (P_off) *P_off = w.P;
+  } else {
+    const Fwd1x16Ws w = fwd_1x16_layout(&v, M, num_sms_or_default());
+    if (codes_off) *codes_off = w.qx.codes;
+    if (scales_off) *scales_off = w.qx.scales;
+    if (P_off) *P_off = 0;
+  }
+  if (amax_off) *amax_off = kAmaxWord;
+  return FT_OK;
+}
+
+int fourtune_linear_fwd_1x16(const ft_linear_1x16_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
+                             ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_fwd_1x16");
+  return fourtune_linear_fwd_1x16_timed(layer, X, M, Y, y_dtype, L_saved, ws, ws_bytes, stream, nullptr, 0);
+}
+
+int fourtune_linear_fwd_1x16_timed(const ft_linear_1x16_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
+                                   ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream, void* const* events,
+                                   int n_events) {
+  FT_RANGE("fourtune_linear_fwd_1x16_timed");
+  const Events evs{events, n_events};
+  int st = check_layer_1x16(layer);
+  if (st) return st;
+  if (!X || !Y || !L_saved || !ws) return FT_ERR_INVALID_ARG;
+  if (y_dtype != FT_DTYPE_F32 && y_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(X) || !al16(Y) || !al16(L_saved) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const ft_linear_t v = view_1x16(layer);
+  const Fwd1x16Ws w = fwd_1x16_layout(&v, M, di.num_sms);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(base + kAmaxWord);
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K = layer->K, N = layer->N, R = rank_all(&v);
+  uint8_t* qc = base + w.qx.codes;
+  uint8_t* qf = base + w.qx.sf;
+  void* Us = base + w.Us;
+  FT_TRY(0, cuda_err(ft::launch_tensor_amax(X, M * K, amax, di.num_sms, s)));
+  // X pass: Q16(X) (below 2^e of max|X|) and L = bf16(X D)
+  FT_TRY(1, run_rowpass(X, M, K, layer->D, R, true, qc, base + w.qx.scales, qf, L_saved,
+                        reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                        di.num_sms, s, false, amax));
+  // U rescaled by 2^-(eX + eR): it shares the accumulator the epilogue scales by 2^(eX + eR)
+  FT_TRY(2, cuda_err(ft::launch_scale_pow2(layer->U, Us, R * N, amax, layer->R_amax, di.num_sms, s)));
+  GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.R2 = R;
+  g.a_codes = qc;
+  g.a_sf = qf;
+  g.b_codes = layer->R_codes;
+  g.b_sf = layer->R_sf;
+  g.transposed = false;
+  g.A2 = L_saved;
+  g.B2 = Us;
+  g.bias = layer->bias;
+  g.out = Y;
+  g.out_bf16 = y_dtype == FT_DTYPE_BF16;
+  g.amax_a = amax;
+  g.amax_b = layer->R_amax;
+  FT_TRY(3, run_gemm(g, status, di.num_sms, s));
+  return FT_OK;
+}
+
+int fourtune_linear_bwd_1x16(const ft_linear_1x16_t* layer, const ft_bf16* dY, const ft_bf16* X,
+                             const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA, float* dB,
+                             int accumulate, void* ws, size_t ws_bytes, void* stream) {
+  FT_RANGE("fourtune_linear_bwd_1x16");
+  return fourtune_linear_bwd_1x16_timed(layer, dY, X, L_saved, M, dX, dx_dtype, dA, dB, accumulate, ws, ws_bytes,
+                                        stream, nullptr, 0);
+}
+
+int fourtune_linear_bwd_1x16_timed(const ft_linear_1x16_t* layer, const ft_bf16* dY, const ft_bf16* X,
+                                   const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA, float* dB,
+                                   int accumulate, void* ws, size_t ws_bytes, void* stream, void* const* events,
+                                   int n_events) {
+  FT_RANGE("fourtune_linear_bwd_1x16_timed");
+  const Events evs{events, n_events};
+  int st = check_layer_1x16(layer);
+  if (st) return st;
+  if (!dY || !X || !L_saved || !dX || !dA || !dB || !ws) return FT_ERR_INVALID_ARG;
+  if (dx_dtype != FT_DTYPE_F32 && dx_dtype != FT_DTYPE_BF16) return FT_ERR_INVALID_ARG;
+  if (M <= 0 || M % 16) return FT_ERR_SHAPE;
+  if (M > (1 << 30)) return FT_ERR_UNSUPPORTED;
+  if (!al16(dY) || !al16(X) || !al16(L_saved) || !al16(dX) || !al16(dA) || !al16(dB) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return FT_ERR_ALIGN;
+  DevInfo di;
+  if ((st = device_info(&di))) return st;
+  const ft_linear_t v = view_1x16(layer);
+  const Bwd1x16Ws w = bwd_1x16_layout(&v, M, di.num_sms);
+  if (ws_bytes < w.total) return FT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(base + kAmaxWord);
+  if (ft::launch_clear_words(base, w.header, s) != cudaSuccess) return FT_ERR_CUDA;
+  const int64_t K = layer->K, N = layer->N, R = rank_all(&v);
+  uint8_t* gc = base + w.qg.codes;
+  uint8_t* gf = base + w.qg.sf;
+  void* P = base + w.P;
+  void* Ds = base + w.Ds;
+  FT_TRY(0, cuda_err(ft::launch_tensor_amax(dY, M * N, amax, di.num_sms, s)));
+  // G pass: Q16(G) and P = bf16(G U^T), U [R, N] read K-major
+  FT_TRY(1, run_rowpass(dY, M, N, layer->U, R, false, gc, base + w.qg.scales, gf, P,
+                        reinterpret_cast<float*>(base + w.rp_part), reinterpret_cast<int*>(base + w.rp_cnt), status,
+                        di.num_sms, s, false, amax));
+  FT_TRY(2, cuda_err(ft::launch_scale_pow2(layer->D, Ds, K * R, amax, layer->R_amax, di.num_sms, s)));
+  // dX = deq(Q16(G)) deq(Q16(R^T))^T + P D^T: B is Q16(R^T) [K, N], B2 = D rescaled
+  GemmArgs g{};
+  g.M = M;
+  g.N = K;
+  g.K = N;
+  g.R2 = R;
+  g.a_codes = gc;
+  g.a_sf = gf;
+  g.b_codes = layer->Rt_codes;
+  g.b_sf = layer->Rt_sf;
+  g.transposed = true;
+  g.A2 = P;
+  g.B2 = Ds;
+  g.out = dX;
+  g.out_bf16 = dx_dtype == FT_DTYPE_BF16;
+  g.amax_a = amax;
+  g.amax_b = layer->R_amax;
+  if (evs.ev || w.g.side_sms == 0) {
+    FT_TRY(3, run_grads(&v, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, false, base, status, s));
+    FT_TRY(4, run_gemm(g, status, di.num_sms, s));
+  } else {
+    st = gemm_and_grads_side(g, &v, M, X, P, dY, L_saved, dA, dB, accumulate != 0, w.g, base, status, di.num_sms,
+                             s);
     if (st) return st;
   }
   return FT_OK;

@@ -497,6 +497,27 @@ __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg)
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
+// ------------------------------------------------------------------ 1x16 groups
+// Per-tensor scale of the 1x16 group-wise layout (the granularity comparator of
+// FourTune §4.3, Table 5): 2^e with e the least integer such that
+// amax <= 2688 * 2^e (2688 = 6 * 448: the E2M1 times the E4M3 maximum), at
+// least -126; 0 for amax = 0.  amax is a non-negative finite float.  With
+// amax = m 2^E (1 <= m < 2) and 2688 = 1.3125 * 2^11: e = E - 11, plus one when
+// m > 1.3125 (m's fraction bits above 0x280000).
+__device__ __forceinline__ int group16_exponent(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  uint32_t b = __float_as_uint(amax);
+  int E = static_cast<int>(b >> 23) - 127;
+  if ((b >> 23) == 0) {                      // subnormal: normalize (exact)
+    b = __float_as_uint(amax * 16777216.0f);
+    E = static_cast<int>(b >> 23) - 127 - 24;
+  }
+  const int e = E - 11 + ((b & 0x7FFFFFu) > 0x280000u ? 1 : 0);
+  return e < -126 ? -126 : e;
+}
+// 2^k for -126 <= k <= 127
+__device__ __forceinline__ float pow2_f32(int k) { return __uint_as_float(static_cast<uint32_t>(k + 127) << 23); }
+
 // Maximum of a non-negative float over the 16 lanes of the warp whose lane bit 0
 // equals this lane's (two half-warp groups, reduced at once).  Non-negative
 // IEEE floats order like their bit patterns, so one integer max reduction does it.

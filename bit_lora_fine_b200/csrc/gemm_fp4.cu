@@ -325,6 +325,19 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const long long ldb = p.ldo * (p.out_bf16 ? 2 : 4);   // output row stride in bytes
     const bool fast = p.out_bf16 != 0;
+    // 1x16 groups: the product's per-tensor scale 2^(eA + eB), as one factor
+    // when it is a float32 number, else as two (then f1 is exact and the
+    // product's own range is exceeded anyway)
+    float f1 = 1.0f, f2 = 1.0f;
+    if (p.amax_a) {
+      const int es = group16_exponent(__uint_as_float(*p.amax_a)) + group16_exponent(__uint_as_float(*p.amax_b));
+      if (es >= -126 && es <= 127) {
+        f1 = pow2_f32(es);
+      } else {
+        f1 = pow2_f32(es / 2);
+        f2 = pow2_f32(es - es / 2);
+      }
+    }
     int j = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++j) {
       if (!mbar_wait(acc_full, j & 1, p.status, abortp)) break;
@@ -358,8 +371,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             for (int e = 0; e < 8; ++e) {
               const uint4 b4 = bw[2 * k + e / 4];
               const uint32_t bb = (e & 3) == 0 ? b4.x : (e & 3) == 1 ? b4.y : (e & 3) == 2 ? b4.z : b4.w;
-              pk[16 * rd + 8 * k + e] = pack_bf16x2(__uint_as_float(v[k][2 * e]) + bf16_bits_to_f32(bb & 0xFFFFu),
-                                                    __uint_as_float(v[k][2 * e + 1]) + bf16_bits_to_f32(bb >> 16));
+              pk[16 * rd + 8 * k + e] =
+                  pack_bf16x2(fmaf(__uint_as_float(v[k][2 * e]) * f1, f2, bf16_bits_to_f32(bb & 0xFFFFu)),
+                              fmaf(__uint_as_float(v[k][2 * e + 1]) * f1, f2, bf16_bits_to_f32(bb >> 16)));
             }
           }
         }
@@ -391,7 +405,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             uint32_t w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              w[e] = __float_as_uint(__uint_as_float(v[8 * hlf + e]) + (bias ? __bfloat162float(bias[nb + e]) : 0.0f));
+              w[e] = __float_as_uint(fmaf(__uint_as_float(v[8 * hlf + e]) * f1, f2,
+                                          bias ? __bfloat162float(bias[nb + e]) : 0.0f));
             store_rows32(buf, w, lane, out_rows + static_cast<long long>(nb) * 4, ldb, rows_left);
           }
         }

@@ -16,6 +16,11 @@ struct RowpassParams {
   int kt_per_split, nsplit;              // 64-column tiles per CTA along K, number of K splits
   int stages;                            // TMA ring depth, 2..rowpass_stages()
   int no_quant;                          // only L: no codes or scales (the 16-bit precision variants)
+  // 1x16 groups (group16.cu): each row's 16 columns get their own scale, the
+  // values scaled by 2^-e of the tensor maximum in *amax (float bits); scales
+  // [M, K/16].  0: 16x16 blocks, scales [M/16, K/16].
+  int group16;
+  const uint32_t* amax;
   uint8_t* codes;                        // [M, K/2]
   uint8_t* scales;                       // [M/16, K/16]
   uint8_t* sf_mma;                       // the same scales in the MMA-ready layout (null = not written)
@@ -57,6 +62,12 @@ struct GemmParams {
   // 16-bit main product (the precision variants): A [M, K] and B [N, K] are
   // bf16 (K contiguous) instead of block16 codes; sfa, sfb unused
   int main_bf16;
+  // 1x16 groups: the accumulator is scaled by 2^(eA + eB), the per-tensor
+  // exponents of the maxima in *amax_a, *amax_b (float bits), before the bias
+  // (null: no scaling).  The low-rank factor B2 must come pre-scaled by the
+  // inverse (launch_scale_pow2).
+  const uint32_t* amax_a;
+  const uint32_t* amax_b;
 };
 
 // The MLP's 4-bit GEMMs with their fused epilogues (FourTune §3.3 "MLP
@@ -128,6 +139,16 @@ cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
 // zero `bytes` (a multiple of 16, 16-aligned) at p after the previous kernel, in a
 // dependent launch (see quant.cu)
 cudaError_t launch_clear_words(void* p, size_t bytes, cudaStream_t stream);
+// 1x16 groups (group16.cu): max|x| of a bf16 tensor (n a multiple of 8) into
+// *word (atomicMax of float bits: the word must start at 0); the group
+// quantizer of W [rows, cols] (transposed: of W^T) with codes [orows, ocols/2],
+// scales [orows, ocols/16] and the MMA-ready copy (null: not written; rows and
+// groups past the matrix are left as they are); dst = src * 2^-(eA + eB)
+cudaError_t launch_tensor_amax(const void* x, long long n, uint32_t* word, int num_sms, cudaStream_t stream);
+cudaError_t launch_quantize_group16(const void* w, int rows, int cols, int transposed, const uint32_t* amax_word,
+                                    uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, cudaStream_t stream);
+cudaError_t launch_scale_pow2(const void* src, void* dst, long long n, const uint32_t* amax_a, const uint32_t* amax_b,
+                              int num_sms, cudaStream_t stream);
 cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
                           cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,

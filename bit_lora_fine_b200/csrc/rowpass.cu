@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kRpThreads, 1)
     const long long half_k = p.K / 2;
     const int kblocks = p.K / 16;
     const bool block_row_ok = m0 + blk * 16 < p.M;
+    // 1x16 groups: this lane's 16 values are one group; the tensor's 2^-e
+    const bool g16 = p.group16 != 0;
+    const float g16_inv = g16 ? pow2_f32(-group16_exponent(__uint_as_float(*p.amax))) : 1.0f;
     bool ok = true;
     int s = 0;
     uint32_t ph = 0;
@@ -195,7 +198,12 @@ __global__ void __launch_bounds__(kRpThreads, 1)
       for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
         for (int e = 0; e < w; ++e) m[e] = fmaxf(m[e], m[e + w]);
-      const float amax = max16_same_parity(m[0], lane);   // over the block's 16 rows
+      float amax = max16_same_parity(m[0], lane);   // over the block's 16 rows
+      if (g16) {                                    // the lane's own group, scaled (exact: 2^-e)
+        amax = m[0] * g16_inv;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] *= g16_inv;
+      }
       const int cstart = (kt0 + i) * 64 + colw;
       const bool inside = block_row_ok && cstart < p.K;
       if (!p.no_quant && (inside || p.sf_mma)) {
@@ -205,7 +213,9 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         if (inside) {
           *reinterpret_cast<uint2*>(p.codes + static_cast<long long>(m0 + r) * half_k + cstart / 2) =
               make_uint2(packed[0], packed[1]);
-          if ((lane >> 1) == 0)
+          if (g16)
+            p.scales[static_cast<long long>(m0 + r) * kblocks + cstart / 16] = static_cast<uint8_t>(sc);
+          else if ((lane >> 1) == 0)
             p.scales[(m0 / 16 + blk) * static_cast<long long>(kblocks) + cstart / 16] = static_cast<uint8_t>(sc);
         }
         if (p.sf_mma) {

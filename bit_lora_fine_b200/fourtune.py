@@ -30,14 +30,20 @@ EXPORTED = ("fourtune_quantize_block16", "fourtune_transpose_codes", "fourtune_l
             "fourtune_mlp_fwd_timed", "fourtune_mlp_bwd_timed", "fourtune_quantize_block16_f32",
             "fourtune_quant_down_static_status", "fourtune_test_wait_timeout", "fourtune_dequantize_block16",
             "fourtune_linear_fwd_a16", "fourtune_linear_bwd_g16", "fourtune_linear_fwd_a16_workspace_size",
-            "fourtune_linear_bwd_g16_workspace_size", "fourtune_stabilizer_residual", "fourtune_gemm_block16")
+            "fourtune_linear_bwd_g16_workspace_size", "fourtune_stabilizer_residual", "fourtune_gemm_block16",
+            "fourtune_quantize_1x16", "fourtune_linear_fwd_1x16_workspace_size",
+            "fourtune_linear_bwd_1x16_workspace_size", "fourtune_linear_fwd_1x16", "fourtune_linear_bwd_1x16",
+            "fourtune_linear_fwd_1x16_timed", "fourtune_linear_bwd_1x16_timed", "fourtune_linear_1x16_ws_offsets")
 SIZE_FUNCS = ("fourtune_linear_fwd_workspace_size", "fourtune_linear_bwd_workspace_size", "fourtune_mma_scales_size",
               "fourtune_mlp_fwd_workspace_size", "fourtune_mlp_bwd_workspace_size",
-              "fourtune_linear_fwd_a16_workspace_size", "fourtune_linear_bwd_g16_workspace_size")
+              "fourtune_linear_fwd_a16_workspace_size", "fourtune_linear_bwd_g16_workspace_size",
+              "fourtune_linear_fwd_1x16_workspace_size", "fourtune_linear_bwd_1x16_workspace_size")
 
 # kernels each call launches, in order (the *_timed entry points bracket each with events)
 FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
 BWD_KERNELS = ("gpass_quant_down", "tgrad_dA_dB", "gemm_fp4_dx")
+FWD_1X16_KERNELS = ("amax_x", "xpass_quant_down_1x16", "scale_u", "gemm_fp4_fwd_1x16")
+BWD_1X16_KERNELS = ("amax_g", "gpass_quant_down_1x16", "scale_d", "tgrad_dA_dB", "gemm_fp4_dx_1x16")
 MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1_gelu_quant_proj", "gemm_fp4_fc2")
 MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_fc2_gelu_bwd_quant_proj", "tgrad_fc2", "tgrad_fc1",
                    "gemm_fp4_dx_fc1")
@@ -54,6 +60,13 @@ class ft_linear_t(ctypes.Structure):
                 ("R_codes", ctypes.c_void_p), ("R_scales", ctypes.c_void_p), ("R_codes_t", ctypes.c_void_p),
                 ("D", ctypes.c_void_p), ("U", ctypes.c_void_p), ("bias", ctypes.c_void_p),
                 ("R_sf", ctypes.c_void_p), ("R_sf_t", ctypes.c_void_p)]
+
+
+class ft_linear_1x16_t(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int64), ("N", ctypes.c_int64), ("r_s", ctypes.c_int64), ("r", ctypes.c_int64),
+                ("R_codes", ctypes.c_void_p), ("R_sf", ctypes.c_void_p), ("Rt_codes", ctypes.c_void_p),
+                ("Rt_sf", ctypes.c_void_p), ("R_amax", ctypes.c_void_p), ("D", ctypes.c_void_p),
+                ("U", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
 
 
 _lib = None
@@ -112,6 +125,15 @@ def load():
                                           vp, sz, vp]
     L.fourtune_linear_fwd_a16_workspace_size.argtypes = [P(ft_linear_t), i64]
     L.fourtune_linear_bwd_g16_workspace_size.argtypes = [P(ft_linear_t), i64]
+    P16 = P(ft_linear_1x16_t)
+    L.fourtune_quantize_1x16.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp]
+    L.fourtune_linear_fwd_1x16_workspace_size.argtypes = [P16, i64]
+    L.fourtune_linear_bwd_1x16_workspace_size.argtypes = [P16, i64]
+    L.fourtune_linear_fwd_1x16.argtypes = [P16, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
+    L.fourtune_linear_bwd_1x16.argtypes = [P16, vp, vp, vp, i64, vp, ctypes.c_int, vp, vp, ctypes.c_int, vp, sz, vp]
+    L.fourtune_linear_fwd_1x16_timed.argtypes = list(L.fourtune_linear_fwd_1x16.argtypes) + [P(vp), ctypes.c_int]
+    L.fourtune_linear_bwd_1x16_timed.argtypes = list(L.fourtune_linear_bwd_1x16.argtypes) + [P(vp), ctypes.c_int]
+    L.fourtune_linear_1x16_ws_offsets.argtypes = [P16, i64, ctypes.c_int, P(sz), P(sz), P(sz), P(sz)]
     for f in SIZE_FUNCS:
         getattr(L, f).restype = sz
     for f in EXPORTED:
@@ -634,3 +656,127 @@ def fault_wait_timeout(X, W, ws, wait_ns=5_000_000):
 def device_status(ws):
     """Synchronize and raise FourtuneError(FT_ERR_TIMEOUT) if a kernel wait expired."""
     _check(load().fourtune_device_status(_ptr(ws), _stream()), "fourtune_device_status")
+
+
+# ------------------------------------------------------- 1x16 group-wise variant
+def quantize_1x16(W, transposed=False):
+    """Q16(W) (or Q16(W^T)) of a bf16 W [rows, cols]: 1x16 groups along the
+    output's rows below the per-tensor scale of max|W|.  Returns (codes
+    [orows, ocols/2], scales [orows, ocols/16], sf (MMA-ready), amax word
+    (int32 [4]: element 0 holds max|W|'s float32 bits))."""
+    _need(W, torch.bfloat16, "W")
+    _ndim2(W, "W")
+    rows, cols = W.shape
+    orows, ocols = (cols, rows) if transposed else (rows, cols)
+    codes = torch.empty((orows, ocols // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((orows, ocols // 16), dtype=torch.uint8, device=W.device)
+    sf = torch.empty(load().fourtune_mma_scales_size(orows, ocols), dtype=torch.uint8, device=W.device)
+    amax = torch.empty(4, dtype=torch.int32, device=W.device)
+    _check(load().fourtune_quantize_1x16(_ptr(W), rows, cols, int(transposed), _ptr(amax), _ptr(codes), _ptr(scales),
+                                          _ptr(sf), _stream()), "fourtune_quantize_1x16")
+    return codes, scales, sf, amax
+
+
+class Linear1x16:
+    """Device tensors of the 1x16 layer: Q16(R) and Q16(R^T) (codes, MMA-ready
+    scales) with the maximum word of R, D = [S_dn | A], U = [S_up ; B] and bias."""
+
+    def __init__(self, R, D, U, r_s, bias=None):
+        _need(R, torch.bfloat16, "R")
+        for t, n in ((D, "D"), (U, "U"), (bias, "bias")):
+            _need(t, torch.bfloat16, n)
+        self.N, self.K = R.shape
+        self.r_s = r_s
+        self.r = D.shape[1] - r_s
+        R_codes, R_scales, R_sf, R_amax = quantize_1x16(R)
+        Rt_codes, Rt_scales, Rt_sf, _ = quantize_1x16(R, transposed=True)
+        self.t = dict(R_codes=R_codes, R_scales=R_scales, R_sf=R_sf, Rt_codes=Rt_codes, Rt_scales=Rt_scales,
+                      Rt_sf=Rt_sf, R_amax=R_amax, D=D, U=U, bias=bias)
+        self.c = ft_linear_1x16_t(self.K, self.N, self.r_s, self.r, *[
+            _ptr(self.t[k]) for k in ("R_codes", "R_sf", "Rt_codes", "Rt_sf", "R_amax", "D", "U", "bias")])
+
+    @classmethod
+    def from_weights(cls, R, S_dn, S_up, A, B, bias=None):
+        D = torch.cat([S_dn, A], dim=1).contiguous()
+        U = torch.cat([S_up, B], dim=0).contiguous()
+        return cls(R, D, U, S_dn.shape[1], bias)
+
+    @property
+    def R_all(self):
+        return self.r_s + self.r
+
+    def _ws(self, fn, M):
+        n = getattr(load(), fn)(ctypes.byref(self.c), M)
+        if n == 0:
+            raise FourtuneError(-2, fn)
+        return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def fwd_workspace(self, M):
+        return self._ws("fourtune_linear_fwd_1x16_workspace_size", M)
+
+    def bwd_workspace(self, M):
+        return self._ws("fourtune_linear_bwd_1x16_workspace_size", M)
+
+    def ws_offsets(self, M, backward):
+        """(codes, scales, maximum word, P) offsets in the forward (backward=False:
+        P is 0) or backward workspace."""
+        c, s, a, p = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load().fourtune_linear_1x16_ws_offsets(ctypes.byref(self.c), M, int(backward), ctypes.byref(c),
+                                                      ctypes.byref(s), ctypes.byref(a), ctypes.byref(p)),
+               "fourtune_linear_1x16_ws_offsets")
+        return c.value, s.value, a.value, p.value
+
+
+def linear_fwd_1x16(layer, X, y_dtype=torch.float32, ws=None, Y=None, L=None, events=None):
+    """The 1x16 forward: Y = deq(Q16(X)) deq(Q16(R))^T + L [S_up ; B] + bias.  Returns (Y, L, ws).
+    `events`: optional 2*len(FWD_1X16_KERNELS) torch.cuda.Events."""
+    _ndim2(X, "X")
+    M = X.shape[0]
+    _shape(X, (M, layer.K), "X")
+    _shape(Y, (M, layer.N), "Y")
+    _shape(L, (M, layer.R_all), "L")
+    _same_device(("X", X), ("Y", Y), ("L", L), ("ws", ws))
+    _out_dtype(Y, "Y")
+    _need(X, torch.bfloat16, "X")
+    Y = torch.empty((M, layer.N), dtype=y_dtype, device=X.device) if Y is None else Y
+    L = torch.empty((M, layer.R_all), dtype=torch.bfloat16, device=X.device) if L is None else L
+    ws = layer.fwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if Y.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(layer.c), _ptr(X), M, _ptr(Y), code, _ptr(L), _ptr(ws), ws.numel(), _stream())
+    if events is None:
+        _check(load().fourtune_linear_fwd_1x16(*args), "fourtune_linear_fwd_1x16")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_linear_fwd_1x16_timed(*args, arr, n), "fourtune_linear_fwd_1x16_timed")
+    return Y, L, ws
+
+
+def linear_bwd_1x16(layer, dY, X, L, dx_dtype=torch.float32, dA=None, dB=None, accumulate=False, ws=None, dX=None,
+                    events=None):
+    """The 1x16 backward: dX = deq(Q16(dY)) deq(Q16(R^T))^T + P [S_dn | A]^T, dA, dB as linear_bwd.
+    Returns (dX, dA, dB, ws)."""
+    _ndim2(dY, "dY")
+    M = dY.shape[0]
+    _shape(dY, (M, layer.N), "dY")
+    _shape(X, (M, layer.K), "X")
+    _shape(L, (M, layer.R_all), "L")
+    _shape(dX, (M, layer.K), "dX")
+    _shape(dA, (layer.K, layer.r), "dA")
+    _shape(dB, (layer.r, layer.N), "dB")
+    _same_device(("dY", dY), ("X", X), ("L", L), ("dX", dX), ("dA", dA), ("dB", dB), ("ws", ws))
+    _out_dtype(dX, "dX")
+    for t, n in ((dY, "dY"), (X, "X"), (L, "L")):
+        _need(t, torch.bfloat16, n)
+    dX = torch.empty((M, layer.K), dtype=dx_dtype, device=dY.device) if dX is None else dX
+    dA = torch.zeros((layer.K, layer.r), dtype=torch.float32, device=dY.device) if dA is None else dA
+    dB = torch.zeros((layer.r, layer.N), dtype=torch.float32, device=dY.device) if dB is None else dB
+    ws = layer.bwd_workspace(M) if ws is None else ws
+    code = FT_DTYPE_F32 if dX.dtype == torch.float32 else FT_DTYPE_BF16
+    args = (ctypes.byref(layer.c), _ptr(dY), _ptr(X), _ptr(L), M, _ptr(dX), code, _ptr(dA), _ptr(dB),
+            int(accumulate), _ptr(ws), ws.numel(), _stream())
+    if events is None:
+        _check(load().fourtune_linear_bwd_1x16(*args), "fourtune_linear_bwd_1x16")
+    else:
+        arr, n = _events(events)
+        _check(load().fourtune_linear_bwd_1x16_timed(*args, arr, n), "fourtune_linear_bwd_1x16_timed")
+    return dX, dA, dB, ws

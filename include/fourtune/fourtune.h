@@ -231,6 +231,70 @@ FT_API int fourtune_linear_bwd_g16(const ft_linear_t* layer, const ft_bf16* W16_
                                    const ft_bf16* X, const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype,
                                    float* dA, float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream);
 
+/* The 1x16 group-wise layer (the quantization-granularity comparator of §4.3,
+ * Table 5, in NVFP4's full form of §2.3): the same triple-branch layer with
+ * X, G and the frozen weight quantized in 1x16 groups -- 16 consecutive
+ * elements of a row along each GEMM's reduction dimension share one E4M3
+ * scale -- below a per-tensor scale 2^e, e the least integer with
+ * max|T| <= 6 * 448 * 2^e (at least -126; 0 for an all-zero tensor).  A group
+ * of T' = T * 2^-e follows the block rules on one row: s = max|t'| / 6 in
+ * fp32, scale = E4M3(s), codes = E2M1(t' / scale).  The forward GEMM reads
+ * Q16(R) [N, K] (groups along K); the backward's dX reads Q16(R^T) [K, N]
+ * (groups along N) -- a transposed operand cannot reuse 1x16 groups, which is
+ * the cost the 16x16 blocks avoid (§3.2).  The product of two tensors carries
+ * 2^(eA + eB), applied to the accumulator before the bias; the low-rank factor
+ * sharing that accumulator (U forward, D for dX) is pre-scaled by the inverse
+ * into the workspace, an exact power-of-two step.
+ *
+ * fourtune_quantize_1x16: W [rows, cols] bf16 -> Q16(W) (transposed = 0,
+ *   output [rows, cols]) or Q16(W^T) (transposed = 1, output [cols, rows]):
+ *   codes [orows, ocols/2], scales [orows, ocols/16] and, when sf_mma is not
+ *   NULL, the MMA-ready copy (fourtune_mma_scales_size(orows, ocols) bytes,
+ *   fully written).  amax_word: 16 bytes of device memory, 16-byte aligned,
+ *   cleared by the call; its first word receives the float32 bits of max|W|,
+ *   the per-tensor scale's source, which the layer reads.  rows % 32 == 0 and
+ *   cols % 32 == 0; W, codes 16-byte aligned.  Offline for the frozen weight;
+ *   also the standalone parity probe of the group quantizer.
+ * ft_linear_1x16_t: Q16(R) and Q16(R^T) (codes and MMA-ready scales, both
+ *   from one fourtune_quantize_1x16 call each on the bf16 R), R_amax the word
+ *   those calls wrote, and the low-rank factors and bias as in ft_linear_t.
+ * fourtune_linear_fwd_1x16 / _bwd_1x16: fourtune_linear_fwd / _bwd with the
+ *   1x16 layout (one more pass each: the maximum of X or G).  The _timed
+ *   kernels, in order -- forward: 0 max|X|, 1 X pass, 2 U rescale, 3 FP4 GEMM;
+ *   backward: 0 max|G|, 1 G pass, 2 D rescale, 3 dA and dB, 4 FP4 dX GEMM.
+ *   fourtune_linear_1x16_ws_offsets gives the workspace offsets of Q16(X)
+ *   (backward = 0) or Q16(G) (backward = 1): codes [M, C/2], scales [M, C/16],
+ *   the tensor's maximum word and (backward) P [M, r_s + r] bf16. */
+typedef struct {
+  int64_t K, N, r_s, r;
+  const uint8_t* R_codes;     /* Q16(R)   [N, K/2] */
+  const uint8_t* R_sf;        /* its MMA-ready scales (rows N, cols K) */
+  const uint8_t* Rt_codes;    /* Q16(R^T) [K, N/2] */
+  const uint8_t* Rt_sf;       /* its MMA-ready scales (rows K, cols N) */
+  const uint32_t* R_amax;     /* device word: float32 bits of max|R| */
+  const ft_bf16* D;
+  const ft_bf16* U;
+  const ft_bf16* bias;
+} ft_linear_1x16_t;
+FT_API int fourtune_quantize_1x16(const ft_bf16* W, int64_t rows, int64_t cols, int transposed, uint32_t* amax_word,
+                                  uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, void* stream);
+FT_API size_t fourtune_linear_fwd_1x16_workspace_size(const ft_linear_1x16_t* layer, int64_t M);
+FT_API size_t fourtune_linear_bwd_1x16_workspace_size(const ft_linear_1x16_t* layer, int64_t M);
+FT_API int fourtune_linear_fwd_1x16(const ft_linear_1x16_t* layer, const ft_bf16* X, int64_t M, void* Y, int y_dtype,
+                                    ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream);
+FT_API int fourtune_linear_bwd_1x16(const ft_linear_1x16_t* layer, const ft_bf16* dY, const ft_bf16* X,
+                                    const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA, float* dB,
+                                    int accumulate, void* ws, size_t ws_bytes, void* stream);
+FT_API int fourtune_linear_fwd_1x16_timed(const ft_linear_1x16_t* layer, const ft_bf16* X, int64_t M, void* Y,
+                                          int y_dtype, ft_bf16* L_saved, void* ws, size_t ws_bytes, void* stream,
+                                          void* const* events, int n_events);
+FT_API int fourtune_linear_bwd_1x16_timed(const ft_linear_1x16_t* layer, const ft_bf16* dY, const ft_bf16* X,
+                                          const ft_bf16* L_saved, int64_t M, void* dX, int dx_dtype, float* dA,
+                                          float* dB, int accumulate, void* ws, size_t ws_bytes, void* stream,
+                                          void* const* events, int n_events);
+FT_API int fourtune_linear_1x16_ws_offsets(const ft_linear_1x16_t* layer, int64_t M, int backward, size_t* codes_off,
+                                           size_t* scales_off, size_t* amax_off, size_t* P_off);
+
 /* The MLP pair (§3.3 "MLP Fusion"): y = FC2(GELU_tanh(FC1(X))), both layers
  * triple-branch, fc1 [K1 -> H], fc2 [H -> N2] (fc1->N == fc2->K).
  * Forward: the X pass, then FC1's 4-bit GEMM (+ L1 U1 + b1) whose epilogue
