@@ -255,8 +255,8 @@ BwdWs bwd_layout(const ft_linear_t* L, int64_t M, int num_sms) {
 }
 
 // Units of the MLP's fused GEMMs (gemm_mlp.cu): a 128-row tile's N tiles split
-// into nsplit runs of `per`; the smallest split whose makespan (tile rounds of
-// the busiest CTA) is within 3 % of the even share of all tiles.
+// into nsplit runs of `per` (each unit writes one fp32 partial of the
+// projection, summed by launch_proj_reduce).
 struct MlpUnits {
   int nsplit, per;
 };
@@ -282,18 +282,17 @@ size_t proj_part_bytes(int64_t M, int64_t N, int64_t RP, int num_sms) {
   return static_cast<size_t>(plan_units(M, N, num_sms).nsplit) * static_cast<size_t>(M) * static_cast<size_t>(RP) * 4;
 }
 
-// MLP forward: header (status, row-pass counters, projection counters) | Q(X) |
+// MLP forward: header (status, row-pass counters) | Q(X) |
 // Q(a) | row-pass partials | FC1 projection partials (L2)
 struct MlpFwdWs {
-  size_t header, rp_cnt, pj_cnt, rp_part, pj_part, total;
+  size_t header, rp_cnt, rp_part, pj_part, total;
   Q16 qx, qa;
 };
 MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M, int num_sms) {
   MlpFwdWs w{};
   Carver c;
   w.rp_cnt = 16;
-  w.pj_cnt = w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128));
-  c.take(w.header = up256(w.pj_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
+  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qx.carve(c, M, fc1->K);
   w.qa.carve(c, M, fc1->N);
   w.rp_part = c.take(rp_part_bytes(M, fc1->K, rank_all(fc1), 1, num_sms));
@@ -303,11 +302,11 @@ MlpFwdWs mlp_fwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
 }
 
 // MLP backward: header (status, counters of both layers' dA/dB, row-pass
-// counters, projection counters) | Q(G) | P2 | d_h | Q(d_h) | P1 | dA/dB
+// counters) | Q(G) | P2 | d_h | Q(d_h) | P1 | dA/dB
 // partials (shared by the two dA/dB launches) | row-pass partials | FC2-dX
 // projection partials (P1)
 struct MlpBwdWs {
-  size_t header, P2, dh, P1, rp_cnt, pj_cnt, rp_part, pj_part, total;
+  size_t header, P2, dh, P1, rp_cnt, rp_part, pj_part, total;
   Q16 qg, qdh;
   GradPair g2, g1;
 };
@@ -322,8 +321,7 @@ MlpBwdWs mlp_bwd_layout(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t 
   w.g1.cntA = w.g2.cntB + 4 * static_cast<size_t>(cdiv(fc2->N, 128));
   w.g1.cntB = w.g1.cntA + 4 * static_cast<size_t>(cdiv(fc1->K, 128));
   w.rp_cnt = 16 + 4 * (grad_counter_words(fc2) + grad_counter_words(fc1));
-  w.pj_cnt = w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128));
-  c.take(w.header = up256(w.pj_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
+  c.take(w.header = up256(w.rp_cnt + 4 * static_cast<size_t>(cdiv(M, 128))));
   w.qg.carve(c, M, fc2->N);
   w.P2 = c.take(static_cast<size_t>(M * rank_all(fc2) * 2));
   w.dh = c.take(static_cast<size_t>(M * H * 2));
@@ -517,7 +515,6 @@ struct MlpGemmArgs {
   int64_t RP;
   void* proj_out;
   float* part;
-  int* counters;
 };
 int run_gemm_mlp(const MlpGemmArgs& m, int* status, int num_sms, cudaStream_t s) {
   const GemmArgs& a = m.g;
@@ -554,9 +551,13 @@ int run_gemm_mlp(const MlpGemmArgs& m, int* status, int num_sms, cudaStream_t s)
   mp.nsplit = un.nsplit;
   mp.per = un.per;
   mp.part = m.part;
-  mp.counters = m.counters;
-  mp.proj_out = m.proj_out;
   return cuda_err(ft::launch_gemm_mlp(tmA, tmB, tmA2, tmB2, tmW, mp, num_sms, s));
+}
+// the split-order sum of the fused GEMM's fp32 projection partials -> bf16 proj_out
+int run_proj_reduce(const MlpGemmArgs& m, int num_sms, cudaStream_t s) {
+  const MlpUnits un = plan_units(m.g.M, m.g.N, num_sms);
+  return cuda_err(ft::launch_proj_reduce(m.part, un.nsplit, static_cast<int>(m.g.M), static_cast<int>(m.RP),
+                                         m.proj_out, num_sms, s));
 }
 
 #define FT_TRY(k, expr)                                          \
@@ -630,7 +631,7 @@ int read_status_word(const void* dev_word, cudaStream_t s) {
   int h = 0;
   if (cudaMemcpyAsync(&h, dev_word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FT_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return FT_ERR_CUDA;
-  return h == 0 ? FT_OK : FT_ERR_TIMEOUT;
+  return h == 0 ? FT_OK : h == 2 ? FT_ERR_UNSUPPORTED : FT_ERR_TIMEOUT;
 }
 }  // namespace
 
@@ -1411,8 +1412,8 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   m.RP = R2;
   m.proj_out = L2_saved;
   m.part = reinterpret_cast<float*>(base + w.pj_part);
-  m.counters = reinterpret_cast<int*>(base + w.pj_cnt);
   FT_TRY(1, run_gemm_mlp(m, status, di.num_sms, s));
+  FT_TRY(2, run_proj_reduce(m, di.num_sms, s));
   // FC2: 4-bit GEMM + L2 U2 + b2 -> Y
   GemmArgs g2{};
   g2.M = M;
@@ -1428,7 +1429,7 @@ int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g2.bias = fc2->bias;
   g2.out = Y;
   g2.out_bf16 = y_dtype == FT_DTYPE_BF16;
-  FT_TRY(2, run_gemm(g2, status, di.num_sms, s));
+  FT_TRY(3, run_gemm(g2, status, di.num_sms, s));
   return FT_OK;
 }
 
@@ -1497,10 +1498,10 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   m.RP = R1;
   m.proj_out = P1;
   m.part = reinterpret_cast<float*>(base + w.pj_part);
-  m.counters = reinterpret_cast<int*>(base + w.pj_cnt);
   FT_TRY(1, run_gemm_mlp(m, status, di.num_sms, s));
+  FT_TRY(2, run_proj_reduce(m, di.num_sms, s));
   // FC2 adapter gradients: dA2 on bf16(GELU(h)) (recomputed from h), dB2 on G
-  FT_TRY(2, run_grads(fc2, M, h_saved, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, false, base, status, s,
+  FT_TRY(3, run_grads(fc2, M, h_saved, P2, dY, L2_saved, dA2, dB2, accumulate != 0, w.g2, false, base, status, s,
                       true));
   // FC1 dX GEMM and adapter gradients (on d_h)
   GemmArgs g1{};
@@ -1518,8 +1519,8 @@ int fourtune_mlp_bwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const
   g1.out = dX;
   g1.out_bf16 = dx_dtype == FT_DTYPE_BF16;
   if (evs.ev || w.g1.side_sms == 0) {
-    FT_TRY(3, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
-    FT_TRY(4, run_gemm(g1, status, di.num_sms, s));
+    FT_TRY(4, run_grads(fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, false, base, status, s));
+    FT_TRY(5, run_gemm(g1, status, di.num_sms, s));
   } else {
     st = gemm_and_grads_side(g1, fc1, M, X, P1, dh, L1_saved, dA1, dB1, accumulate != 0, w.g1, base, status,
                              di.num_sms, s);

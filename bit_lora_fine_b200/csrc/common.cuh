@@ -15,6 +15,7 @@ namespace ft {
 
 // status word values written by kernels (0 = ok)
 constexpr int kDevTimeout = 1;
+constexpr int kDevUnsupported = 2;   // a launch found its shared memory misaligned
 // a wait that has not completed after this many nanoseconds gives up
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

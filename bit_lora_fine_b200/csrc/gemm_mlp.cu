@@ -12,7 +12,8 @@
 //
 // The main loop is the single-CTA FP4 GEMM's (gemm_fp4.cu): 128 x 256 output
 // tiles, TMA code boxes per 256-wide K-block, scale warps writing the block
-// scales into TMEM, the low-rank blocks accumulated by bf16 MMAs.  What is new
+// scales into TMEM (from shared memory here: each K-block's scale blocks come
+// into its stage by bulk copies), the low-rank blocks accumulated by bf16 MMAs.  What is new
 // is the epilogue's low-rank projection T Wp (T = bf16(a) or d_h) -- a
 // reduction over the N columns of the GEMM, i.e. across output tiles:
 //   * a CTA walks units: N tiles [sp*per, +per) of one 128-row tile, so that
@@ -23,13 +24,17 @@
 //     cores -- issued after the next tile's main loop, so that the epilogue of
 //     one tile overlaps the MMAs of the next;
 //   * at the end of a unit its fp32 partial [128, RP] goes to global memory;
-//     the last unit of a 128-row tile (a counter) sums the partials in split
-//     order (deterministic) and rounds once to bf16.
-// Shared memory: three 48 KB stages, the 64 KB T buffer (which also stages h /
-// d_h for whole-row stores) and 1 KB of code scratch per epilogue warp (code
-// rows leave in 32-byte pieces, not 8).  TMEM: the 256-column accumulator, two
-// 48-column scale slots (a stage uses slot g % 2, rewritten once the MMAs of
-// stage g - 2 are done) and the projection accumulator.
+//     launch_proj_reduce then sums the partials in split order
+//     (deterministic) and rounds once to bf16, over all row tiles at once (a
+//     last-unit sum inside this kernel fell on a few CTAs: in rounds of
+//     lockstep units the same CTA finishes last for many row tiles).
+// Shared memory: three 54 KB stages (codes or bf16 tiles, and the K-block's
+// MMA-ready scale blocks: the scale warps read them from there, so that large
+// K keeps three stages of scales in flight without registers) and the 64 KB T
+// buffer (which also stages h / d_h for whole-row stores).  TMEM: the
+// 256-column accumulator, two 48-column scale slots (a stage uses slot g % 2,
+// rewritten once the MMAs of stage g - 2 are done) and the projection
+// accumulator.
 //
 // Warp roles: warp 0 lane 0 producer; warp 1 TMEM owner, lane 0 issues the
 // MMAs; warps 2..17 epilogue (warp w: TMEM lanes 32 (w % 4).., columns
@@ -57,16 +62,20 @@ static_assert(((kMlThreads / 32 + 3) / 4) * 32 * kMlMaxReg <= 16384, "registers 
 constexpr int kMlBN = 256;
 constexpr uint32_t kMlA = 128 * 128;                  // A codes / A2 bf16 tile
 constexpr uint32_t kMlB = kMlBN * 128;                // B codes / B2 bf16 tile / projection weight
-constexpr uint32_t kMlStage = kMlA + kMlB;            // 48 KB
+constexpr uint32_t kMlSfA = 4 * 512;                  // A's scale blocks of a K-block (4 k-steps)
+constexpr uint32_t kMlSfB = 2 * 4 * 512;              // B's: [128-row chunk][k-step][512 B]
+constexpr uint32_t kMlStage = kMlA + kMlB + kMlSfA + kMlSfB;   // 54 KB
 constexpr uint32_t kMlT = 4 * 128 * 128;              // T: four [128 x 64] bf16 chunks
-constexpr uint32_t kMlCodes = kMlEpiWarps * 1024;     // per epilogue warp: its 32 rows x 32 bytes of Q(T) codes
 constexpr uint32_t kMlTail = 512;
-constexpr uint32_t kMlSmem = 1024 + kMlStages * kMlStage + kMlT + kMlCodes + kMlTail;
+// no alignment slack: the dynamic shared memory starts 1024-byte aligned (the
+// kernel checks it and refuses to run otherwise)
+constexpr uint32_t kMlSmem = kMlStages * kMlStage + kMlT + kMlTail;
 constexpr int kMlSfSlots = 2;
 constexpr uint32_t kMlSfCols = 16 + 32;               // A's 4 k-steps x 4, B's 4 k-steps x 2 chunks x 4
 constexpr uint32_t kMlProjCol = kMlBN + kMlSfSlots * kMlSfCols;
 constexpr int kMlProjStages = 2;                      // Wp's 256 rows: two stages of two 64-row chunks
 static_assert(kMlSmem <= 232448, "shared memory budget");
+static_assert(kMlStage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
 static_assert(kMlProjCol + 128 <= 512, "TMEM budget");
 
 __device__ __forceinline__ uint32_t ml_pack_bf16x2(float lo, float hi) {
@@ -88,11 +97,14 @@ __global__ void __maxnreg__(kMlMaxReg)
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const __grid_constant__ CUtensorMap tmW, const MlpGemmParams mp) {
   const GemmParams& p = mp.g;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {   // uniform: every thread leaves before any barrier or TMEM use
+    if (threadIdx.x == 0 && blockIdx.x == 0 && mp.g.status) atomicCAS(mp.g.status, 0, kDevUnsupported);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* tbuf = smem + kMlStages * kMlStage;
-  uint8_t* cbuf = tbuf + kMlT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + kMlCodes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(tbuf + kMlT);
   uint64_t* empty = full + kMlStages;
   uint64_t* sf_full = empty + kMlStages;        // [kMlSfSlots] scale warps -> MMA
   uint64_t* sf_empty = sf_full + kMlSfSlots;    // [kMlSfSlots] MMAs that read the slot are done
@@ -103,7 +115,6 @@ __global__ void __maxnreg__(kMlMaxReg)
   uint64_t* mma_done = t_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* s_last = abort_flag + 1;
   volatile int* abortp = abort_flag;
   static_assert((2 * kMlStages + 2 * kMlSfSlots + 5) * 8 + 16 <= kMlTail, "barriers and flags fit the tail");
 
@@ -197,9 +208,18 @@ __global__ void __maxnreg__(kMlMaxReg)
           for (int i = 0; i < TM && ok; ++i) {
             ok = stage([&](uint8_t* st, uint64_t* bar) {
               if (i < KB) {
-                mbar_arrive_expect_tx(bar, kMlA + kMlB);
+                // codes by TMA, the K-block's MMA-ready scale blocks by bulk copies
+                // (nks 512-byte blocks each for A and for B's 128-row chunks)
+                const int nks = min(4, KS - 4 * i);
+                const uint32_t sfbytes = static_cast<uint32_t>(nks) * 512u;
+                const int nb = (n0 / 128 + 1 < nchunk_b) ? 2 : 1;
+                mbar_arrive_expect_tx(bar, kMlA + kMlB + sfbytes * static_cast<uint32_t>(1 + nb));
                 tma_load_2d(st, &tmA, bar, i * 128, m0);
                 tma_load_2d(st + kMlA, &tmB, bar, i * 128, n0);
+                bulk_load(st + kMlA + kMlB, p.sfa + (static_cast<size_t>(m0 / 128) * KS + 4 * i) * 512, sfbytes, bar);
+                for (int c = 0; c < nb; ++c)
+                  bulk_load(st + kMlA + kMlB + kMlSfA + c * 2048,
+                            p.sfb + (static_cast<size_t>(n0 / 128 + c) * KS + 4 * i) * 512, sfbytes, bar);
               } else {
                 const int e = i - KB;
                 mbar_arrive_expect_tx(bar, kMlA + kMlB);
@@ -322,30 +342,32 @@ __global__ void __maxnreg__(kMlMaxReg)
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
     int g = 0;
     bool ok = true;
-    auto fetch = [&](int mt, int nt, int i, uint32_t (&a)[4], uint32_t (&b)[32]) {
+    // stage g's scale blocks, from the stage once its copies have landed
+    auto fetch = [&](int nt, int i, uint32_t (&a)[4], uint32_t (&b)[32]) -> bool {
+      const int s = g % kMlStages;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(&full[s], (g / kMlStages) & 1, p.status, abortp);
+      if (__shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) == 0) return false;
+      const uint8_t* sf = smem + s * kMlStage + kMlA + kMlB;
       const int nks = min(4, KS - 4 * i);
       const int nc = nt * 2;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        a[t] = 0u;
-        if (t < nks)
-          a[t] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa + (static_cast<size_t>(mt) * KS + 4 * i + t) * 512 +
-                                                         16 * lane + 4 * q));
-      }
+      for (int t = 0; t < 4; ++t)
+        a[t] = t < nks ? *reinterpret_cast<const uint32_t*>(sf + t * 512 + 16 * lane + 4 * q) : 0u;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           uint4 x = make_uint4(0u, 0u, 0u, 0u);   // zero scales past N (their codes are zero)
           if (t < nks && nc + c < nchunk_b)
-            x = __ldg(reinterpret_cast<const uint4*>(p.sfb + (static_cast<size_t>(nc + c) * KS + 4 * i + t) * 512 +
-                                                     16 * lane));
+            x = *reinterpret_cast<const uint4*>(sf + kMlSfA + c * 2048 + t * 512 + 16 * lane);
           b[4 * (2 * t + c)] = x.x;
           b[4 * (2 * t + c) + 1] = x.y;
           b[4 * (2 * t + c) + 2] = x.z;
           b[4 * (2 * t + c) + 3] = x.w;
         }
       }
+      return true;
     };
     // pass ring stage g: wait for its scale slot, write the scales (if any), hand it to the MMA
     auto put = [&](bool has, const uint32_t (&a)[4], const uint32_t (&b)[32]) -> bool {
@@ -370,18 +392,12 @@ __global__ void __maxnreg__(kMlMaxReg)
     };
     bool have_prev = false;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      const int mt = u / mp.nsplit, sp = u % mp.nsplit;
+      const int sp = u % mp.nsplit;
       const int nhi = min(tiles_n, (sp + 1) * mp.per);
       for (int nt = sp * mp.per; nt < nhi && ok; ++nt) {
-        // the tile's FP4 stages: stage i + 1's words are loaded as soon as stage
-        // i's are in TMEM (one stage in registers: 80 registers leave no room
-        // for two without spilling)
+        // the tile's FP4 stages: each stage's scale blocks arrive with its codes
         uint32_t a0[4], b0[32];
-        if (KB > 0) fetch(mt, nt, 0, a0, b0);
-        for (int i = 0; i < KB && ok; ++i) {
-          ok = put(true, a0, b0);
-          if (ok && i + 1 < KB) fetch(mt, nt, i + 1, a0, b0);
-        }
+        for (int i = 0; i < KB && ok; ++i) ok = fetch(nt, i, a0, b0) && put(true, a0, b0);
         for (int i = 0; i < EB && ok; ++i) ok = put(false, a0, b0);
         for (int i = 0; have_prev && i < kMlProjStages && ok; ++i) ok = put(false, a0, b0);
         have_prev = true;
@@ -395,7 +411,6 @@ __global__ void __maxnreg__(kMlMaxReg)
     // ---- epilogue: 16 warps; warp w owns rows 32 q.. (q = w % 4: the TMEM lane
     // quadrant a warp may access) of the tile and columns c_lo .. c_lo + 63.  The
     // sixteen warps leave together (named_bar_or).
-    const int et = static_cast<int>(threadIdx.x) - 32 * kMlEpi0;   // 0 .. 511
     const int q = warp & 3;
     const int cq = (warp - kMlEpi0) >> 2;
     const int c_lo = 64 * cq;
@@ -409,8 +424,8 @@ __global__ void __maxnreg__(kMlMaxReg)
     int prev_m0 = 0, prev_sp = 0;
     bool have_prev = false, prev_last = false;
 
-    // The unit's projection accumulator -> fp32 partial; the last unit of the
-    // 128-row tile sums all partials in split order and rounds to bf16.
+    // The unit's projection accumulator -> its fp32 partial (the split-order
+    // sum of all units' partials is launch_proj_reduce's)
     auto finish_unit = [&](int m0, int sp) {
       const int row = m0 + r_loc;
       for (int c = 0; c < quarter; c += 16) {
@@ -426,58 +441,11 @@ __global__ void __maxnreg__(kMlMaxReg)
                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
       }
-      // one thread publishes this unit's partial (ordered before it by the
-      // barrier) with a gpu-scope fence before its counter increment; the last
-      // unit's fence after the increment orders its reads after all others
-      named_bar_sync(1, kMlEpiThreads);
-      if (et == 0) {
-        __threadfence();
-        const int prev = atomicAdd(&mp.counters[m0 / 128], 1);
-        __threadfence();
-        *s_last = (prev == mp.nsplit - 1);
-      }
-      named_bar_sync(1, kMlEpiThreads);
-      if (*s_last) {
-        const int c4 = RP / 4;
-        for (int idx = et; idx < 128 * c4; idx += kMlEpiThreads) {
-          const int rr = m0 + idx / c4, cc = 4 * (idx % c4);
-          if (rr >= p.M) continue;
-          // split order, four loads in flight at a time
-          const float4* src = reinterpret_cast<const float4*>(mp.part + static_cast<long long>(rr) * RP + cc);
-          const long long stride4 = static_cast<long long>(p.M) * RP / 4;
-          float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          int s2 = 0;
-          for (; s2 + 4 <= mp.nsplit; s2 += 4) {
-            float4 x[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) x[k] = __ldcg(src + (s2 + k) * stride4);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              acc.x += x[k].x;
-              acc.y += x[k].y;
-              acc.z += x[k].z;
-              acc.w += x[k].w;
-            }
-          }
-          for (; s2 < mp.nsplit; ++s2) {
-            const float4 x = __ldcg(src + s2 * stride4);
-            acc.x += x.x;
-            acc.y += x.y;
-            acc.z += x.z;
-            acc.w += x.w;
-          }
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(mp.proj_out) + static_cast<long long>(rr) * RP + cc) =
-              make_uint2(ml_pack_bf16x2(acc.x, acc.y), ml_pack_bf16x2(acc.z, acc.w));
-        }
-        if (et == 0) mp.counters[m0 / 128] = 0;
-      }
     };
 
     // this lane's row of T: chunk cq (the warp's 64 columns), 128-byte swizzled
     uint8_t* const t_row = tbuf + cq * 16384 + r_loc * 128;
     const int sw = r_loc & 7;
-    uint8_t* const cbase = cbuf + (warp - kMlEpi0) * 1024;   // the warp's code scratch
-    uint8_t* const c_row = cbase + lane * 32;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int m0 = (u / mp.nsplit) * 128, sp = u % mp.nsplit;
@@ -577,7 +545,6 @@ __global__ void __maxnreg__(kMlMaxReg)
         // place) the block's Q(T) codes and scale, T being the shared bf16 input
         // of the next layer's branches (bf16(a) or d_h)
         uint32_t sfw = 0u;
-        __syncwarp();   // the previous tile's reads of the code scratch are done
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           const int col = n0 + 16 * c;
@@ -613,23 +580,12 @@ __global__ void __maxnreg__(kMlMaxReg)
           quantize_block_row<16>(v, amax, packed, &sc);      // bf16 values: the exact division-free path
           if (!inside) sc = 0u;
           sfw |= sc << (8 * c);
-          // codes into the warp's scratch: row `lane`, 8-byte unit c at
-          // position c ^ ((lane >> 2) & 3) (16 lanes cover the 32 banks)
-          *reinterpret_cast<uint2*>(c_row + 8 * (c ^ ((lane >> 2) & 3))) = make_uint2(packed[0], packed[1]);
-          if (inside && (lane & 15) == 0)
-            mp.q_scales[static_cast<long long>(row / 16) * (p.N / 16) + col / 16] = static_cast<uint8_t>(sc);
-        }
-        __syncwarp();
-        // the codes of the warp's 32 rows x 64 columns: 32 bytes a row, two
-        // rows per lane pair, 16 bytes (32 columns) per lane
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int lr = 16 * i + (lane >> 1), hf = lane & 1, x = (lr >> 2) & 3;
-          uint4 v4 = *reinterpret_cast<const uint4*>(cbase + lr * 32 + 16 * (hf ^ (x >> 1)));
-          if (x & 1) v4 = make_uint4(v4.z, v4.w, v4.x, v4.y);   // the pair's two units stored swapped
-          const int rr = m0 + 32 * q + lr;
-          if (rr < p.M && n0 + 32 * hf < p.N)
-            *reinterpret_cast<uint4*>(mp.q_codes + static_cast<long long>(rr) * (p.N / 2) + n0 / 2 + 16 * hf) = v4;
+          if (inside) {
+            *reinterpret_cast<uint2*>(mp.q_codes + static_cast<long long>(row) * (p.N / 2) + col / 2) =
+                make_uint2(packed[0], packed[1]);
+            if ((lane & 15) == 0)
+              mp.q_scales[static_cast<long long>(row / 16) * (p.N / 16) + col / 16] = static_cast<uint8_t>(sc);
+          }
         }
         // the MMA-ready copy of the scales: the warp's k-step, four scales of
         // this row in one word (rows past M and groups past N hold 0)
@@ -661,6 +617,37 @@ __global__ void __maxnreg__(kMlMaxReg)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+namespace {
+// out [M, RP] = bf16(sum over s in split order of part[s, M, RP]), one float4 a thread
+__global__ void __launch_bounds__(256) proj_reduce_kernel(const float4* __restrict__ part, int nsplit, long long n4,
+                                                          uint2* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 acc = __ldcs(part + i);
+    for (int sp = 1; sp < nsplit; ++sp) {
+      const float4 x = __ldcs(part + sp * n4 + i);
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    out[i] = make_uint2(ml_pack_bf16x2(acc.x, acc.y), ml_pack_bf16x2(acc.z, acc.w));
+  }
+}
+}  // namespace
+
+cudaError_t launch_proj_reduce(const float* part, int nsplit, int M, int RP, void* out, int num_sms,
+                               cudaStream_t stream) {
+  if (nsplit < 1 || M < 1 || RP % 4) return cudaErrorInvalidValue;
+  const long long n4 = static_cast<long long>(M) * RP / 4;
+  const long long want = (n4 + 255) / 256;
+  const int grid = static_cast<int>(want < 4LL * num_sms ? want : 4LL * num_sms);
+  return launch_pdl(proj_reduce_kernel, dim3(grid), dim3(256), 0, stream, reinterpret_cast<const float4*>(part),
+                    nsplit, n4, static_cast<uint2*>(out));
 }
 
 cudaError_t launch_gemm_mlp(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,

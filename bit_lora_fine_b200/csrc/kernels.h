@@ -78,9 +78,10 @@ struct GemmParams {
 //            (-> dbg if set);  Q(a) -> q_*;  T = bf16(a)
 //   epi == 2 (FC2 dX):       d_h = bf16(acc * GELU'(h)) -> out_h;  Q(d_h) -> q_*;
 //            T = d_h
-// and projects it: proj_out [M, RP] = bf16(T Wp), Wp [N, RP] read from D2
-// [N, RP] (wp_mn_major = 1) or from U1 [RP, N] (0), summed over the N tiles of
-// a unit in TMEM and over units through fp32 partials.
+// and projects it: part [nsplit, M, RP] = T Wp over each unit's N tiles (fp32,
+// accumulated in TMEM), Wp [N, RP] read from D2 [N, RP] (wp_mn_major = 1) or
+// from U1 [RP, N] (0); launch_proj_reduce then forms bf16(sum of the partials
+// in split order).
 struct MlpGemmParams {
   GemmParams g;                          // main product (M, N, K, R2, scales, bias, status)
   int epi;                               // 1 or 2 (above)
@@ -94,12 +95,13 @@ struct MlpGemmParams {
   int wp_mn_major;
   int nsplit, per;                       // units: N tiles [sp*per, +per) of one 128-row tile
   float* part;                           // fp32 [nsplit, M, RP]
-  int* counters;                         // [ceil(M/128)], zero on entry, left zero
-  void* proj_out;                        // bf16 [M, RP]
 };
 cudaError_t launch_gemm_mlp(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const CUtensorMap& tmW, const MlpGemmParams& p, int num_sms,
                             cudaStream_t stream);
+// out [M, RP] bf16 = sum over s = 0 .. nsplit - 1 (in that order) of part [s, M, RP] (fp32)
+cudaError_t launch_proj_reduce(const float* part, int nsplit, int M, int RP, void* out, int num_sms,
+                               cudaStream_t stream);
 
 // out[p, j] (+)= sum_m T[m, p] * V[m, v0 + j]   for p < P, j < r (r <= 64)
 struct TgradParams {

@@ -44,8 +44,9 @@ FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fwd")
 BWD_KERNELS = ("gpass_quant_down", "tgrad_dA_dB", "gemm_fp4_dx")
 FWD_1X16_KERNELS = ("amax_x", "xpass_quant_down_1x16", "scale_u", "gemm_fp4_fwd_1x16")
 BWD_1X16_KERNELS = ("amax_g", "gpass_quant_down_1x16", "scale_d", "tgrad_dA_dB", "gemm_fp4_dx_1x16")
-MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1_gelu_quant_proj", "gemm_fp4_fc2")
-MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_fc2_gelu_bwd_quant_proj", "tgrad_fc2", "tgrad_fc1",
+MLP_FWD_KERNELS = ("xpass_quant_down", "gemm_fp4_fc1_gelu_quant_proj", "proj_reduce_l2", "gemm_fp4_fc2")
+MLP_BWD_KERNELS = ("gpass_quant_down_fc2", "gemm_fp4_dx_fc2_gelu_bwd_quant_proj", "proj_reduce_p1", "tgrad_fc2",
+                   "tgrad_fc1",
                    "gemm_fp4_dx_fc1")
 
 

@@ -24,7 +24,9 @@
  *     shared by calls that may run concurrently.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
  *     the legacy default stream).  A kernel whose internal wait times out
- *     records it in the workspace; fourtune_device_status() reports it.
+ *     records it in the workspace; fourtune_device_status() reports it
+ *     (FT_ERR_TIMEOUT; FT_ERR_UNSUPPORTED if the MLP's fused GEMM found its
+ *     dynamic shared memory not 1024-byte aligned and did nothing).
  *   - bf16 tensors are arrays of IEEE bfloat16 bit patterns (ft_bf16), row-major,
  *     16-byte aligned.  Dimensions must be multiples of 16; K and N must also be
  *     multiples of 32 (4-bit rows are copied in 16-byte units).
@@ -298,12 +300,14 @@ FT_API int fourtune_linear_1x16_ws_offsets(const ft_linear_1x16_t* layer, int64_
 /* The MLP pair (§3.3 "MLP Fusion"): y = FC2(GELU_tanh(FC1(X))), both layers
  * triple-branch, fc1 [K1 -> H], fc2 [H -> N2] (fc1->N == fc2->K).
  * Forward: the X pass, then FC1's 4-bit GEMM (+ L1 U1 + b1) whose epilogue
- * forms h = bf16(FC1(X)) (saved), a = GELU_tanh(h) in fp32, Q(a) (block16 of
- * the fp32 values, FC2's 4-bit input) and L2 = bf16(bf16(a) D2) (FC2's
- * low-rank input) -- the hidden activation a is never stored -- then FC2's
- * 4-bit GEMM (+ L2 U2 + b2).  Writes Y [M, N2], h_saved [M, H], L1_saved
+ * forms h = bf16(FC1(X)) (saved), a = GELU_tanh(h) in fp32 and FC2's input
+ * bf16(a), shared by FC2's three branches: Q(bf16(a)) (FC2's 4-bit input) and
+ * the fp32 partials of bf16(a) D2 per run of N tiles (a small reduction sums
+ * them in split order into L2 = bf16(bf16(a) D2), FC2's low-rank input) --
+ * the hidden activation is never stored -- then FC2's 4-bit GEMM
+ * (+ L2 U2 + b2).  Writes Y [M, N2], h_saved [M, H], L1_saved
  * [M, r_s1 + r1], L2_saved [M, r_s2 + r2]; dbg_a, when not NULL, receives the
- * fp32 a [M, H] that was quantized (for inspection). */
+ * fp32 a [M, H] (for inspection). */
 FT_API size_t fourtune_mlp_fwd_workspace_size(const ft_linear_t* fc1, const ft_linear_t* fc2, int64_t M);
 FT_API int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M, void* Y,
                             int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved, float* dbg_a,
@@ -311,7 +315,8 @@ FT_API int fourtune_mlp_fwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
 
 /* MLP backward.  FC2's G pass, then FC2's dX GEMM whose epilogue forms
  * d_h = bf16(d_a GELU'(h)) -- FC1's incoming gradient, taken by all three of
- * its branches -- with Q(d_h) (FC1's 4-bit gradient) and P1 = bf16(d_h U1^T).
+ * its branches -- with Q(d_h) (FC1's 4-bit gradient) and the partials of
+ * d_h U1^T (summed by the reduction into P1 = bf16(d_h U1^T)).
  * FC2's dA2 = bf16(GELU(h))^T P2[:, r_s2:] recomputes GELU(h) from h (nothing
  * of the activation is stored).  Writes dX [M, K1] and the four adapter
  * gradients (fp32; accumulate = 1 adds).  FC1's dA1/dB1 run beside FC1's dX
@@ -324,8 +329,9 @@ FT_API int fourtune_mlp_bwd(const ft_linear_t* fc1, const ft_linear_t* fc2, cons
 
 /* The MLP calls with per-kernel CUDA events, as fourtune_linear_*_timed.  Kernels,
  * in order -- forward: 0 X pass, 1 FC1 GEMM with the GELU / Q(a) / L2 epilogue,
- * 2 FC2 GEMM; backward: 0 G pass (FC2), 1 FC2 dX GEMM with the GELU' / Q(d_h) / P1
- * epilogue, 2 FC2 dA/dB, 3 FC1 dA/dB, 4 FC1 dX GEMM. */
+ * 2 L2 reduction, 3 FC2 GEMM; backward: 0 G pass (FC2), 1 FC2 dX GEMM with the
+ * GELU' / Q(d_h) / P1 epilogue, 2 P1 reduction, 3 FC2 dA/dB, 4 FC1 dA/dB, 5 FC1
+ * dX GEMM. */
 FT_API int fourtune_mlp_fwd_timed(const ft_linear_t* fc1, const ft_linear_t* fc2, const ft_bf16* X, int64_t M,
                                   void* Y, int y_dtype, ft_bf16* h_saved, ft_bf16* L1_saved, ft_bf16* L2_saved,
                                   float* dbg_a, void* ws, size_t ws_bytes, void* stream, void* const* events,
