@@ -464,35 +464,39 @@ __device__ __forceinline__ void quantize_1block_f32(const float* v, float amax, 
 // through 0.5 (1 + tanh(u)) = 1 / (1 + e^{-2u}) =: s (no cancellation for very
 // negative h), so GELU(h) = h s.  Its derivative, with 1 - tanh(u)^2 = 4 s (1 - s)
 // and 1 - s = s e^{-2u}: GELU'(h) = s + 2 h s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 h^2).
-// The exponential and the quotient are the fast hardware forms (__expf,
-// __fdividef): for |u| <= 40 e^{-2u} is within ~5e-6 (relative), the relative
-// error of GELU(h) and of s.  Beyond that s is 0 or 1 to far below fp32
-// resolution of the result: u < -40 gives GELU = -0 and GELU' = 0 (true values
-// below 1e-32 in magnitude), u > 40 gives GELU = h and GELU' = 1 (exact in fp32);
-// both hold for any h, however large (h^3 may overflow to infinity).  The
-// limits are taken as selects, so a warp never branches on its values.
-constexpr float kGeluC = 0.7978845608028654f;  // sqrt(2/pi)
+// e^{-2u} = 2^(-2 log2(e) u) on the hardware base-2 exponential and s on the
+// hardware reciprocal (PTX ex2.approx / rcp.approx: relative errors near
+// 2^-22; with the rounding of the exponent's product, e^{-2u} is within ~6e-6
+// for |u| <= 44).  Their limits need no special cases: for u < -44.3 e^{-2u}
+// is +inf and s = 1/inf = +0, so GELU = h * 0 = -0 (true value below 3e-39 |h|);
+// for u > 44 e^{-2u} = 0, s = 1 and GELU = h (exact in fp32).  The derivative
+// takes GELU' = 0 for u < -40 and 1 for u > 40 (true values within 1e-32 of
+// those), as selects, so that s (1 - s) = s * s e^{-2u} is never inf * 0.
+constexpr float kGeluC = 0.7978845608028654f;   // sqrt(2/pi)
 constexpr float kGeluK = 0.044715f;
-// s = 0.5 (1 + tanh u) with the limits taken as selects (no branches)
-__device__ __forceinline__ float gelu_s(float u, float* e_out) {
-  const float uc = fminf(fmaxf(u, -40.0f), 40.0f);
-  const float e = __expf(-2.0f * uc);
-  float s = __fdividef(1.0f, 1.0f + e);
-  s = u < -40.0f ? 0.0f : s;
-  s = u > 40.0f ? 1.0f : s;
-  *e_out = e;
-  return s;
+constexpr float kGeluM2Log2e = -2.8853900817779268f;   // -2 log2(e)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// u = sqrt(2/pi) (h + 0.044715 h^3)
+__device__ __forceinline__ float gelu_u(float h) { return h * fmaf(kGeluC * kGeluK, h * h, kGeluC); }
 __device__ __forceinline__ float gelu_tanh(float h) {
-  float e;
-  return h * gelu_s(kGeluC * (h + kGeluK * h * h * h), &e);
+  const float e = ex2_approx(kGeluM2Log2e * gelu_u(h));
+  return h * rcp_approx(1.0f + e);
 }
 __device__ __forceinline__ void gelu_tanh_and_grad(float h, float* g, float* dg) {
-  const float u = kGeluC * (h + kGeluK * h * h * h);
-  float e;
-  const float s = gelu_s(u, &e);
+  const float u = gelu_u(h);
+  const float e = ex2_approx(kGeluM2Log2e * u);
+  const float s = rcp_approx(1.0f + e);
   *g = h * s;
-  const float d = s + 2.0f * h * s * (e * s) * kGeluC * (1.0f + 3.0f * kGeluK * h * h);
+  const float d = fmaf(2.0f * h * s * (e * s), kGeluC * fmaf(3.0f * kGeluK, h * h, 1.0f), s);
   *dg = u > 40.0f ? 1.0f : (u < -40.0f ? 0.0f : d);
 }
 
