@@ -93,7 +93,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-template <int BN>
+// SCALED: the 1x16 layout's product scale 2^(eA + eB) in the epilogue (its own
+// instantiation, so that the block layout's accumulator readout -- on the
+// next tile's critical path -- carries no extra multiply)
+template <int BN, bool SCALED>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     // when it is a float32 number, else as two (then f1 is exact and the
     // product's own range is exceeded anyway)
     float f1 = 1.0f, f2 = 1.0f;
-    if (p.amax_a) {
+    if (SCALED) {
       const int es = group16_exponent(__uint_as_float(*p.amax_a)) + group16_exponent(__uint_as_float(*p.amax_b));
       if (es >= -126 && es <= 127) {
         f1 = pow2_f32(es);
@@ -371,9 +374,13 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             for (int e = 0; e < 8; ++e) {
               const uint4 b4 = bw[2 * k + e / 4];
               const uint32_t bb = (e & 3) == 0 ? b4.x : (e & 3) == 1 ? b4.y : (e & 3) == 2 ? b4.z : b4.w;
-              pk[16 * rd + 8 * k + e] =
-                  pack_bf16x2(fmaf(__uint_as_float(v[k][2 * e]) * f1, f2, bf16_bits_to_f32(bb & 0xFFFFu)),
-                              fmaf(__uint_as_float(v[k][2 * e + 1]) * f1, f2, bf16_bits_to_f32(bb >> 16)));
+              float x0 = __uint_as_float(v[k][2 * e]), x1 = __uint_as_float(v[k][2 * e + 1]);
+              if (SCALED) {
+                x0 *= f1;
+                x1 *= f1;
+              }
+              pk[16 * rd + 8 * k + e] = pack_bf16x2(fmaf(x0, f2, bf16_bits_to_f32(bb & 0xFFFFu)),
+                                                    fmaf(x1, f2, bf16_bits_to_f32(bb >> 16)));
             }
           }
         }
@@ -405,8 +412,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             uint32_t w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              w[e] = __float_as_uint(fmaf(__uint_as_float(v[8 * hlf + e]) * f1, f2,
-                                          bias ? __bfloat162float(bias[nb + e]) : 0.0f));
+              w[e] = __float_as_uint(fmaf(SCALED ? __uint_as_float(v[8 * hlf + e]) * f1 : __uint_as_float(v[8 * hlf + e]),
+                                          f2, bias ? __bfloat162float(bias[nb + e]) : 0.0f));
             store_rows32(buf, w, lane, out_rows + static_cast<long long>(nb) * 4, ldb, rows_left);
           }
         }
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int BN = kGemmBN;
-  auto kernel = gemm_fp4_kernel<BN>;
+  auto kernel = p.amax_a ? gemm_fp4_kernel<BN, true> : gemm_fp4_kernel<BN, false>;
   const uint32_t smem = GemmLayout<BN>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
