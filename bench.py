@@ -424,8 +424,13 @@ def run_ours(args, rank, world, local_rank):
                          "note": "value = the median of back-to-back timed blocks of exactly K steps"},
     }
     if world == 1 and not args.no_extra:
+        names = [n for n in args.extra.split(",") if n]
+        bad = [n for n in names if n not in EXTRA_WORKLOADS]
+        if bad:
+            raise SystemExit(f"unknown --extra workload(s) {bad}; choose from {EXTRA_WORKLOADS}")
         line["configs_extra"] = measure_extra(ft, synth, dev, flush, peaks, steps=max(3, min(args.steps, 10)),
-                                              warmup=max(1, min(args.warmup, 3)))
+                                              warmup=max(1, min(args.warmup, 3)), names=names)
+    if world == 1 and not args.no_extra and not args.no_variants:
         v = measure_variants(ft, synth, dev, flush, steps=max(3, min(args.steps, 10)), warmup=max(1, min(args.warmup, 3)))
         ours_ms = total_ms / args.steps
         for rec in v["variants"].values():
@@ -448,7 +453,7 @@ def run_ours(args, rank, world, local_rank):
 EXTRA_WORKLOADS = ("flux-mlp-3072", "flux-single-stream", "video-mlp-5120")
 
 
-def measure_extra(ft, synth, dev, flush, peaks, steps, warmup):
+def measure_extra(ft, synth, dev, flush, peaks, steps, warmup, names=EXTRA_WORKLOADS):
     """The other workloads (MLP pair, single-stream block linears, video MLP): device
     time of fwd+bwd steps (L2 flushed before each, no events inside), then one step
     with an event pair around every kernel for the breakdown."""
@@ -456,7 +461,7 @@ def measure_extra(ft, synth, dev, flush, peaks, steps, warmup):
     up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16)
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     out = {}
-    for name in EXTRA_WORKLOADS:
+    for name in names:
         wl = synth.WORKLOADS[name]
         M = wl.M
         layers = []
@@ -682,6 +687,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' timings")
+    ap.add_argument("--extra", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated subset of the other workloads to time (default: all)")
+    ap.add_argument("--no-variants", action="store_true", help="skip the ablation variants' timings")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
