@@ -128,6 +128,10 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
 }
 
 // ------------------------------------------------------------------ TMA
+// pull the 128-byte line holding p into L2 (no registers, no completion)
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -531,6 +531,11 @@ __global__ void __maxnreg__(kMlMaxReg)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);   // the next tile's MMAs may start
+        // EPI 2: the next tile of the unit reads this lane's row of h 256 columns
+        // on; pull its line into L2 now, so that the prefetch into registers at
+        // the top of the next tile does not wait on HBM
+        if (EPI == 2 && nt + 1 < nhi && row_ok && n0 + kMlBN < p.N)
+          prefetch_l2(static_cast<const __nv_bfloat16*>(mp.h) + static_cast<long long>(row) * p.N + n0 + kMlBN);
         // h / d_h to global memory from T: the warp's 32 rows x 128 bytes, four
         // whole rows (512 contiguous-by-row bytes) per store
 #pragma unroll 2
