@@ -129,7 +129,8 @@ class ClockSampler:
 def oracle_step(p, Rc, Rs, X, dY):
     from oracle import layer as olayer
     f = olayer.linear_fwd(X, Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"], p.get("bias"))
-    olayer.linear_bwd(dY, X, f["L"], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"])
+    b = olayer.linear_bwd(dY, X, f["L"], Rc, Rs, p["S_dn"], p["S_up"], p["A"], p["B"])
+    return f, b
 
 
 def cpu_cores():
@@ -152,14 +153,29 @@ def oracle_inputs(rows):
 
 
 def time_oracle(rows, repeats=1):
+    """Times the CPU oracle on the first `rows` tokens; returns (times, FLOPs, outputs)."""
     wl, spec, p, Rc, Rs, X, dY = oracle_inputs(rows)
     times = []
+    out = None
     for _ in range(repeats):
         t0 = time.perf_counter()
-        oracle_step(p, Rc, Rs, X, dY)
+        out = oracle_step(p, Rc, Rs, X, dY)
         times.append(time.perf_counter() - t0)
     fp4, lr = layer_work(rows, spec.K, spec.N, spec.r_s, spec.r)
-    return times, (fp4 + lr)
+    return times, (fp4 + lr), out
+
+
+def parity_record(ref, Y, dX, dA, dB):
+    """The timed configuration's own outputs (bf16 y and dX, fp32 dA and dB of the
+    last step) against the oracle's on the same inputs: max-normwise error
+    max|g - r| / max|r| per output (the bf16 outputs carry their own rounding,
+    up to 2^-9 of an element)."""
+    f, b = ref
+    host = lambda t: t.float().cpu().numpy().astype(np.float64)
+    nw = lambda g, r: float(np.abs(g - r).max() / np.abs(r).max())
+    return {"y_bf16": nw(host(Y), f["y"]), "dX_bf16": nw(host(dX), b["dX"]), "dA": nw(host(dA), b["dA"]),
+            "dB": nw(host(dB), b["dB"]),
+            "note": "max-normwise error of the bench's own outputs vs the CPU oracle on the whole workload"}
 
 
 def run_reference(args, rank, world):
@@ -439,8 +455,9 @@ def run_ours(args, rank, world, local_rank):
                      "(ms_per_step); the bf16 LoRA layer has no stabilizer (rank-32 adapter only)")
         line["variants"] = v
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, flop_s = time_oracle(M, repeats=1)
+        times, flop_s, ref = time_oracle(M, repeats=1)
         t = min(times)
+        line["parity"] = parity_record(ref, Y, dX, dA, dB)
         line["cpu_baseline"] = {"value": flop_s / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
                                 "kind": "oracle",
                                 "sample": f"one full fwd+bwd of the workload ({M} tokens, K=N={K}), {t:.1f} s"}
