@@ -128,6 +128,17 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
 }
 
 // ------------------------------------------------------------------ TMA
+// Split-K counter: returns the old value.  acq_rel at gpu scope: the release
+// half publishes every write ordered before this thread's atomic (the CTA's
+// partial, through the CTA barrier that precedes it); the acquire half orders
+// the reads that follow (through the next CTA barrier, the last CTA's loads of
+// the other CTAs' partials) after every earlier increment's release.  One
+// atomic in place of fence, atomic, fence.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 // pull the 128-byte line holding p into L2 (no registers, no completion)
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));

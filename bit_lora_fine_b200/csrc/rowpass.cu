@@ -269,15 +269,13 @@ __global__ void __launch_bounds__(kRpThreads, 1)
         }
         if (p.nsplit > 1) {
           // the last CTA of this row tile to finish sums every split's partial, in
-          // split order.  One thread publishes the CTA's partial writes (ordered
-          // before it by the barrier) with a gpu-scope fence before its counter
-          // increment; the last CTA's fence after reading the counter orders the
-          // partial reads after every other CTA's increment.
+          // split order.  One thread's acq_rel counter increment publishes the
+          // CTA's partial writes (ordered before it by the barrier) and, in the
+          // last CTA, orders the partial reads (after the next barrier) after
+          // every other CTA's increment.
           named_bar_sync(1, 32 * kRpQuantWarps);
           if (threadIdx.x == 128) {
-            __threadfence();
-            const int prev = atomicAdd(&p.counters[blockIdx.x], 1);
-            __threadfence();
+            const int prev = atomic_add_acq_rel_gpu(&p.counters[blockIdx.x], 1);
             *s_last = (prev == p.nsplit - 1);
           }
           named_bar_sync(1, 32 * kRpQuantWarps);

@@ -189,14 +189,12 @@ __global__ void __launch_bounds__(kTgThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             if (e < nq) dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-          // one thread publishes the CTA's partial (ordered before it by the
-          // barrier) with a gpu-scope fence before the counter increment; the last
-          // CTA's fence after the increment orders its partial reads after all others
+          // one thread's acq_rel counter increment publishes the CTA's partial
+          // (ordered before it by the barrier) and, in the last CTA, orders its
+          // partial reads (after the next barrier) after all other increments
           named_bar_sync(1, 128);
           if (threadIdx.x == 128) {
-            __threadfence();
-            const int prev = atomicAdd(&p.counters[ptile], 1);
-            __threadfence();
+            const int prev = atomic_add_acq_rel_gpu(&p.counters[ptile], 1);
             *s_last = (prev == p.nsplit - 1);
           }
           named_bar_sync(1, 128);
