@@ -13,31 +13,32 @@
 // Persistent kernel: one CTA per SM walks the 128 x BN output tiles (BN = 256)
 // in row-major tile order, so that the CTAs of one wave share the rows of A and
 // all of B in L2.  One pipeline stage = one K-block of 256 FP4 elements: the A
-// and B code boxes (128-byte swizzled rows).  Both operands' scales, kept in
-// global memory in the MMA-ready layout (kernels.h), must sit in TMEM when
-// the MMAs run: the MMA reads A's scales of lane quadrant w from column
-// base + w of that quadrant, and B's scales from all four columns of every
-// quadrant, so B's scales are needed four times over.  Moving them with
+// and B code boxes (128-byte swizzled rows) and the K-block's scale blocks of
+// both operands, kept in global memory in the MMA-ready layout (kernels.h) and
+// brought into the stage by bulk copies beside the code boxes.  The scales must
+// sit in TMEM when the MMAs run: the MMA reads A's scales of lane quadrant w
+// from column base + w of that quadrant, and B's scales from all four columns
+// of every quadrant, so B's scales are needed four times over.  Moving them with
 // tcgen05.cp 32x128b.warpx4 (which replicates into the four quadrants) costs
 // ~70 cycles a copy, 12 copies per K-block, on the same queue as the MMAs --
 // more than the 4 MMAs of the K-block take.  Instead four scale warps, one per
-// lane quadrant, load each K-block's scale words from global memory (L2) into
-// registers and write them into their quadrant with tcgen05.st, which runs
-// beside the MMAs.
+// lane quadrant, read each stage's scale words from shared memory once the
+// stage has landed and write them into their quadrant with tcgen05.st, which
+// runs beside the MMAs.  (Loading the words from global memory one stage ahead
+// instead, in registers, left the MMAs waiting on scale loads: 41.5 / 43.4 us
+// against 39.4 / 39.3 us at FLUX width.)
 // Warp roles:
-//   warp 0 lane 0  producer: TMA code boxes per K-block; then the bf16
-//                  low-rank blocks A2
-//                  [128 x 64] and B2 (K-major [BN x 64] or MN-major [64 x BN]
-//                  in four boxes)
+//   warp 0 lane 0  producer: TMA code boxes and scale bulk copies per K-block;
+//                  then the bf16 low-rank blocks A2 [128 x 64] and B2 (K-major
+//                  [BN x 64] or MN-major [64 x BN] in four boxes)
 //   warp 1         TMEM owner; lane 0 issues
 //                  tcgen05.mma kind::mxf4nvf4.block_scale.block16 (M=128,
 //                  N=BN, K=64) once a stage's codes and scales are in, then
 //                  kind::f16 for the low-rank blocks
-//   warps 12..15   scale warps: warp 12+q fills
-//                  quadrant q's scale columns of each stage, one stage ahead
-//                  in registers; a stage's columns are rewritten only after
-//                  the MMAs that read them have completed (the stage's
-//                  empty barrier)
+//   warps 12..15   scale warps: warp 12+q fills quadrant q's scale columns of
+//                  each stage from the stage's scale blocks once the stage has
+//                  landed (its full barrier, which also means the MMAs that
+//                  read the columns' previous contents have completed)
 //   warps 4..11    epilogue, warp w on TMEM lanes 32 (w % 4).. and half of the
 //                  columns.  bf16 output: the warp's accumulator slice goes to
 //                  registers (+ bias, packed to bf16), the accumulator is
@@ -58,7 +59,9 @@ struct GemmLayout {
   static constexpr int kNC = BN / 128;                       // 128-row scale chunks of the B tile
   static constexpr uint32_t kA = 128 * 128;                  // A codes / A2 bf16 tile
   static constexpr uint32_t kB = BN * 128;                   // B codes / B2 bf16 tile
-  static constexpr uint32_t kStage = kA + kB;                // multiple of 1024
+  static constexpr uint32_t kSFA = 4 * 512;                 // A's scale blocks of a K-block
+  static constexpr uint32_t kSFB = kNC * 4 * 512;           // B's: [128-row chunk][k-step][512 B]
+  static constexpr uint32_t kStage = kA + kB + kSFA + kSFB;  // multiple of 1024
   static constexpr uint32_t kEpi = 8 * 1024;                 // one transpose buffer per epilogue warp
   static constexpr uint32_t kSmem = 1024 + kGmStages * kStage + kEpi + 256;
   // TMEM columns: accumulator, then per stage 16 (SFA) + 16*kNC (SFB)
@@ -176,9 +179,22 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           }
           uint8_t* st = smem + s * Lay::kStage;
           if (i < KB) {
-            mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
             // a K-block is 128 bytes of each row: 256 FP4 codes or 64 bf16 values
             const int kx = bf16main ? i * 64 : i * 128;
+            if (bf16main) {
+              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB);
+            } else {
+              // the K-block's MMA-ready scale blocks ride in the stage (bulk copies)
+              const int nks = min(4, KS - 4 * i);
+              const uint32_t sfbytes = static_cast<uint32_t>(nks) * 512u;
+              const int nb = (n0 / 128 + 1 < nchunk_b) ? 2 : 1;
+              mbar_arrive_expect_tx(&full[s], Lay::kA + Lay::kB + sfbytes * static_cast<uint32_t>(1 + nb));
+              bulk_load(st + Lay::kA + Lay::kB, p.sfa + (static_cast<size_t>(m0 / 128) * KS + 4 * i) * 512, sfbytes,
+                        &full[s]);
+              for (int c = 0; c < nb; ++c)
+                bulk_load(st + Lay::kA + Lay::kB + Lay::kSFA + c * 2048,
+                          p.sfb + (static_cast<size_t>(n0 / 128 + c) * KS + 4 * i) * 512, sfbytes, &full[s]);
+            }
             tma_load_2d(st, &tmA, &full[s], kx, m0);
             tma_load_2d(st + Lay::kA, &tmB, &full[s], kx, n0);
           } else {
@@ -261,63 +277,46 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int bx = static_cast<int>(blockIdx.x), gx = static_cast<int>(gridDim.x);
     const int G = (bx < tiles ? (tiles - 1 - bx) / gx + 1 : 0) * T;
     constexpr int NB = 4 * 4 * Lay::kNC;
-    auto fetch = [&](int gg, uint32_t (&a)[4], uint32_t (&b)[NB]) {
-      const int tile = bx + (gg / T) * gx;
-      const int i = gg % T;
-      const int nks = (i < KB && !bf16main) ? min(4, KS - 4 * i) : 0;
-      const int mc = tile / tiles_n, nc = (tile % tiles_n) * Lay::kNC;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        a[t] = 0u;
-        if (t < nks)
-          a[t] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa + (static_cast<size_t>(mc) * KS + 4 * i + t) * 512 +
-                                                         16 * lane + 4 * q));
-      }
-#pragma unroll
-      for (int c = 0; c < Lay::kNC; ++c) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          uint4 x = make_uint4(0u, 0u, 0u, 0u);   // zero scales past N (their codes are zero)
-          if (t < nks && nc + c < nchunk_b)
-            x = __ldg(reinterpret_cast<const uint4*>(p.sfb + (static_cast<size_t>(nc + c) * KS + 4 * i + t) * 512 +
-                                                     16 * lane));
-          b[4 * (t * Lay::kNC + c)] = x.x;
-          b[4 * (t * Lay::kNC + c) + 1] = x.y;
-          b[4 * (t * Lay::kNC + c) + 2] = x.z;
-          b[4 * (t * Lay::kNC + c) + 3] = x.w;
-        }
-      }
-    };
-    auto put = [&](int gg, const uint32_t (&a)[4], const uint32_t (&b)[NB]) -> bool {
+    // each stage's scale blocks, from the stage once its copies have landed
+    // (full[s] of this use implies the MMAs of the slot's previous use are done)
+    for (int gg = 0; gg < G; ++gg) {
       const int s = gg % kGmStages;
       const uint32_t ph = (gg / kGmStages) & 1;
       bool okw = true;
-      if (lane == 0) okw = mbar_wait(&empty[s], ph ^ 1, p.status, abortp);   // MMAs that read the slot are done
-      okw = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
-      if (!okw) return false;
-      tc_fence_after();
-      if (gg % T < KB && !bf16main) {
-        const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
-        uint32_t a16[16];
+      if (lane == 0) okw = mbar_wait(&full[s], ph, p.status, abortp);
+      if (__shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) == 0) break;
+      const int i = gg % T;
+      if (i < KB && !bf16main) {
+        const int tile = bx + (gg / T) * gx;
+        const int nks = min(4, KS - 4 * i);
+        const int nc = (tile % tiles_n) * Lay::kNC;
+        const uint8_t* sf = smem + s * Lay::kStage + Lay::kA + Lay::kB;
+        uint32_t b[NB];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a16[e] = a[e >> 2];
-        tmem_st_32x32b_x16(trow + sf_col, a16);
+        for (int c = 0; c < Lay::kNC; ++c) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);   // zero scales past N (their codes are zero)
+            if (t < nks && nc + c < nchunk_b)
+              x = *reinterpret_cast<const uint4*>(sf + Lay::kSFA + c * 2048 + t * 512 + 16 * lane);
+            b[4 * (t * Lay::kNC + c)] = x.x;
+            b[4 * (t * Lay::kNC + c) + 1] = x.y;
+            b[4 * (t * Lay::kNC + c) + 2] = x.z;
+            b[4 * (t * Lay::kNC + c) + 3] = x.w;
+          }
+        }
+        tc_fence_after();
+        const uint32_t sf_col = BN + s * Lay::kSfColsPerStage;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          tmem_st_32x32b_x4_rep(trow + sf_col + 4 * t,
+                                t < nks ? *reinterpret_cast<const uint32_t*>(sf + t * 512 + 16 * lane + 4 * q) : 0u);
         tmem_st_32x32b_x32(trow + sf_col + 16, b);
         tmem_st_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sf_full[s]);
-      return true;
-    };
-    // two register sets: stage gg+1's loads are in flight while stage gg is stored
-    uint32_t a0[4], b0[NB], a1[4], b1[NB];
-    if (G > 0) fetch(0, a0, b0);
-    for (int gg = 0; gg < G; gg += 2) {
-      if (gg + 1 < G) fetch(gg + 1, a1, b1);
-      if (!put(gg, a0, b0) || gg + 1 >= G) break;
-      if (gg + 2 < G) fetch(gg + 2, a0, b0);
-      if (!put(gg + 1, a1, b1)) break;
     }
   } else if (warp >= 4) {
     // two warps per TMEM lane quadrant, each owning half of the tile's columns
