@@ -181,14 +181,20 @@ size_t grad_counter_words(const ft_linear_t* L) { return cdiv(L->K, 128) + cdiv(
 // rest: split in proportion to the two kernels' work at the per-SM rates
 // measured on this part when they share the GPU (FP4 GEMM ~14 TFLOP/s, dA/dB
 // ~44 GB/s of X and G per SM -- both are paced per SM by TMA latency, not by
-// the GPU-wide L2 or HBM bandwidth); even, 8 .. half of the SMs.  0 (run them
-// one after the other) on parts with fewer than 16 SMs.
+// the GPU-wide L2 or HBM bandwidth).  The GEMM's time goes in whole waves of
+// output tiles, so it keeps the fewest SMs that give it the same number of
+// waves and dA/dB take the rest; even, 8 .. half of the SMs.  0 (run them one
+// after the other) on parts with fewer than 16 SMs.
 int grad_side_sms(const ft_linear_t* L, int64_t M, int num_sms) {
   if (num_sms < 16) return 0;
   const double t_gemm = 2.0 * static_cast<double>(M) * L->N * L->K / 14.0e12;
   const double t_grad = 2.0 * static_cast<double>(M) * static_cast<double>(L->K + L->N) / 44.0e9;
   int n = static_cast<int>(std::lround(num_sms * t_grad / (t_grad + t_gemm)));
   n = std::max(8, std::min(num_sms / 2, n));
+  const int64_t tiles = static_cast<int64_t>(cdiv(L->K, ft::kGemmBN)) * cdiv(M, ft::kGemmBM);   // dX output tiles
+  const int64_t waves = cdiv(tiles, num_sms - n);
+  n = std::max(n, num_sms - static_cast<int>(cdiv(tiles, waves)));
+  n = std::min(num_sms / 2, n);
   return n & ~1;
 }
 // Serial: dA reads X from HBM; dB reads G, which the G pass has just streamed

@@ -135,9 +135,6 @@ int rowpass_stages(int R, int w_mn_major);
 // persistent: min(tiles, num_sms) CTAs
 cudaError_t launch_gemm_fp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                             const CUtensorMap& tmB2, const GemmParams& p, int num_sms, cudaStream_t stream);
-// compact block16 scales -> MMA-ready layout of the operand [rows, cols]; with
-// `transposed`, the operand is the transpose of the quantized matrix, whose
-// compact scales are [cols/16, rows/16]
 // zero `bytes` (a multiple of 16, 16-aligned) at p after the previous kernel, in a
 // dependent launch (see quant.cu)
 cudaError_t launch_clear_words(void* p, size_t bytes, cudaStream_t stream);
@@ -151,6 +148,9 @@ cudaError_t launch_quantize_group16(const void* w, int rows, int cols, int trans
                                     uint8_t* codes, uint8_t* scales, uint8_t* sf_mma, cudaStream_t stream);
 cudaError_t launch_scale_pow2(const void* src, void* dst, long long n, const uint32_t* amax_a, const uint32_t* amax_b,
                               int num_sms, cudaStream_t stream);
+// compact block16 scales -> MMA-ready layout of the operand [rows, cols]; with
+// `transposed`, the operand is the transpose of the quantized matrix, whose
+// compact scales are [cols/16, rows/16]
 cudaError_t launch_sf_mma(const uint8_t* scales, int rows, int cols, int transposed, uint8_t* out,
                           cudaStream_t stream);
 cudaError_t launch_tgrad2(const CUtensorMap& tmT0, const CUtensorMap& tmV0, const TgradParams& p0,
