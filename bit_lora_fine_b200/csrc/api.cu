@@ -192,8 +192,9 @@ int grad_side_sms(const ft_linear_t* L, int64_t M, int num_sms) {
   int n = static_cast<int>(std::lround(num_sms * t_grad / (t_grad + t_gemm)));
   n = std::max(8, std::min(num_sms / 2, n));
   const int64_t tiles = static_cast<int64_t>(cdiv(L->K, ft::kGemmBN)) * cdiv(M, ft::kGemmBM);   // dX output tiles
-  const int64_t waves = cdiv(tiles, num_sms - n);
-  n = std::max(n, num_sms - static_cast<int>(cdiv(tiles, waves)));
+  const int64_t waves = (tiles + (num_sms - n) - 1) / (num_sms - n);
+  const int64_t keep = (tiles + waves - 1) / waves;   // fewest SMs with that many waves (<= num_sms - n)
+  n = std::max(n, num_sms - static_cast<int>(keep));
   n = std::min(num_sms / 2, n);
   return n & ~1;
 }
